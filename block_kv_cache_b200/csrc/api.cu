@@ -1,0 +1,279 @@
+// C-ABI entry points of the Fast-dLLM step library: argument validation,
+// device selection, workspace checks and dispatch to the kernels. See
+// include/fdllm.h for the contract of every function.
+#include "../../include/fdllm.h"
+#include "launch.h"
+#include "common.cuh"
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+struct fdl_ctx {
+    int device;
+    int sm_count;
+    int* d_err;              // device error word (4 bytes)
+};
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+    return fail(FDL_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Make ctx->device current for the duration of a call; restore afterwards.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) { ok = false; return; }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_attn(const fdl_attn_desc* d) {
+    if (!d) return fail(FDL_EINVAL, "attention: desc is NULL");
+    if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->seq_len < 1)
+        return fail(FDL_EINVAL, "attention: batch, heads and seq_len must be >= 1");
+    if (d->n_q_heads % d->n_kv_heads)
+        return fail(FDL_EINVAL, "attention: n_q_heads (%d) must be a multiple of n_kv_heads (%d)",
+                    d->n_q_heads, d->n_kv_heads);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(FDL_EUNSUPPORTED, "attention: head_dim %d not supported (64 or 128)",
+                    d->head_dim);
+    if (d->block_len < 1 || d->block_len > 128)
+        return fail(FDL_EINVAL, "attention: block_len %d outside [1, 128]", d->block_len);
+    if (d->block_start < 0 || d->block_start + d->block_len > d->seq_len)
+        return fail(FDL_EINVAL, "attention: block [%d, %d) outside [0, %d)", d->block_start,
+                    d->block_start + d->block_len, d->seq_len);
+    if (d->dtype != FDL_F32 && d->dtype != FDL_BF16)
+        return fail(FDL_EINVAL, "attention: unknown dtype %d", d->dtype);
+    if (!(d->scale >= 0.f) || isinf(d->scale))
+        return fail(FDL_EINVAL, "attention: scale must be finite and >= 0");
+    return FDL_OK;
+}
+
+fdl::AttnShape attn_shape(const fdl_attn_desc* d) {
+    fdl::AttnShape s{d->batch, d->n_q_heads, d->n_kv_heads, d->head_dim, d->seq_len,
+                     d->block_start, d->block_len, d->scale};
+    if (s.scale == 0.f) s.scale = 1.0f / sqrtf((float)d->head_dim);
+    return s;
+}
+
+int check_lm(const fdl_lmhead_desc* d) {
+    if (!d) return fail(FDL_EINVAL, "lmhead: desc is NULL");
+    if (d->rows < 1 || d->vocab < 2 || d->hidden < 64)
+        return fail(FDL_EINVAL, "lmhead: need rows >= 1, vocab >= 2, hidden >= 64");
+    if (d->hidden % 64)
+        return fail(FDL_EUNSUPPORTED, "lmhead: hidden %d must be a multiple of 64", d->hidden);
+    if (d->dtype != FDL_F32 && d->dtype != FDL_BF16)
+        return fail(FDL_EINVAL, "lmhead: unknown dtype %d", d->dtype);
+    return FDL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fdl_abi_version(void) { return FDL_ABI_VERSION; }
+
+const char* fdl_last_error(void) { return g_msg; }
+
+int fdl_create(fdl_ctx** out, int device) {
+    if (!out) return fail(FDL_EINVAL, "fdl_create: out is NULL");
+    *out = nullptr;
+    int n = 0;
+    cudaError_t e = cudaGetDeviceCount(&n);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+    if (device < 0 || device >= n)
+        return fail(FDL_EINVAL, "fdl_create: device %d not in [0, %d)", device, n);
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, device);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10 || prop.minor != 0)
+        return fail(FDL_EUNSUPPORTED, "fdl_create: device %d is sm_%d%d; this library is built "
+                    "for sm_100a (B200)", device, prop.major, prop.minor);
+    DeviceGuard g(device);
+    if (!g.ok) return fail(FDL_ECUDA, "fdl_create: cannot select device %d", device);
+    fdl_ctx* c = new fdl_ctx;
+    c->device = device;
+    c->sm_count = prop.multiProcessorCount;
+    c->d_err = nullptr;
+    e = cudaMalloc(&c->d_err, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(int));
+    if (e != cudaSuccess) {
+        if (c->d_err) cudaFree(c->d_err);
+        delete c;
+        return cuda_fail(e, "fdl_create: error word");
+    }
+    *out = c;
+    return FDL_OK;
+}
+
+int fdl_destroy(fdl_ctx* ctx) {
+    if (!ctx) return FDL_OK;
+    DeviceGuard g(ctx->device);
+    if (ctx->d_err) cudaFree(ctx->d_err);
+    delete ctx;
+    return FDL_OK;
+}
+
+int fdl_get_device_status(fdl_ctx* ctx, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "fdl_get_device_status: ctx is NULL");
+    DeviceGuard g(ctx->device);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "fdl_get_device_status: sync");
+    int code = 0;
+    e = cudaMemcpy(&code, ctx->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "fdl_get_device_status: read");
+    if (code != 0) {
+        e = cudaMemset(ctx->d_err, 0, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e, "fdl_get_device_status: clear");
+    }
+    if (code == fdl::DEV_TIMEOUT) return fail(FDL_ETIMEOUT, "device: a bounded wait ran out");
+    if (code == fdl::DEV_NO_PROGRESS)
+        return fail(FDL_EDEVICE, "device: every candidate of a block had a NaN confidence");
+    if (code != 0) return fail(FDL_EDEVICE, "device: error code %d", code);
+    return FDL_OK;
+}
+
+size_t fdl_attention_workspace_bytes(const fdl_ctx* ctx, const fdl_attn_desc* desc) {
+    if (!ctx) { fail(FDL_EINVAL, "attention workspace: ctx is NULL"); return 0; }
+    if (check_attn(desc) != FDL_OK) return 0;
+    return fdl::attn_workspace_bytes(attn_shape(desc), ctx->sm_count);
+}
+
+int fdl_dualcache_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
+                            const void* k_cache, const void* v_cache, void* out, float* lse,
+                            void* ws, size_t ws_bytes, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "attention: ctx is NULL");
+    int rc = check_attn(desc);
+    if (rc) return rc;
+    if (!q || !k_cache || !v_cache || !out)
+        return fail(FDL_EINVAL, "attention: q, k_cache, v_cache and out must be non-NULL");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+        (lse && ((uintptr_t)lse & 3u)))
+        return fail(FDL_EINVAL, "attention: q/k_cache/v_cache/out must be 16-byte aligned");
+    fdl::AttnShape s = attn_shape(desc);
+    const size_t need = fdl::attn_workspace_bytes(s, ctx->sm_count);
+    if (!ws || ws_bytes < need || !aligned16(ws))
+        return fail(FDL_EWORKSPACE, "attention: workspace needs %zu bytes (16-byte aligned), "
+                    "got %zu", need, ws ? ws_bytes : (size_t)0);
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return fail(FDL_ECUDA, "attention: cannot select device");
+    cudaError_t e = desc->dtype == FDL_F32
+        ? fdl::launch_attention_f32(s, (const float*)q, (const float*)k_cache,
+                                    (const float*)v_cache, (float*)out, lse, ws, ctx->sm_count,
+                                    (cudaStream_t)stream)
+        : fdl::launch_attention_bf16(s, q, k_cache, v_cache, out, lse, ws, ctx->sm_count,
+                                     (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return FDL_OK;
+}
+
+int fdl_kv_store(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* k_new, const void* v_new,
+                 int start, int n, void* k_cache, void* v_cache, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "kv_store: ctx is NULL");
+    if (!desc) return fail(FDL_EINVAL, "kv_store: desc is NULL");
+    if (desc->batch < 1 || desc->n_kv_heads < 1 || desc->seq_len < 1)
+        return fail(FDL_EINVAL, "kv_store: batch, n_kv_heads and seq_len must be >= 1");
+    if (desc->head_dim != 64 && desc->head_dim != 128)
+        return fail(FDL_EUNSUPPORTED, "kv_store: head_dim %d not supported", desc->head_dim);
+    if (desc->dtype != FDL_F32 && desc->dtype != FDL_BF16)
+        return fail(FDL_EINVAL, "kv_store: unknown dtype %d", desc->dtype);
+    if (n < 1 || start < 0 || start + n > desc->seq_len)
+        return fail(FDL_EINVAL, "kv_store: rows [%d, %d) outside [0, %d)", start, start + n,
+                    desc->seq_len);
+    if (!k_new || !v_new || !k_cache || !v_cache)
+        return fail(FDL_EINVAL, "kv_store: NULL buffer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return fail(FDL_EINVAL, "kv_store: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return fail(FDL_ECUDA, "kv_store: cannot select device");
+    const int eb = desc->dtype == FDL_F32 ? 4 : 2;
+    cudaError_t e = fdl::launch_kv_store(desc->batch, desc->n_kv_heads, desc->head_dim,
+                                         desc->seq_len, eb, k_new, v_new, start, n, k_cache,
+                                         v_cache, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_store launch");
+    return FDL_OK;
+}
+
+size_t fdl_lmhead_workspace_bytes(const fdl_ctx* ctx, const fdl_lmhead_desc* desc) {
+    if (!ctx) { fail(FDL_EINVAL, "lmhead workspace: ctx is NULL"); return 0; }
+    if (check_lm(desc) != FDL_OK) return 0;
+    fdl::LMShape s{desc->rows, desc->hidden, desc->vocab};
+    return fdl::lmhead_workspace_bytes(s);
+}
+
+int fdl_lmhead_confidence(fdl_ctx* ctx, const fdl_lmhead_desc* desc, const void* h,
+                          const void* w, const int32_t* bias_tok, const float* bias_val,
+                          float* conf, int32_t* tok, void* ws, size_t ws_bytes, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "lmhead: ctx is NULL");
+    int rc = check_lm(desc);
+    if (rc) return rc;
+    if (!h || !w || !conf || !tok) return fail(FDL_EINVAL, "lmhead: NULL buffer");
+    if ((bias_tok == nullptr) != (bias_val == nullptr))
+        return fail(FDL_EINVAL, "lmhead: bias_tok and bias_val go together");
+    if (!aligned16(h) || !aligned16(w))
+        return fail(FDL_EINVAL, "lmhead: h and w must be 16-byte aligned");
+    fdl::LMShape s{desc->rows, desc->hidden, desc->vocab};
+    const size_t need = fdl::lmhead_workspace_bytes(s);
+    if (!ws || ws_bytes < need || !aligned16(ws))
+        return fail(FDL_EWORKSPACE, "lmhead: workspace needs %zu bytes (16-byte aligned), got %zu",
+                    need, ws ? ws_bytes : (size_t)0);
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return fail(FDL_ECUDA, "lmhead: cannot select device");
+    cudaError_t e = desc->dtype == FDL_F32
+        ? fdl::launch_lmhead_f32(s, (const float*)h, (const float*)w, bias_tok, bias_val, conf,
+                                 tok, ws, (cudaStream_t)stream)
+        : fdl::launch_lmhead_bf16(s, h, w, bias_tok, bias_val, conf, tok, ws, ctx->sm_count,
+                                  ctx->d_err, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "lmhead launch");
+    return FDL_OK;
+}
+
+int fdl_threshold_unmask(fdl_ctx* ctx, const fdl_unmask_desc* desc, const float* conf,
+                         const int32_t* tok, int32_t* x, uint8_t* masked, int32_t* remaining,
+                         int32_t* n_decoded, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "unmask: ctx is NULL");
+    if (!desc) return fail(FDL_EINVAL, "unmask: desc is NULL");
+    if (desc->batch < 1 || desc->seq_len < 1)
+        return fail(FDL_EINVAL, "unmask: batch and seq_len must be >= 1");
+    if (desc->block_len < 1 || desc->block_len > 1024)
+        return fail(FDL_EINVAL, "unmask: block_len %d outside [1, 1024]", desc->block_len);
+    if (desc->block_start < 0 || desc->block_start + desc->block_len > desc->seq_len)
+        return fail(FDL_EINVAL, "unmask: block [%d, %d) outside [0, %d)", desc->block_start,
+                    desc->block_start + desc->block_len, desc->seq_len);
+    if (!isfinite(desc->tau)) return fail(FDL_EINVAL, "unmask: tau must be finite");
+    if (!conf || !tok || !x || !masked || !remaining)
+        return fail(FDL_EINVAL, "unmask: NULL buffer");
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return fail(FDL_ECUDA, "unmask: cannot select device");
+    cudaError_t e = fdl::launch_threshold_unmask(desc->batch, desc->seq_len, desc->block_start,
+                                                 desc->block_len, desc->tau, conf, tok, x,
+                                                 masked, remaining, n_decoded, ctx->d_err,
+                                                 (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "unmask launch");
+    return FDL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,46 @@
+// Host-side launchers shared between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fdl {
+
+struct AttnShape {
+    int batch, n_q_heads, n_kv_heads, head_dim, seq_len, block_start, block_len;
+    float scale;  // resolved (never 0)
+};
+
+// split-KV partition used by the attention kernels
+int attn_num_splits(const AttnShape& s, int sm_count);
+size_t attn_workspace_bytes(const AttnShape& s, int sm_count);
+
+cudaError_t launch_attention_f32(const AttnShape& s, const float* q, const float* k,
+                                 const float* v, float* out, float* lse, void* ws,
+                                 int sm_count, cudaStream_t st);
+cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
+                                  const void* v, void* out, float* lse, void* ws,
+                                  int sm_count, cudaStream_t st);
+
+cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len,
+                            int elem_bytes, const void* k_new, const void* v_new,
+                            int start, int n, void* k_cache, void* v_cache,
+                            cudaStream_t st);
+
+struct LMShape { int rows, hidden, vocab; };
+size_t lmhead_workspace_bytes(const LMShape& s);
+cudaError_t launch_lmhead_f32(const LMShape& s, const float* h, const float* w,
+                              const int32_t* bias_tok, const float* bias_val,
+                              float* conf, int32_t* tok, void* ws, cudaStream_t st);
+cudaError_t launch_lmhead_bf16(const LMShape& s, const void* h, const void* w,
+                               const int32_t* bias_tok, const float* bias_val,
+                               float* conf, int32_t* tok, void* ws, int sm_count,
+                               int* dev_err, cudaStream_t st);
+
+cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
+                                    int block_len, float tau, const float* conf,
+                                    const int32_t* tok, int32_t* x, uint8_t* masked,
+                                    int32_t* remaining, int32_t* n_decoded,
+                                    int* dev_err, cudaStream_t st);
+
+}  // namespace fdl

@@ -1,0 +1,239 @@
+"""Python binding of libfdllm.so, the C-ABI library of the Fast-dLLM step.
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels. torch provides device memory (outputs and scratch are allocated as
+torch tensors) and the current CUDA stream. If the shared object is missing,
+every call raises: there is no fallback of any kind.
+
+Layouts follow include/fdllm.h:
+  q, out   [b, B, Hq, d]     k_cache, v_cache [b, Hkv, L, d]
+  h        [M, D]            w [V, D]
+  conf/tok [b, B]            x [b, L] int32, masked [b, L] uint8
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfdllm.so")
+
+FDL_OK, FDL_EINVAL, FDL_EUNSUPPORTED, FDL_ECUDA, FDL_ETIMEOUT, FDL_EWORKSPACE, FDL_EDEVICE = (
+    0, -1, -2, -3, -4, -5, -6)
+FDL_F32, FDL_BF16 = 0, 1
+
+EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
+           "fdl_get_device_status", "fdl_attention_workspace_bytes",
+           "fdl_dualcache_attention", "fdl_kv_store", "fdl_lmhead_workspace_bytes",
+           "fdl_lmhead_confidence", "fdl_threshold_unmask")
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("seq_len", ctypes.c_int), ("block_start", ctypes.c_int),
+                ("block_len", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+class LMHeadDesc(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("hidden", ctypes.c_int),
+                ("vocab", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class UnmaskDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seq_len", ctypes.c_int),
+                ("block_start", ctypes.c_int), ("block_len", ctypes.c_int),
+                ("tau", ctypes.c_float)]
+
+
+class FdlError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"fdllm error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libfdllm.so and declare its signatures (raises if not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m block_kv_cache_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.fdl_abi_version.restype = i
+    L.fdl_create.argtypes = [ctypes.POINTER(vp), i]
+    L.fdl_destroy.argtypes = [vp]
+    L.fdl_last_error.restype = ctypes.c_char_p
+    L.fdl_get_device_status.argtypes = [vp, vp]
+    L.fdl_attention_workspace_bytes.argtypes = [vp, ctypes.POINTER(AttnDesc)]
+    L.fdl_attention_workspace_bytes.restype = sz
+    L.fdl_dualcache_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp,
+                                          vp, sz, vp]
+    L.fdl_kv_store.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, i, i, vp, vp, vp]
+    L.fdl_lmhead_workspace_bytes.argtypes = [vp, ctypes.POINTER(LMHeadDesc)]
+    L.fdl_lmhead_workspace_bytes.restype = sz
+    L.fdl_lmhead_confidence.argtypes = [vp, ctypes.POINTER(LMHeadDesc), vp, vp, vp, vp, vp,
+                                        vp, vp, sz, vp]
+    L.fdl_threshold_unmask.argtypes = [vp, ctypes.POINTER(UnmaskDesc), vp, vp, vp, vp, vp,
+                                       vp, vp]
+    for name in EXPORTS:
+        getattr(L, name).restype = getattr(L, name).restype or i
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != FDL_OK:
+        raise FdlError(rc, load().fdl_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return FDL_F32
+    if t.dtype == torch.bfloat16:
+        return FDL_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Context:
+    """One library context on one CUDA device. Holds a torch-allocated scratch
+    buffer that grows to the largest workspace asked for."""
+
+    def __init__(self, device: int | None = None):
+        L = load()
+        self.device = torch.cuda.current_device() if device is None else int(device)
+        h = ctypes.c_void_p()
+        _check(L.fdl_create(ctypes.byref(h), self.device))
+        self._h = h
+        self._ws = None
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load().fdl_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- scratch ---------------------------------------------------------
+    def workspace(self, nbytes: int) -> torch.Tensor:
+        nbytes = max(int(nbytes), 16)
+        if self._ws is None or self._ws.numel() < nbytes:
+            self._ws = torch.empty(nbytes, dtype=torch.uint8, device=f"cuda:{self.device}")
+        return self._ws
+
+    def device_status(self, stream=None) -> int:
+        """Synchronise and raise FdlError if a kernel recorded a device error."""
+        _check(load().fdl_get_device_status(self._h, _stream(stream)))
+        return FDL_OK
+
+    # -- (a) attention ----------------------------------------------------
+    def attn_desc(self, q, k_cache, block_start, scale=0.0) -> AttnDesc:
+        b, B, Hq, d = q.shape
+        _, Hkv, L, _ = k_cache.shape
+        return AttnDesc(b, Hq, Hkv, d, L, int(block_start), B, _dtype_code(q), float(scale))
+
+    def attention_workspace_bytes(self, desc: AttnDesc) -> int:
+        return int(load().fdl_attention_workspace_bytes(self._h, ctypes.byref(desc)))
+
+    def dualcache_attention(self, q, k_cache, v_cache, block_start, *, out=None, lse=None,
+                            want_lse=False, scale=0.0, ws=None, stream=None):
+        for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+            _need(t, n, q.dtype, 4)
+        d = self.attn_desc(q, k_cache, block_start, scale)
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty((d.batch, d.n_q_heads, d.block_len), dtype=torch.float32,
+                              device=q.device)
+        need = self.attention_workspace_bytes(d)
+        if ws is None:
+            ws = self.workspace(need)
+        _check(load().fdl_dualcache_attention(self._h, ctypes.byref(d), _ptr(q), _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(ws),
+                                              ws.numel() * ws.element_size(), _stream(stream)))
+        return (out, lse) if (want_lse or lse is not None) else out
+
+    def kv_store(self, k_new, v_new, k_cache, v_cache, start, stream=None):
+        _need(k_new, "k_new", k_cache.dtype, 4)
+        _need(v_new, "v_new", k_cache.dtype, 4)
+        _need(k_cache, "k_cache", None, 4)
+        _need(v_cache, "v_cache", k_cache.dtype, 4)
+        b, Hkv, L, d = k_cache.shape
+        n = k_new.shape[1]
+        desc = AttnDesc(b, Hkv, Hkv, d, L, 0, 1, _dtype_code(k_cache), 0.0)
+        _check(load().fdl_kv_store(self._h, ctypes.byref(desc), _ptr(k_new), _ptr(v_new),
+                                   int(start), int(n), _ptr(k_cache), _ptr(v_cache),
+                                   _stream(stream)))
+
+    # -- (b) LM head + confidence ----------------------------------------
+    def lmhead_workspace_bytes(self, desc: LMHeadDesc) -> int:
+        return int(load().fdl_lmhead_workspace_bytes(self._h, ctypes.byref(desc)))
+
+    def lmhead_confidence(self, h, w, bias_tok=None, bias_val=None, *, conf=None, tok=None,
+                          ws=None, stream=None):
+        _need(h, "h", None, 2)
+        _need(w, "w", h.dtype, 2)
+        if bias_tok is not None:
+            _need(bias_tok, "bias_tok", torch.int32, 1)
+            _need(bias_val, "bias_val", torch.float32, 1)
+        M, D = h.shape
+        V = w.shape[0]
+        d = LMHeadDesc(M, D, V, _dtype_code(h))
+        if conf is None:
+            conf = torch.empty(M, dtype=torch.float32, device=h.device)
+        if tok is None:
+            tok = torch.empty(M, dtype=torch.int32, device=h.device)
+        if ws is None:
+            ws = self.workspace(self.lmhead_workspace_bytes(d))
+        _check(load().fdl_lmhead_confidence(self._h, ctypes.byref(d), _ptr(h), _ptr(w),
+                                            _ptr(bias_tok), _ptr(bias_val), _ptr(conf),
+                                            _ptr(tok), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)))
+        return conf, tok
+
+    # -- (b) threshold select + scatter -----------------------------------
+    def threshold_unmask(self, conf, tok, x, masked, block_start, tau, *, remaining=None,
+                         n_decoded=None, stream=None):
+        _need(conf, "conf", torch.float32, 2)
+        _need(tok, "tok", torch.int32, 2)
+        _need(x, "x", torch.int32, 2)
+        _need(masked, "masked", torch.uint8, 2)
+        b, L = x.shape
+        B = conf.shape[1]
+        if remaining is None:
+            remaining = torch.empty(b, dtype=torch.int32, device=x.device)
+        d = UnmaskDesc(b, L, int(block_start), B, float(tau))
+        _check(load().fdl_threshold_unmask(self._h, ctypes.byref(d), _ptr(conf), _ptr(tok),
+                                           _ptr(x), _ptr(masked), _ptr(remaining),
+                                           _ptr(n_decoded), _stream(stream)))
+        return remaining

@@ -19,6 +19,7 @@ these seeded draws stand in for them.
 """
 from __future__ import annotations
 
+import os
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -35,11 +36,10 @@ def rng(seed: int) -> np.random.Generator:
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:
-    """float32 -> bf16 bit patterns (uint16), round to nearest, ties to even."""
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) & 0xFFFF
+    """float32 -> bf16 bit patterns (uint16), round to nearest, ties to even.
+    Inputs are finite (the draws here never produce NaN)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
 
 
@@ -49,13 +49,33 @@ def bf16_value(bits: np.ndarray) -> np.ndarray:
     return u.view(np.float32)
 
 
-def _draw(g: np.random.Generator, shape, std: float, dtype: str) -> np.ndarray:
-    """Gaussian draw N(0, std^2), returned as float32 values exactly
-    representable in `dtype` ("f32" or "bf16")."""
-    a = (g.standard_normal(shape) * std).astype(np.float32)
+_CHUNK = 1 << 22
+
+
+def _fill(seed, n, std, dtype):
+    a = rng(int(seed)).standard_normal(n, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
     if dtype == "bf16":
         a = bf16_value(bf16_bits(a))
     return a
+
+
+def _draw(g: np.random.Generator, shape, std: float, dtype: str) -> np.ndarray:
+    """Gaussian draw N(0, std^2) as float32 values exactly representable in
+    `dtype` ("f32" or "bf16"). Large draws are split into fixed 4 Mi-element
+    chunks, each from its own PCG64 stream seeded by `g`, and filled on a
+    thread pool; the result depends only on `g`'s state and the shape."""
+    n = int(np.prod(shape))
+    nch = max(1, (n + _CHUNK - 1) // _CHUNK)
+    seeds = g.integers(0, 2**63 - 1, nch)
+    if nch == 1:
+        return _fill(seeds[0], n, std, dtype).reshape(shape)
+    from concurrent.futures import ThreadPoolExecutor
+    sizes = [min(_CHUNK, n - i * _CHUNK) for i in range(nch)]
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        parts = list(ex.map(lambda i: _fill(seeds[i], sizes[i], std, dtype), range(nch)))
+    return np.concatenate(parts).reshape(shape)
 
 
 # ---------------------------------------------------------------------------

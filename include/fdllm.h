@@ -1,0 +1,218 @@
+/*
+ * fdllm.h - C ABI of the B200 (sm_100a) Fast-dLLM block-decoding step.
+ *
+ * The library computes one decoding step of a masked diffusion LLM with the
+ * two techniques of "Fast-dLLM: Training-free Acceleration of Diffusion LLM
+ * by Enabling KV Cache and Parallel Decoding" (arXiv 2505.22618):
+ *   (a) DualCache block attention: the current block's queries attend,
+ *       without a causal mask, over [cached prefix K/V | fresh block K/V |
+ *       cached masked-suffix K/V]; the caches are rewritten when a block
+ *       completes;
+ *   (b) confidence-aware parallel unmasking: the LM head over the block's
+ *       rows is reduced on the fly to (confidence, token) per row, and every
+ *       masked position whose confidence exceeds a threshold is decoded.
+ *
+ * Conventions shared by every entry point
+ *  - All pointers named as device buffers are CUDA device pointers on the
+ *    context's device, owned by the caller. The library never allocates or
+ *    frees them; scratch memory is passed in by the caller (`ws`), sized by
+ *    the matching *_workspace_bytes query.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every compute
+ *    call is asynchronous on that stream: it returns after enqueueing.
+ *  - Return value: FDL_OK (0) or a negative fdl_status. Argument errors are
+ *    detected on the host before anything is enqueued, so nothing runs on an
+ *    error return. fdl_last_error() gives a message for the calling thread's
+ *    last failure. No C++ exception crosses this boundary.
+ *  - Faults found on the device (a bounded wait that ran out, a confidence
+ *    that is NaN for every candidate) never trap: the kernel records a code in
+ *    the context's device error word and finishes; fdl_get_device_status()
+ *    reports and clears it.
+ *  - Layouts are row-major with the last named dimension contiguous.
+ *    bf16 is IEEE bfloat16 (as torch.bfloat16); f32 is IEEE single.
+ */
+#ifndef FDLLM_H
+#define FDLLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FDL_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FDL_API __attribute__((visibility("default")))
+#else
+#define FDL_API
+#endif
+
+typedef enum {
+    FDL_OK = 0,
+    FDL_EINVAL = -1,        /* bad argument: null pointer, shape, alignment, value */
+    FDL_EUNSUPPORTED = -2,  /* valid but not implemented (e.g. head_dim 96) */
+    FDL_ECUDA = -3,         /* a CUDA runtime/driver call failed */
+    FDL_ETIMEOUT = -4,      /* device: a bounded wait ran out */
+    FDL_EWORKSPACE = -5,    /* ws is NULL or smaller than the query says */
+    FDL_EDEVICE = -6        /* device: the step could not make progress (all-NaN confidences) */
+} fdl_status;
+
+typedef enum { FDL_F32 = 0, FDL_BF16 = 1 } fdl_dtype;
+
+typedef struct fdl_ctx fdl_ctx;   /* opaque: device id, device error word, launch config */
+
+/* ABI version of the loaded library (FDL_ABI_VERSION it was built with). */
+FDL_API int fdl_abi_version(void);
+
+/* Create a context on CUDA device `device`. Allocates the 4-byte device error
+ * word (the only allocation the library makes, once, here) and reads the
+ * device's properties. Fails with FDL_EUNSUPPORTED unless the device is
+ * compute capability 10.0 (B200). *out is set to NULL on failure. */
+FDL_API int fdl_create(fdl_ctx** out, int device);
+
+/* Free the context and its error word. NULL is accepted. */
+FDL_API int fdl_destroy(fdl_ctx* ctx);
+
+/* Message for the calling thread's last non-OK return ("" if none). The
+ * pointer stays valid until the thread's next failing call. */
+FDL_API const char* fdl_last_error(void);
+
+/* Synchronise `stream`, read the device error word, clear it, and return
+ * FDL_OK, FDL_ETIMEOUT or FDL_EDEVICE accordingly. */
+FDL_API int fdl_get_device_status(fdl_ctx* ctx, void* stream);
+
+/* ------------------------------------------------------------------------
+ * (a) DualCache block attention
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int batch;        /* b  >= 1 sequences (all of length seq_len) */
+    int n_q_heads;    /* Hq >= 1 */
+    int n_kv_heads;   /* Hkv >= 1, Hq % Hkv == 0; q head h reads kv head h / (Hq/Hkv) */
+    int head_dim;     /* d in {64, 128} */
+    int seq_len;      /* L = prefix + block + suffix, >= 1 */
+    int block_start;  /* s, first position of the current block */
+    int block_len;    /* B, 1 <= B <= 128, s + B <= L */
+    int dtype;        /* fdl_dtype of q, caches and out; accumulation is f32 */
+    float scale;      /* softmax scale; 0 means 1/sqrt(head_dim) */
+} fdl_attn_desc;
+
+/* Bytes of scratch fdl_dualcache_attention needs for this shape on ctx's
+ * device (split-KV partial results; the split count follows the device's SM
+ * count). Returns 0 for an invalid context or descriptor. */
+FDL_API size_t fdl_attention_workspace_bytes(const fdl_ctx* ctx, const fdl_attn_desc* desc);
+
+/* DualCache block attention (Fast-dLLM: block-wise approximate KV cache,
+ * DualCache variant; aibase news "Innovations" 1, README "Key techniques" 1).
+ *
+ * For each sequence b, q-head h and block row i:
+ *   out[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . K[b,g,j,:]) V[b,g,j,:]
+ * over ALL j in [0, L) (bidirectional: no mask), g = h / (Hq/Hkv). The cache
+ * rows [s, s+B) must already hold the block's fresh K/V (fdl_kv_store); the
+ * other rows are the cached prefix and masked-suffix K/V.
+ *
+ *   q       [b, B, Hq, d]   dtype, device, 16-byte aligned
+ *   k_cache [b, Hkv, L, d]  dtype, device, 16-byte aligned
+ *   v_cache [b, Hkv, L, d]  dtype, device, 16-byte aligned
+ *   out     [b, B, Hq, d]   dtype, device (written)
+ *   lse     [b, Hq, B] f32, device, optional (NULL = not written):
+ *           natural-log softmax denominator, lse = log sum_j exp(scale q.k_j)
+ *   ws      device scratch of >= fdl_attention_workspace_bytes(desc) bytes
+ * Errors: FDL_EINVAL (shape, null, alignment), FDL_EUNSUPPORTED (head_dim),
+ * FDL_EWORKSPACE, FDL_ECUDA. */
+FDL_API int fdl_dualcache_attention(fdl_ctx* ctx, const fdl_attn_desc* desc,
+                            const void* q, const void* k_cache,
+                            const void* v_cache, void* out, float* lse,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Store fresh K/V rows into the caches in place: the block slot at every
+ * step (start = s, n = B) and the whole cache at a refresh after a block
+ * completes (start = 0, n = L; ICLR reviews, review 4 question 2: all K/V
+ * are recomputed once a block is done).
+ *
+ *   k_new, v_new [b, n, Hkv, d] dtype, device (token-major, as a projection
+ *                writes them), 16-byte aligned
+ *   k_cache, v_cache [b, Hkv, L, d] dtype, device; rows [start, start+n)
+ *                written, all other rows untouched
+ * Uses desc->batch, n_kv_heads, head_dim, seq_len, dtype.
+ * Errors: FDL_EINVAL (start < 0, start + n > L, n < 1, null, alignment). */
+FDL_API int fdl_kv_store(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* k_new,
+                 const void* v_new, int start, int n, void* k_cache,
+                 void* v_cache, void* stream);
+
+/* ------------------------------------------------------------------------
+ * (b) LM head fused with the vocabulary-wide confidence reduction
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int rows;     /* M >= 1 hidden rows (the block's masked positions) */
+    int hidden;   /* D, multiple of 64 */
+    int vocab;    /* V >= 2 */
+    int dtype;    /* fdl_dtype of h and w; logits and reductions are f32 */
+} fdl_lmhead_desc;
+
+/* Bytes of scratch fdl_lmhead_confidence needs (per-tile partial maxima,
+ * sums and arguments). Returns 0 for an invalid context or descriptor. */
+FDL_API size_t fdl_lmhead_workspace_bytes(const fdl_ctx* ctx, const fdl_lmhead_desc* desc);
+
+/* Confidence of each row (Fast-dLLM abstract and README "Key techniques" 2:
+ * tokens are decoded when their confidence exceeds a threshold; confidence is
+ * read as the largest softmax probability of the predicted token).
+ *
+ *   z[r, v]  = h[r,:] . w[v,:] (+ bias_val[r] if v == bias_tok[r])   (f32)
+ *   conf[r]  = exp(max_v z - logsumexp_v z) = 1 / sum_v exp(z[r,v] - max z)
+ *   tok[r]   = smallest v with z[r, v] == max z
+ * The [M, V] logits are never written to memory.
+ *
+ *   h        [M, D] dtype, device, 16-byte aligned
+ *   w        [V, D] dtype, device, 16-byte aligned (each vocab row contiguous)
+ *   bias_tok [M] int32, device, optional (NULL: no bias); entries in [0, V)
+ *   bias_val [M] f32, device; required iff bias_tok is given
+ *   conf     [M] f32, device (written); tok [M] int32, device (written)
+ *   ws       device scratch >= fdl_lmhead_workspace_bytes(desc)
+ * Errors: FDL_EINVAL, FDL_EUNSUPPORTED, FDL_EWORKSPACE, FDL_ECUDA. */
+FDL_API int fdl_lmhead_confidence(fdl_ctx* ctx, const fdl_lmhead_desc* desc,
+                          const void* h, const void* w,
+                          const int32_t* bias_tok, const float* bias_val,
+                          float* conf, int32_t* tok, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* ------------------------------------------------------------------------
+ * (b) threshold select + scatter
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int batch;        /* b >= 1 */
+    int seq_len;      /* L */
+    int block_start;  /* s */
+    int block_len;    /* B, 1 <= B <= 1024, s + B <= L */
+    float tau;        /* threshold, finite */
+} fdl_unmask_desc;
+
+/* One confidence-aware parallel unmask step (Fast-dLLM abstract; README "Key
+ * techniques" 2; aibase news "Innovations" 2).
+ *
+ * For each sequence, the candidates are the positions p in [s, s+B) with
+ * masked[b,p] != 0. Selected = candidates with conf > tau (strict; NaN never
+ * selected). If none is selected but a candidate exists, the single candidate
+ * with the largest confidence is selected, the lowest position on ties.
+ * For every selected p: x[b,p] = tok[b, p-s], masked[b,p] = 0. Positions
+ * outside the block and already-decoded positions are never written.
+ *
+ *   conf      [b, B] f32, device: slot i describes position s+i (slots of
+ *             decoded positions are ignored)
+ *   tok       [b, B] int32, device
+ *   x         [b, L] int32, device, updated in place
+ *   masked    [b, L] uint8, device, updated in place (0 = decoded)
+ *   remaining [b] int32, device (written): masked positions left in the block
+ *   n_decoded [b] int32, device, optional (NULL = not written)
+ * A block whose candidates all have NaN confidence decodes nothing and sets
+ * FDL_EDEVICE in the device error word.
+ * Errors: FDL_EINVAL (shape, null, non-finite tau), FDL_ECUDA. */
+FDL_API int fdl_threshold_unmask(fdl_ctx* ctx, const fdl_unmask_desc* desc,
+                         const float* conf, const int32_t* tok, int32_t* x,
+                         uint8_t* masked, int32_t* remaining,
+                         int32_t* n_decoded, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FDLLM_H */
