@@ -1,0 +1,103 @@
+"""Run one library call repeatedly on seeded synthetic input and time it.
+
+    python -m block_kv_cache_b200.kernel_cases lmhead --rows 32 [--iters 20]
+    python -m block_kv_cache_b200.kernel_cases attention --heads 32 --kv-heads 32 \
+        --prefix 512 --block 32 --suffix 224 [--layers 32]
+
+Used to profile a single kernel (e.g. under ncu with -k/-c) and to time it
+with CUDA events. Prints one JSON line: mean µs per call and the achieved
+algorithmic bandwidth / throughput of that call.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+import torch
+
+from block_kv_cache_b200 import fdllm, synth
+
+
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()
+
+
+def run_lmhead(a, ctx):
+    c = synth.lmhead_case(rows=a.rows, hidden=a.hidden, vocab=a.vocab, seed=1, w_seed=0,
+                          mask_id=min(126336, a.vocab - 1))
+    h, w = _bf16(c.h), _bf16(c.w)
+    bt, bv = torch.from_numpy(c.bias_tok).cuda(), torch.from_numpy(c.bias_val).cuda()
+    conf, tok = ctx.lmhead_confidence(h, w, bt, bv)
+    for _ in range(a.warmup):
+        ctx.lmhead_confidence(h, w, bt, bv, conf=conf, tok=tok)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        ctx.lmhead_confidence(h, w, bt, bv, conf=conf, tok=tok)
+    e1.record()
+    torch.cuda.synchronize()
+    ctx.device_status()
+    us = e0.elapsed_time(e1) * 1e3 / a.iters
+    nbytes = a.vocab * a.hidden * 2 + a.rows * a.hidden * 2 + a.rows * 16
+    flops = 2.0 * a.rows * a.hidden * a.vocab
+    return {"op": "lmhead_confidence", "rows": a.rows, "hidden": a.hidden, "vocab": a.vocab,
+            "us": us, "GBps": nbytes / us / 1e3, "TFLOPs": flops / us / 1e6}
+
+
+def run_attention(a, ctx):
+    cases = [synth.attn_case(batch=a.batch, n_q_heads=a.heads, n_kv_heads=a.kv_heads,
+                             head_dim=a.head_dim, prefix=a.prefix, block=a.block,
+                             suffix=a.suffix, dtype="bf16", seed=l) for l in range(a.layers)]
+    q = [_bf16(c.q) for c in cases]
+    kc = [_bf16(c.k_cache) for c in cases]
+    vc = [_bf16(c.v_cache) for c in cases]
+    out = torch.empty_like(q[0])
+    s = a.prefix
+    for l in range(a.layers):
+        ctx.dualcache_attention(q[l], kc[l], vc[l], s, out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for it in range(a.iters):
+        l = it % a.layers
+        ctx.dualcache_attention(q[l], kc[l], vc[l], s, out=out)
+    e1.record()
+    torch.cuda.synchronize()
+    ctx.device_status()
+    us = e0.elapsed_time(e1) * 1e3 / a.iters
+    L = a.prefix + a.block + a.suffix
+    nbytes = (2 * a.batch * a.kv_heads * L * a.head_dim * 2
+              + 2 * a.batch * a.block * a.heads * a.head_dim * 2)
+    flops = 4.0 * a.batch * a.heads * a.block * L * a.head_dim
+    return {"op": "dualcache_attention", "heads": a.heads, "kv_heads": a.kv_heads, "L": L,
+            "block": a.block, "batch": a.batch, "us": us, "GBps": nbytes / us / 1e3,
+            "TFLOPs": flops / us / 1e6}
+
+
+def main():
+    p = argparse.ArgumentParser()
+    p.add_argument("op", choices=["lmhead", "attention"])
+    p.add_argument("--rows", type=int, default=32)
+    p.add_argument("--hidden", type=int, default=4096)
+    p.add_argument("--vocab", type=int, default=126464)
+    p.add_argument("--batch", type=int, default=1)
+    p.add_argument("--heads", type=int, default=32)
+    p.add_argument("--kv-heads", type=int, default=32)
+    p.add_argument("--head-dim", type=int, default=128)
+    p.add_argument("--prefix", type=int, default=512)
+    p.add_argument("--block", type=int, default=32)
+    p.add_argument("--suffix", type=int, default=224)
+    p.add_argument("--layers", type=int, default=32)
+    p.add_argument("--iters", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    a = p.parse_args()
+    ctx = fdllm.Context(0)
+    r = run_lmhead(a, ctx) if a.op == "lmhead" else run_attention(a, ctx)
+    print(json.dumps(r), flush=True)
+    ctx.close()
+
+
+if __name__ == "__main__":
+    main()
