@@ -277,3 +277,13 @@ int fdl_threshold_unmask(fdl_ctx* ctx, const fdl_unmask_desc* desc, const float*
 }
 
 }  // extern "C"
+
+namespace fdl {
+// Device id of a context (for library-internal entry points in other files).
+int ctx_device(const fdl_ctx* ctx) { return ctx ? ctx->device : -1; }
+}  // namespace fdl
+
+namespace fdl {
+// Record `msg` as the calling thread's last error and return `code`.
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace fdl

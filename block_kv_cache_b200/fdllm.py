@@ -26,7 +26,8 @@ FDL_F32, FDL_BF16 = 0, 1
 EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
            "fdl_get_device_status", "fdl_attention_workspace_bytes",
            "fdl_dualcache_attention", "fdl_kv_store", "fdl_lmhead_workspace_bytes",
-           "fdl_lmhead_confidence", "fdl_threshold_unmask")
+           "fdl_lmhead_confidence", "fdl_threshold_unmask",
+           "fdl_lmhead_confidence_noalloc")
 
 
 class AttnDesc(ctypes.Structure):
@@ -80,6 +81,8 @@ def load() -> ctypes.CDLL:
     L.fdl_lmhead_workspace_bytes.restype = sz
     L.fdl_lmhead_confidence.argtypes = [vp, ctypes.POINTER(LMHeadDesc), vp, vp, vp, vp, vp,
                                         vp, vp, sz, vp]
+    L.fdl_lmhead_confidence_noalloc.argtypes = [vp, ctypes.POINTER(LMHeadDesc), vp, vp, vp, vp,
+                                                vp, vp, vp]
     L.fdl_threshold_unmask.argtypes = [vp, ctypes.POINTER(UnmaskDesc), vp, vp, vp, vp, vp,
                                        vp, vp]
     for name in EXPORTS:
@@ -219,6 +222,26 @@ class Context:
                                             _ptr(bias_tok), _ptr(bias_val), _ptr(conf),
                                             _ptr(tok), _ptr(ws), ws.numel() * ws.element_size(),
                                             _stream(stream)))
+        return conf, tok
+
+    def lmhead_confidence_noalloc(self, h, w, bias_tok=None, bias_val=None, *, conf=None,
+                                  tok=None, stream=None):
+        """fdl_lmhead_confidence_noalloc: no workspace argument; the library's
+        built-in 8 MiB scratch array is used (see include/fdllm.h)."""
+        _need(h, "h", None, 2)
+        _need(w, "w", h.dtype, 2)
+        if bias_tok is not None:
+            _need(bias_tok, "bias_tok", torch.int32, 1)
+            _need(bias_val, "bias_val", torch.float32, 1)
+        M, D = h.shape
+        d = LMHeadDesc(M, D, w.shape[0], _dtype_code(h))
+        if conf is None:
+            conf = torch.empty(M, dtype=torch.float32, device=h.device)
+        if tok is None:
+            tok = torch.empty(M, dtype=torch.int32, device=h.device)
+        _check(load().fdl_lmhead_confidence_noalloc(self._h, ctypes.byref(d), _ptr(h), _ptr(w),
+                                                    _ptr(bias_tok), _ptr(bias_val), _ptr(conf),
+                                                    _ptr(tok), _stream(stream)))
         return conf, tok
 
     # -- (b) threshold select + scatter -----------------------------------

@@ -176,6 +176,30 @@ FDL_API int fdl_lmhead_confidence(fdl_ctx* ctx, const fdl_lmhead_desc* desc,
                           float* conf, int32_t* tok, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* The same computation as fdl_lmhead_confidence, for callers that cannot
+ * provide a workspace: C hosts that own only their inputs and outputs, and
+ * engines whose device memory belongs entirely to their own pool, where one
+ * more cudaMalloc would fail or would bring the device-wide synchronisation
+ * cudaMalloc/cudaFree can cause. (The Fast-dLLM paper has no counterpart to
+ * this entry point; it is a deployment convenience of this library.)
+ *
+ * Its scratch is an 8 MiB array inside the library's device module, so every
+ * GPU that loads the library holds those 8 MiB until the process exits; the
+ * call itself allocates and frees nothing. Shapes whose scratch would exceed
+ * 8 MiB (rows x ceil(vocab / 128) x 12 bytes, e.g. more than 707 rows at a
+ * vocabulary of 126464) are rejected with FDL_EINVAL before anything runs.
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's
+ * contents; each call writes every entry it later reads. Calls whose
+ * executions overlap on the GPU (different streams, or different contexts
+ * on one device) race on the array and must be ordered by the caller.
+ * Arguments, layouts and other errors as fdl_lmhead_confidence. */
+FDL_API int fdl_lmhead_confidence_noalloc(fdl_ctx* ctx, const fdl_lmhead_desc* desc,
+                                          const void* h, const void* w,
+                                          const int32_t* bias_tok, const float* bias_val,
+                                          float* conf, int32_t* tok, void* stream);
+
 /* ------------------------------------------------------------------------
  * (b) threshold select + scatter
  * ------------------------------------------------------------------------ */
