@@ -73,7 +73,7 @@ int check_attn(const fdl_attn_desc* d) {
 
 fdl::AttnShape attn_shape(const fdl_attn_desc* d) {
     fdl::AttnShape s{d->batch, d->n_q_heads, d->n_kv_heads, d->head_dim, d->seq_len,
-                     d->block_start, d->block_len, d->scale};
+                     d->block_start, d->block_len, d->scale, d->dtype == FDL_BF16 ? 1 : 0};
     if (s.scale == 0.f) s.scale = 1.0f / sqrtf((float)d->head_dim);
     return s;
 }
@@ -185,7 +185,7 @@ int fdl_dualcache_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void*
                                     (const float*)v_cache, (float*)out, lse, ws, ctx->sm_count,
                                     (cudaStream_t)stream)
         : fdl::launch_attention_bf16(s, q, k_cache, v_cache, out, lse, ws, ctx->sm_count,
-                                     (cudaStream_t)stream);
+                                     ctx->d_err, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
     return FDL_OK;
 }

@@ -11,8 +11,10 @@
 // the log2 domain (scale * log2(e) folded in) so exp2f serves the softmax.
 // Pass 2: per (query row, head, sequence) the partials are merged.
 //
-// This SIMT version computes in f32 FFMA (the f32 instantiation must stay
-// within 1e-4 relative error, out of reach of TF32 tensor cores).
+// This SIMT version serves f32 tensors: it computes in f32 FFMA, because the
+// f32 path must stay within 1e-4 relative error, out of reach of TF32 tensor
+// cores. bf16 tensors go to the tcgen05 kernel (attention_tc.cu), which
+// writes the same partials and is merged by the same combine kernel.
 #include "common.cuh"
 #include "launch.h"
 
@@ -21,7 +23,7 @@ namespace fdl {
 constexpr int ATT_THREADS = 256;          // 8 warps
 constexpr int ATT_KT = 32;                // keys per smem tile (one per lane)
 
-int attn_num_splits(const AttnShape& s, int sm_count) {
+static int attn_num_splits(const AttnShape& s, int sm_count) {
     const int heads = s.batch * s.n_q_heads;
     const int max_splits = (s.seq_len + ATT_KT - 1) / ATT_KT;
     int want = (2 * sm_count + heads - 1) / heads;
@@ -31,6 +33,7 @@ int attn_num_splits(const AttnShape& s, int sm_count) {
 }
 
 size_t attn_workspace_bytes(const AttnShape& s, int sm_count) {
+    if (s.bf16) return attn_tc_workspace_bytes(s, sm_count);
     const size_t ns = attn_num_splits(s, sm_count);
     const size_t rows = (size_t)s.batch * s.n_q_heads * ns * s.block_len;
     return rows * (s.head_dim + 2) * sizeof(float);
@@ -192,11 +195,18 @@ cudaError_t launch_attention_f32(const AttnShape& s, const float* q, const float
     return dispatch_attn<float>(s, q, k, v, out, lse, ws, sm_count, st);
 }
 
-cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
-                                  const void* v, void* out, float* lse, void* ws,
-                                  int sm_count, cudaStream_t st) {
-    return dispatch_attn<bf16>(s, (const bf16*)q, (const bf16*)k, (const bf16*)v, (bf16*)out,
-                               lse, ws, sm_count, st);
+
+cudaError_t launch_attn_combine_bf16(const float* ws_o, const float* ws_ml, void* out, float* lse,
+                                     int batch, int B, int Hq, int D, int n_splits,
+                                     cudaStream_t st) {
+    dim3 g2(B, Hq, batch);
+    if (D == 128)
+        attn_combine_kernel<bf16, 128><<<g2, 128, 0, st>>>(ws_o, ws_ml, (bf16*)out, lse, B, Hq,
+                                                           n_splits);
+    else
+        attn_combine_kernel<bf16, 64><<<g2, 64, 0, st>>>(ws_o, ws_ml, (bf16*)out, lse, B, Hq,
+                                                         n_splits);
+    return cudaGetLastError();
 }
 
 }  // namespace fdl

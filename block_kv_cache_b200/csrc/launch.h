@@ -9,18 +9,19 @@ namespace fdl {
 struct AttnShape {
     int batch, n_q_heads, n_kv_heads, head_dim, seq_len, block_start, block_len;
     float scale;  // resolved (never 0)
+    int bf16;     // 1: bf16 tensors (tcgen05 kernel), 0: f32 (SIMT kernel)
 };
 
-// split-KV partition used by the attention kernels
-int attn_num_splits(const AttnShape& s, int sm_count);
+// Scratch for the split-KV partials of either attention kernel.
 size_t attn_workspace_bytes(const AttnShape& s, int sm_count);
+size_t attn_tc_workspace_bytes(const AttnShape& s, int sm_count);
 
 cudaError_t launch_attention_f32(const AttnShape& s, const float* q, const float* k,
                                  const float* v, float* out, float* lse, void* ws,
                                  int sm_count, cudaStream_t st);
 cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
                                   const void* v, void* out, float* lse, void* ws,
-                                  int sm_count, cudaStream_t st);
+                                  int sm_count, int* dev_err, cudaStream_t st);
 
 cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len,
                             int elem_bytes, const void* k_new, const void* v_new,
