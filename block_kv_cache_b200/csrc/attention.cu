@@ -196,17 +196,4 @@ cudaError_t launch_attention_f32(const AttnShape& s, const float* q, const float
 }
 
 
-cudaError_t launch_attn_combine_bf16(const float* ws_o, const float* ws_ml, void* out, float* lse,
-                                     int batch, int B, int Hq, int D, int n_splits,
-                                     cudaStream_t st) {
-    dim3 g2(B, Hq, batch);
-    if (D == 128)
-        attn_combine_kernel<bf16, 128><<<g2, 128, 0, st>>>(ws_o, ws_ml, (bf16*)out, lse, B, Hq,
-                                                           n_splits);
-    else
-        attn_combine_kernel<bf16, 64><<<g2, 64, 0, st>>>(ws_o, ws_ml, (bf16*)out, lse, B, Hq,
-                                                         n_splits);
-    return cudaGetLastError();
-}
-
 }  // namespace fdl

@@ -4,34 +4,49 @@
 // 1): the block's queries attend, without a mask, over the whole cache
 // [prefix | block slot | masked suffix]; the block slot holds fresh K/V.
 //
-// One CTA = one key tile of KT keys of one (sequence, kv head, head chunk).
-// All query heads that share the kv head (GQA group, or a chunk of it) are
-// packed into the MMA's M dimension, so each K/V tile is read from HBM once
-// per group: rows r = i * hc + j hold query i of head (chunk*hc + j).
-//   warp 4 (one thread): TMA loads of Q (3-D box: d x heads x queries), K and
-//          V tiles (128-byte swizzle); tcgen05.mma S = Q K^T into TMEM
-//          (M=128 per row tile, N=KT, K=d); after the softmax, O = P V with V
-//          as an MN-major operand (N=d, K=KT)
-//   warps 0-3: thread = query row: read S from TMEM, softmax in the log2
-//          domain (scale * log2 e folded in), P as bf16 into shared memory in
-//          the swizzled K-major layout the MMA reads, then O from TMEM to
-//          the split-KV workspace with the row's (max, sum)
-// A second kernel merges the splits (attention.cu, attn_combine_kernel).
+// Work decomposition. The query heads that share a kv head (the GQA group,
+// or a chunk of it) are packed as R = hc * B query rows, row r = i*hc + j
+// holding query i of head j of the chunk. A CTA owns one (sequence, kv head,
+// head chunk) and a contiguous range ("split") of 64-key tiles streamed
+// through a TMA ring, so every K/V byte is read from HBM once. The splits of
+// one (sequence, kv head, chunk) form a thread-block cluster and merge their
+// partial softmaxes through distributed shared memory; the cluster writes the
+// final bf16 output and LSE, with no second pass over memory.
+//
+// The 128 TMEM lanes are the MMA's M dimension: R <= 128 packed rows use one
+// 128-row tile, R in (128, 256] two, each with its own softmax warpgroup. A
+// softmax warp reads only its own 32-lane quarter of TMEM; warps whose rows
+// are all padding sit out. (With one block of 32 queries per head, one warp
+// per tile does the softmax: 64 exponentials per tile per thread, less than
+// the time a 64-key tile takes to arrive at this SM's share of HBM bandwidth.)
+//
+//   softmax warps (4 per 128-row tile): thread = TMEM lane; online softmax in
+//       the log2 domain (scale*log2 e folded into one FFMA); P(t) as bf16 into
+//       one of two shared-memory buffers; O rescaled in TMEM only when the
+//       running max grows by more than 8 (a factor 2^8)
+//   TMA warp (1 thread): Q once, then K and V tiles
+//   MMA warp (1 thread): TMEM owner; tcgen05.mma S(t) = Q K(t)^T into one of
+//       two S buffers, then O += P(t) V(t) with V as an MN-major operand
 //
 // Roofline: HBM. Algorithmic bytes per call = K and V once (2*b*Hkv*L*d*2)
-// + q and out (2*b*B*Hq*d*2); the MMAs run at ~30 flop per byte.
+// + q and out (2*b*B*Hq*d*2).
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
 
 namespace fdl {
 
+constexpr int ATT_KT = 64;          // keys per tile
+constexpr int ATT_MAX_SPLITS = 8;   // portable cluster size
+
 struct AttnPlan {
-    int kt;        // keys per CTA
-    int mt;        // 128-row tiles of packed queries (1 or 2)
     int hc;        // query heads packed per CTA
     int n_chunks;  // head chunks per kv head
-    int n_splits;  // key tiles per (sequence, kv head)
+    int rows;      // packed rows R = hc * B
+    int mt;        // 128-row MMA tiles (1 or 2)
+    int tiles;     // 64-key tiles per (sequence, kv head)
+    int tps;       // tiles per split
+    int n_splits;  // cluster size
 };
 
 AttnPlan attn_tc_plan(const AttnShape& s, int sm_count) {
@@ -41,290 +56,459 @@ AttnPlan attn_tc_plan(const AttnShape& s, int sm_count) {
     if (p.hc > grp) p.hc = grp;
     if (p.hc < 1) p.hc = 1;
     p.n_chunks = (grp + p.hc - 1) / p.hc;
-    p.mt = p.hc * s.block_len > 128 ? 2 : 1;
+    p.rows = p.hc * s.block_len;
+    p.mt = p.rows > 128 ? 2 : 1;
+    p.tiles = (s.seq_len + ATT_KT - 1) / ATT_KT;
     const int units = s.batch * s.n_kv_heads * p.n_chunks;
-    static const int kts1[] = {192, 128, 64}, kts2[] = {128, 64};
-    const int* kts = p.mt == 1 ? kts1 : kts2;
-    const int nk = p.mt == 1 ? 3 : 2;
-    long best_waves = -1;
-    p.kt = kts[0];
-    for (int i = 0; i < nk; ++i) {
-        const long ctas = (long)units * ((s.seq_len + kts[i] - 1) / kts[i]);
-        const long waves = (ctas + sm_count - 1) / sm_count;
-        if (best_waves < 0 || waves <= best_waves) {   // ties: the smaller tile, more CTAs
-            best_waves = waves;
-            p.kt = kts[i];
-        }
-    }
-    p.n_splits = (s.seq_len + p.kt - 1) / p.kt;
+    int splits = sm_count / units;
+    if (splits < 1) splits = 1;
+    if (splits > ATT_MAX_SPLITS) splits = ATT_MAX_SPLITS;
+    if (splits > p.tiles) splits = p.tiles;
+    p.tps = (p.tiles + splits - 1) / splits;
+    p.n_splits = (p.tiles + p.tps - 1) / p.tps;
     return p;
 }
 
 namespace {
 
-constexpr int TC_THREADS = 160;
-
-template <int D, int KT, int MT>
-struct AttnSmem {
-    static constexpr int DC = D / 64;                       // 64-wide d chunks
-    static constexpr int Q_CHUNK = MT * 128 * 128;          // bytes per d chunk of Q
-    static constexpr int Q_BYTES = DC * Q_CHUNK;
-    static constexpr int KV_CHUNK = KT * 128;               // bytes per d chunk of K or V
-    static constexpr int KV_BYTES = DC * KV_CHUNK;
-    static constexpr int P_CHUNK = 128 * 128;               // 64 keys x 128 rows
-    static constexpr int P_TILE = (KT / 64) * P_CHUNK;      // one 128-row tile
+template <int D, int MT>
+struct Att4 {
+    static constexpr int STAGES = MT == 1 ? 3 : 2;
+    static constexpr int THREADS = 32 * (4 * MT + 2);
+    static constexpr int TMA_WARP = 4 * MT, MMA_WARP = 4 * MT + 1;
+    static constexpr int DC = D / 64;
+    static constexpr int Q_CHUNK = MT * 128 * 128;
+    static constexpr int KV_CHUNK = ATT_KT * 128;
+    static constexpr int KV_TILE = DC * KV_CHUNK;
+    static constexpr int P_TILE = 128 * 128;                // 128 rows x 64 keys
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + Q_BYTES;
-    static constexpr int OFF_V = OFF_K + KV_BYTES;
-    static constexpr int OFF_P = OFF_V + KV_BYTES;
-    static constexpr int OFF_BAR = OFF_P + MT * P_TILE;
-    static constexpr size_t TOTAL = 1024 + OFF_BAR + 128;
-    static constexpr uint32_t TMEM_S = 0;                    // S[mt] at mt*KT
-    static constexpr uint32_t TMEM_O = MT * KT;              // O[mt] at MT*KT + mt*D
-    static constexpr uint32_t TMEM_USED = MT * (KT + D);
-    static constexpr uint32_t TMEM_ALLOC = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64
-                                         : TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+    static constexpr int OFF_K = OFF_Q + DC * Q_CHUNK;
+    static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
+    static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;   // P[buffer][m]
+    static constexpr int OFF_RED = OFF_P + 2 * MT * P_TILE;  // 256 x (max, sum) floats
+    static constexpr int OFF_BAR = OFF_RED + 256 * 2 * 4;
+    static constexpr size_t TOTAL = 1024 + OFF_BAR + 256;
+    // After the last MMA, [OFF_K, OFF_RED) holds this CTA's partial output
+    // (R rows x D floats, float4 slots XOR-swizzled by row) for the cluster.
+    static_assert(128 * MT * D * 4 <= OFF_RED - OFF_K, "partial buffer");
+    static constexpr uint32_t TMEM_S = 0;                    // S[b2][m] at (b2*MT + m)*64
+    static constexpr uint32_t TMEM_O = 2 * MT * ATT_KT;      // O[m] at TMEM_O + m*D
+    static constexpr uint32_t TMEM_USED = 2 * MT * ATT_KT + MT * D;
+    static constexpr uint32_t TMEM_ALLOC = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
     static_assert(TMEM_USED <= 512, "TMEM budget");
     static_assert(TOTAL <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, int KT, int MT>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 2^x on the special-function unit (PTX ex2.approx, flush-to-zero); -inf -> 0.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+struct AttnArgs {
+    bf16* out;
+    float* lse;         // optional
+    int B, Hq, Hkv, L, hc, n_chunks, rows, tiles, tps, n_splits;
+    float scale_log2;
+    int* err;
+};
+
+template <int D, int MT>
+__global__ void __launch_bounds__(Att4<D, MT>::THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, float* __restrict__ ws_o,
-               float* __restrict__ ws_ml, int B, int Hq, int Hkv, int L, int hc, int n_chunks,
-               int n_splits, float scale_log2, int* err) {
+               const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
     using namespace sm100;
-    using S = AttnSmem<D, KT, MT>;
+    using S = Att4<D, MT>;
+    constexpr int KT = ATT_KT, STAGES = S::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* smem = smem_raw + pad;
     const uint32_t sb = raw + pad;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+    const uint32_t bar_q = smem_u32(bars + 0);
+    auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
+    auto v_full = [&](int s) { return smem_u32(bars + 1 + STAGES + s); };
+    auto kv_empty = [&](int s) { return smem_u32(bars + 1 + 2 * STAGES + s); };
+    auto s_full = [&](int b) { return smem_u32(bars + 1 + 3 * STAGES + b); };
+    auto s_free = [&](int b) { return smem_u32(bars + 3 + 3 * STAGES + b); };
+    auto p_full = [&](int b) { return smem_u32(bars + 5 + 3 * STAGES + b); };
+    auto o_done = [&](int b) { return smem_u32(bars + 7 + 3 * STAGES + b); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 3 * STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const uint32_t bar_qk = smem_u32(bars + 0), bar_v = smem_u32(bars + 1);
-    const uint32_t bar_s = smem_u32(bars + 2), bar_p = smem_u32(bars + 3);
-    const uint32_t bar_o = smem_u32(bars + 4);
 
-    const int split = blockIdx.x;
-    const int g = blockIdx.y / n_chunks, chunk = blockIdx.y % n_chunks;
+    const int split = blockIdx.x;                    // == rank in the cluster
+    const int g = blockIdx.y / a.n_chunks, chunk = blockIdx.y % a.n_chunks;
     const int bb = blockIdx.z;
-    const int grp = Hq / Hkv;
-    const int k0 = split * KT;
-    const int nk = min(KT, L - k0);
+    const int grp = a.Hq / a.Hkv;
+    const int t_begin = split * a.tps;
+    const int nt = min(a.tps, a.tiles - t_begin);
+    const int k_begin = t_begin * KT;
+    const int k_end = min(a.L, k_begin + nt * KT);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // softmax warps with at least one real row (a warp covers 32 packed rows)
+    const int live_warps = (a.rows + 31) / 32;
+    const int live_threads = live_warps * 32;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_qk, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_p, 128);
-        mbar_init(bar_o, 1);
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(v_full(s), 1);
+            mbar_init(kv_empty(s), 1);
+        }
+        for (int b2 = 0; b2 < 2; ++b2) {
+            mbar_init(s_full(b2), 1);
+            mbar_init(s_free(b2), live_threads);
+            mbar_init(p_full(b2), live_threads);
+            mbar_init(o_done(b2), 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 4) tmem_alloc(smem_u32(tmem_slot), S::TMEM_ALLOC);
+    if (warp == S::MMA_WARP) tmem_alloc(smem_u32(tmem_slot), S::TMEM_ALLOC);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    bool ok = true;
 
-    if (warp == 4) {
+    if (warp == S::TMA_WARP) {
+        // ---------------------------------------------------------------- TMA
         if (lane == 0) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            const int krow = (bb * Hkv + g) * L + k0;
-            const int head0 = g * grp + chunk * hc;
-            mbar_arrive_expect_tx(bar_qk, (uint32_t)(S::DC * hc * B * 128 + S::KV_BYTES));
-            for (int c = 0; c < S::DC; ++c) {
-                tma_load_3d(sb + S::OFF_Q + c * S::Q_CHUNK, &tmQ, bar_qk, c * 64, head0, bb * B);
-                tma_load_2d(sb + S::OFF_K + c * S::KV_CHUNK, &tmK, bar_qk, c * 64, krow);
+            const int head0 = g * grp + chunk * a.hc;
+            mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
+            for (int dc = 0; dc < S::DC; ++dc)
+                tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
+                            bb * a.B);
+            const int krow0 = (bb * a.Hkv + g) * a.L + k_begin;
+            int t = 0;
+            for (; ok && t < nt; ++t) {
+                const int st = t % STAGES;
+                if (!(ok = mbar_wait(kv_empty(st), ((t / STAGES) & 1) ^ 1, abort_flag, a.err)))
+                    break;
+                mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
+                for (int dc = 0; dc < S::DC; ++dc)
+                    tma_load_2d(sb + S::OFF_K + st * S::KV_TILE + dc * S::KV_CHUNK, &tmK,
+                                k_full(st), dc * 64, krow0 + t * KT);
+                mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
+                for (int dc = 0; dc < S::DC; ++dc)
+                    tma_load_2d(sb + S::OFF_V + st * S::KV_TILE + dc * S::KV_CHUNK, &tmV,
+                                v_full(st), dc * 64, krow0 + t * KT);
             }
-            mbar_arrive_expect_tx(bar_v, (uint32_t)S::KV_BYTES);
-            for (int c = 0; c < S::DC; ++c)
-                tma_load_2d(sb + S::OFF_V + c * S::KV_CHUNK, &tmV, bar_v, c * 64, krow);
-
-            bool ok = mbar_wait(bar_qk, 0, abort_flag, err);
-            if (ok) {
-                tc_fence_after();
-                constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
+            // tail: every stage handed out has been released again
+            for (int u = t; ok && u < t + STAGES; ++u)
+                ok = mbar_wait(kv_empty(u % STAGES), ((u / STAGES) & 1) ^ 1, abort_flag, a.err);
+        }
+    } else if (warp == S::MMA_WARP) {
+        // ---------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
+            constexpr uint32_t idesc_o = umma_idesc_bf16_f32(128, D, true);
+            ok = mbar_wait(bar_q, 0, abort_flag, a.err);
+            for (int t = 0; ok && t <= nt; ++t) {
+                if (t < nt) {
+                    const int st = t % STAGES, b2 = t & 1;
+                    if (!(ok = mbar_wait(k_full(st), (t / STAGES) & 1, abort_flag, a.err))) break;
+                    if (!(ok = mbar_wait(s_free(b2), ((t >> 1) & 1) ^ 1, abort_flag, a.err)))
+                        break;
+                    tc_fence_after();
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
+                    for (int m = 0; m < MT; ++m)
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t qa = sb + S::OFF_Q + (kk >> 2) * S::Q_CHUNK + m * 16384 +
-                                            (kk & 3) * 32;
-                        const uint32_t ka = sb + S::OFF_K + (kk >> 2) * S::KV_CHUNK + (kk & 3) * 32;
-                        umma_bf16(tmem + S::TMEM_S + m * KT, umma_desc_sw128(qa),
-                                  umma_desc_sw128(ka), idesc_s, kk > 0);
-                    }
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t qa = sb + S::OFF_Q + (kk >> 2) * S::Q_CHUNK +
+                                                m * 16384 + (kk & 3) * 32;
+                            const uint32_t ka = sb + S::OFF_K + st * S::KV_TILE +
+                                                (kk >> 2) * S::KV_CHUNK + (kk & 3) * 32;
+                            umma_bf16(tmem + S::TMEM_S + (b2 * MT + m) * KT, umma_desc_sw128(qa),
+                                      umma_desc_sw128(ka), idesc_s, kk > 0);
+                        }
+                    umma_commit(s_full(b2));
                 }
-                umma_commit(bar_s);
-                ok = mbar_wait(bar_v, 0, abort_flag, err) && mbar_wait(bar_p, 0, abort_flag, err);
-            }
-            if (ok) {
-                tc_fence_after();
-                constexpr uint32_t idesc_o = umma_idesc_bf16_f32(128, D, true);
+                if (t > 0) {
+                    const int u = t - 1, su = u % STAGES, pb = u & 1;
+                    if (!(ok = mbar_wait(p_full(pb), (u >> 1) & 1, abort_flag, a.err))) break;
+                    if (!(ok = mbar_wait(v_full(su), (u / STAGES) & 1, abort_flag, a.err))) break;
+                    tc_fence_after();
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
+                    for (int m = 0; m < MT; ++m)
 #pragma unroll
-                    for (int ks = 0; ks < KT / 16; ++ks) {
-                        const uint32_t pa = sb + S::OFF_P + m * S::P_TILE + (ks >> 2) * S::P_CHUNK +
-                                            (ks & 3) * 32;
-                        const uint32_t va = sb + S::OFF_V + ks * 2048;
-                        umma_bf16(tmem + S::TMEM_O + m * D, umma_desc_sw128(pa),
-                                  umma_desc_sw128_mn(va, S::KV_CHUNK), idesc_o, ks > 0);
-                    }
+                        for (int ks = 0; ks < KT / 16; ++ks) {
+                            const uint32_t pa = sb + S::OFF_P + (pb * MT + m) * S::P_TILE +
+                                                (ks & 3) * 32;
+                            const uint32_t va = sb + S::OFF_V + su * S::KV_TILE + ks * 2048;
+                            umma_bf16(tmem + S::TMEM_O + m * D, umma_desc_sw128(pa),
+                                      umma_desc_sw128_mn(va, S::KV_CHUNK), idesc_o,
+                                      (u > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    umma_commit(o_done(pb));
+                    umma_commit(kv_empty(su));
                 }
-                umma_commit(bar_o);
             }
         }
-    } else {
-        // softmax / epilogue warps: warp w reads TMEM lanes [32w, 32w+32)
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(bar_s, 0, abort_flag, err);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        float mrow[MT], lrow[MT];
-        if (ok) {
+    } else if (warp < live_warps) {
+        // ------------------------------------------------------------ softmax
+        const int q = warp & 3;                          // TMEM lane quarter
+        const int m = warp >> 2;                         // 128-row tile
+        const int r = q * 32 + lane;                     // row within the tile
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        float m_run = -INFINITY, l_run = 0.f;            // running max (log2 units), sum
+        for (int t = 0; t < nt; ++t) {
+            const int b2 = t & 1;
+            if (!(ok = mbar_wait_warp(s_full(b2), (t >> 1) & 1, abort_flag, a.err))) break;
             tc_fence_after();
+            float sr[KT];
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const uint32_t tS = tmem + ((uint32_t)(warp * 32) << 16) + S::TMEM_S + m * KT;
-                float mx = -INFINITY;
-#pragma unroll 1
-                for (int c = 0; c < KT / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c * 32 + j < nk) mx = fmaxf(mx, __uint_as_float(r[j]) * scale_log2);
-                }
-                float l = 0.f;
-                const int row = warp * 32 + lane;                    // row within the tile
-                uint8_t* prow = smem + S::OFF_P + m * S::P_TILE + row * 128;
-#pragma unroll 1
-                for (int c = 0; c < KT / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(tS + c * 32, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const int key = c * 32 + j;
-                        const float p0 = key < nk ? exp2f(fmaf(__uint_as_float(r[j]), scale_log2, -mx)) : 0.f;
-                        const float p1 = key + 1 < nk ? exp2f(fmaf(__uint_as_float(r[j + 1]), scale_log2, -mx)) : 0.f;
-                        l += p0 + p1;
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                        pk[j >> 1] = *reinterpret_cast<uint32_t*>(&h2);
-                    }
-                    // 32 keys = 4 pieces of 16 B in chunk (c/2), pieces 4*(c&1)..+3
-                    uint8_t* pc = prow + (c >> 1) * S::P_CHUNK;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int piece = (c & 1) * 4 + q4;
-                        const int phys = piece ^ (row & 7);
-                        *reinterpret_cast<uint4*>(pc + phys * 16) =
-                            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-                    }
-                }
-                mrow[m] = mx;
-                lrow[m] = l;
-            }
-            fence_proxy_async();          // P (generic-proxy stores) -> MMA (async proxy)
+            for (int j = 0; j < KT; j += 16)
+                tmem_ld16(tmem + lane_base + S::TMEM_S + (b2 * MT + m) * KT + j,
+                          reinterpret_cast<uint32_t*>(sr) + j);
+            tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(bar_p);
-            if (lane == 0) ok = mbar_wait(bar_o, 0, abort_flag, err);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+            mbar_arrive(s_free(b2));
+
+            const int kbase = k_begin + t * KT;          // global key of sr[0]
+            if (kbase + KT > k_end) {                    // ragged last tile
+#pragma unroll
+                for (int j = 0; j < KT; ++j)
+                    if (kbase + j >= k_end) sr[j] = -INFINITY;
+            }
+            float mx = sr[0];
+#pragma unroll
+            for (int j = 1; j < KT; ++j) mx = fmaxf(mx, sr[j]);
+            mx *= a.scale_log2;                          // scale > 0 commutes with max
+            float alpha = 1.f;
+            bool rescale = false;
+            if (mx > m_run + 8.f || m_run == -INFINITY) {
+                const float mn = fmaxf(m_run, mx);
+                if (mn != -INFINITY) {
+                    alpha = ex2(m_run - mn);             // 0 on the first update
+                    rescale = m_run != -INFINITY;
+                    m_run = mn;
+                }
+            }
+            const float nmr = m_run == -INFINITY ? 0.f : -m_run;
+            float l = 0.f;
+            uint32_t pk[KT / 2];
+#pragma unroll
+            for (int j = 0; j < KT; j += 2) {
+                const float p0 = ex2(fmaf(sr[j], a.scale_log2, nmr));
+                const float p1 = ex2(fmaf(sr[j + 1], a.scale_log2, nmr));
+                l += p0 + p1;
+                pk[j >> 1] = pack_bf16(p0, p1);
+            }
+            l_run = l_run * alpha + l;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O holds P V up to tile t-1: wait for PV(t-1), then scale it
+                if (t > 0) {
+                    if (!(ok = mbar_wait_warp(o_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag,
+                                              a.err)))
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int d0 = 0; d0 < D; d0 += 16) {
+                        uint32_t o[16];
+                        const uint32_t ta = tmem + lane_base + S::TMEM_O + m * D + d0;
+                        tmem_ld16(ta, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 16; ++x)
+                            o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                        tmem_st16(ta, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P buffer b2 is free once PV(t-2) is done
+            if (!(ok = mbar_wait_warp(o_done(b2), ((t >> 1) & 1) ^ 1, abort_flag, a.err))) break;
+            uint8_t* prow = smem + S::OFF_P + (b2 * MT + m) * S::P_TILE + r * 128;
+#pragma unroll
+            for (int piece = 0; piece < 8; ++piece)      // 8 keys per 16-byte piece
+                *reinterpret_cast<uint4*>(prow + ((piece ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * piece], pk[4 * piece + 1], pk[4 * piece + 2],
+                               pk[4 * piece + 3]);
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(p_full(b2));
         }
+        // ----------------------------------------------------------- epilogue
+        if (ok)
+            ok = mbar_wait_warp(o_done((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, a.err);
+        // the live softmax warps agree on running the epilogue; every wait
+        // above is bounded, so all of them get here
+        named_sync(1, live_threads);
+        ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
         if (ok) {
             tc_fence_after();
+            float o[D];
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                const int r = m * 128 + warp * 32 + lane;            // packed row
-                const int i = r / hc, j = r % hc;
-                const int head_in_grp = chunk * hc + j;
-                const bool valid = i < B && head_in_grp < grp;
-                const int head = g * grp + head_in_grp;
-                const uint32_t tO = tmem + ((uint32_t)(warp * 32) << 16) + S::TMEM_O + m * D;
-                const size_t prow = valid ? (((size_t)bb * Hq + head) * n_splits + split) * B + i : 0;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(tO + c * 32, rr);
-                    tmem_wait_ld();
-                    if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + c * 32);
-#pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
-                            dst[q4] = make_float4(__uint_as_float(rr[4 * q4]),
-                                                  __uint_as_float(rr[4 * q4 + 1]),
-                                                  __uint_as_float(rr[4 * q4 + 2]),
-                                                  __uint_as_float(rr[4 * q4 + 3]));
-                    }
-                }
+            for (int d0 = 0; d0 < D; d0 += 16)
+                tmem_ld16(tmem + lane_base + S::TMEM_O + m * D + d0,
+                          reinterpret_cast<uint32_t*>(o) + d0);
+            tmem_wait_ld();
+            const int pr = m * 128 + r;                  // packed row
+            const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
+            const bool row_ok = pr < a.rows;
+            const bool valid = row_ok && i < a.B && hig < grp;
+            if (a.n_splits == 1) {
                 if (valid) {
-                    ws_ml[prow * 2 + 0] = mrow[m];
-                    ws_ml[prow * 2 + 1] = lrow[m];
+                    const int head = g * grp + hig;
+                    const float inv = 1.f / l_run;
+                    bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D;
+#pragma unroll
+                    for (int d = 0; d < D; d += 8)
+                        *reinterpret_cast<uint4*>(dst + d) = make_uint4(
+                            pack_bf16(o[d] * inv, o[d + 1] * inv),
+                            pack_bf16(o[d + 2] * inv, o[d + 3] * inv),
+                            pack_bf16(o[d + 4] * inv, o[d + 5] * inv),
+                            pack_bf16(o[d + 6] * inv, o[d + 7] * inv));
+                    if (a.lse)
+                        a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
+                            (m_run + log2f(l_run)) * 0.69314718055994530942f;
                 }
+            } else if (row_ok) {
+                // publish this CTA's partial for the cluster merge
+                float* part = reinterpret_cast<float*>(smem + S::OFF_K) + (size_t)pr * D;
+#pragma unroll
+                for (int d4 = 0; d4 < D / 4; ++d4)
+                    *reinterpret_cast<float4*>(part + ((d4 ^ (pr & 7)) << 2)) =
+                        make_float4(o[4 * d4], o[4 * d4 + 1], o[4 * d4 + 2], o[4 * d4 + 3]);
+                float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
+                red[2 * pr] = m_run;
+                red[2 * pr + 1] = l_run;
             }
         }
     }
+
+    if (a.n_splits > 1) {
+        // ------------------------------------------------ cluster merge of splits
+        // every thread of every CTA of the cluster takes part in both barriers
+        cluster_sync();
+        const int rpc = (a.rows + a.n_splits - 1) / a.n_splits;      // rows per CTA
+        const int r0 = split * rpc, r1 = min(a.rows, r0 + rpc);
+        const int items = (r1 > r0 ? r1 - r0 : 0) * (D / 4);
+        const uint32_t part_base = sb + S::OFF_K, red_base = sb + S::OFF_RED;
+        for (int it = threadIdx.x; it < items; it += S::THREADS) {
+            const int pr = r0 + it / (D / 4), d4 = it % (D / 4);
+            const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
+            if (i >= a.B || hig >= grp) continue;
+            float2 ml[ATT_MAX_SPLITS];
+            float4 v[ATT_MAX_SPLITS];
+            const uint32_t off_ml = red_base + pr * 8;
+            const uint32_t off_o = part_base + (uint32_t)(pr * D + ((d4 ^ (pr & 7)) << 2)) * 4;
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {    // issue every remote load first
+                if (cc < a.n_splits) {
+                    ml[cc] = ld_cluster_f2(cluster_map(off_ml, cc));
+                    v[cc] = ld_cluster_f4(cluster_map(off_o, cc));
+                }
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc)
+                if (cc < a.n_splits) M = fmaxf(M, ml[cc].x);
+            float Lsum = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {
+                if (cc < a.n_splits && ml[cc].x != -INFINITY) {
+                    const float w = ex2(ml[cc].x - M);
+                    Lsum += ml[cc].y * w;
+                    acc.x += v[cc].x * w; acc.y += v[cc].y * w;
+                    acc.z += v[cc].z * w; acc.w += v[cc].w * w;
+                }
+            }
+            const float inv = 1.f / Lsum;
+            const int head = g * grp + hig;
+            bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D + d4 * 4;
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+            if (a.lse && d4 == 0)
+                a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
+                    (M + log2f(Lsum)) * 0.69314718055994530942f;
+        }
+        cluster_sync();                    // no CTA leaves while others read its smem
+    }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == S::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, S::TMEM_ALLOC);
     }
 }
 
-template <int D, int KT, int MT>
-cudaError_t run_tc(const AttnShape& s, const AttnPlan& p, const CUtensorMap& tq,
-                   const CUtensorMap& tk, const CUtensorMap& tv, float* ws_o, float* ws_ml,
-                   int* err, cudaStream_t st) {
-    using S = AttnSmem<D, KT, MT>;
-    auto kfn = attn_tc_kernel<D, KT, MT>;
+template <int D, int MT>
+cudaError_t run_tc(const AttnPlan& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                   const CUtensorMap& tv, const AttnArgs& a, int batch, int hkv,
+                   cudaStream_t st) {
+    using S = Att4<D, MT>;
+    auto kfn = attn_tc_kernel<D, MT>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S::TOTAL);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_splits, s.n_kv_heads * p.n_chunks, s.batch);
-    kfn<<<grid, TC_THREADS, S::TOTAL, st>>>(tq, tk, tv, ws_o, ws_ml, s.block_len, s.n_q_heads,
-                                            s.n_kv_heads, s.seq_len, p.hc, p.n_chunks,
-                                            p.n_splits, s.scale * 1.4426950408889634f, err);
-    return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t dispatch_tc(const AttnShape& s, const AttnPlan& p, const CUtensorMap& tq,
-                        const CUtensorMap& tk, const CUtensorMap& tv, float* ws_o, float* ws_ml,
-                        int* err, cudaStream_t st) {
-    if (p.mt == 1) {
-        if (p.kt == 192) return run_tc<D, 192, 1>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
-        if (p.kt == 128) return run_tc<D, 128, 1>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
-        return run_tc<D, 64, 1>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
-    }
-    if (p.kt == 128) return run_tc<D, 128, 2>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
-    return run_tc<D, 64, 2>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_splits, hkv * p.n_chunks, batch);
+    cfg.blockDim = dim3(S::THREADS);
+    cfg.dynamicSmemBytes = S::TOTAL;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kfn, tq, tk, tv, a);
 }
 
 }  // namespace
 
-size_t attn_tc_workspace_bytes(const AttnShape& s, int sm_count) {
-    const AttnPlan p = attn_tc_plan(s, sm_count);
-    const size_t rows = (size_t)s.batch * s.n_q_heads * p.n_splits * s.block_len;
-    return rows * (s.head_dim + 2) * sizeof(float);
+size_t attn_tc_workspace_bytes(const AttnShape&, int) {
+    return 16;   // the splits merge on chip; no scratch is needed
 }
-
-cudaError_t launch_attn_combine_bf16(const float* ws_o, const float* ws_ml, void* out, float* lse,
-                                     int batch, int B, int Hq, int D, int n_splits,
-                                     cudaStream_t st);
 
 cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
                                   const void* v, void* out, float* lse, void* ws, int sm_count,
                                   int* err, cudaStream_t st) {
+    (void)ws;
     const AttnPlan p = attn_tc_plan(s, sm_count);
     const int D = s.head_dim;
     CUtensorMap tq, tk, tv;
@@ -335,18 +519,30 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
     cudaError_t e = make_tmap_bf16(&tq, q, 3, qdims, qstr, qbox);
     if (e != cudaSuccess) return e;
     const uint64_t kv_rows = (uint64_t)s.batch * s.n_kv_heads * s.seq_len;
-    e = make_tmap_bf16_2d(&tk, k, kv_rows, D, p.kt, 64);
+    e = make_tmap_bf16_2d(&tk, k, kv_rows, D, ATT_KT, 64);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_2d(&tv, v, kv_rows, D, p.kt, 64);
+    e = make_tmap_bf16_2d(&tv, v, kv_rows, D, ATT_KT, 64);
     if (e != cudaSuccess) return e;
-    float* ws_o = (float*)ws;
-    const size_t rows = (size_t)s.batch * s.n_q_heads * p.n_splits * s.block_len;
-    float* ws_ml = ws_o + rows * D;
-    e = D == 128 ? dispatch_tc<128>(s, p, tq, tk, tv, ws_o, ws_ml, err, st)
-                 : dispatch_tc<64>(s, p, tq, tk, tv, ws_o, ws_ml, err, st);
-    if (e != cudaSuccess) return e;
-    return launch_attn_combine_bf16(ws_o, ws_ml, out, lse, s.batch, s.block_len, s.n_q_heads, D,
-                                    p.n_splits, st);
+    AttnArgs a;
+    a.out = (bf16*)out;
+    a.lse = lse;
+    a.B = s.block_len;
+    a.Hq = s.n_q_heads;
+    a.Hkv = s.n_kv_heads;
+    a.L = s.seq_len;
+    a.hc = p.hc;
+    a.n_chunks = p.n_chunks;
+    a.rows = p.rows;
+    a.tiles = p.tiles;
+    a.tps = p.tps;
+    a.n_splits = p.n_splits;
+    a.scale_log2 = s.scale * 1.4426950408889634f;
+    a.err = err;
+    if (D == 128)
+        return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st)
+                         : run_tc<128, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
+    return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st)
+                     : run_tc<64, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
 }
 
 }  // namespace fdl

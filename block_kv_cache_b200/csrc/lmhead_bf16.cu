@@ -145,10 +145,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int m_tile = item % num_m, n_tile = item / num_m;
             const int row = m_tile * BM + r_in;
             const int n0 = n_tile * BN;
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait(tfull_bar(acc), aphase, abort_flag, err);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
+            if (!mbar_wait_warp(tfull_bar(acc), aphase, abort_flag, err)) break;
             tc_fence_after();
             int bt = -1;
             float bv = 0.f;

@@ -61,19 +61,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete. Returns false
 // (after raising *abort and recording DEV_TIMEOUT) if it does not complete in
 // time, or at once if another thread of the CTA has already given up.
+// The clock and the abort flag are consulted only every 64 polls, so a wait
+// that completes soon costs no more than the try_wait itself.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+    uint32_t n = 0;
+    uint64_t t0 = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > kWaitTimeoutNs) {
-            *abort = 1;
-            record_error(err, DEV_TIMEOUT);
-            return false;
+        if ((++n & 63u) == 0) {
+            if (*abort) return false;
+            const uint64_t now = globaltimer();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitTimeoutNs) {
+                *abort = 1;
+                record_error(err, DEV_TIMEOUT);
+                return false;
+            }
         }
     }
+}
+
+// Whole-warp wait: every lane polls the barrier, then the warp agrees on the
+// outcome (all lanes leave together, also on the give-up path).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int* abort, int* err) {
+    const bool ok = mbar_wait(bar, parity, abort, err);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // 2-D TMA tile load global -> shared, completion counted on `bar` in bytes.
@@ -204,6 +219,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- thread-block clusters --------------------------------------------------------
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// Address in the shared::cluster window of `smem_addr` of CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t smem_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+    return v;
 }
 
 }  // namespace sm100

@@ -5,8 +5,9 @@
         --prefix 512 --block 32 --suffix 224 [--layers 32]
 
 Used to profile a single kernel (e.g. under ncu with -k/-c) and to time it
-with CUDA events. Prints one JSON line: mean µs per call and the achieved
-algorithmic bandwidth / throughput of that call.
+with CUDA events. With --graph the timed calls are captured once in a CUDA
+graph and replayed, so host-side launch cost is excluded. Prints one JSON
+line: mean µs per call and the achieved algorithmic bandwidth / throughput.
 """
 from __future__ import annotations
 
@@ -23,27 +24,45 @@ def _bf16(a):
     return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).cuda()
 
 
+def _timed(a, call):
+    """Mean µs per call of call(i) over a.iters calls (graph-replayed with --graph)."""
+    for i in range(a.warmup):
+        call(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if a.graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(a.iters):
+                call(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(a.reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / (a.iters * a.reps)
+    e0.record()
+    for i in range(a.iters):
+        call(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / a.iters
+
+
 def run_lmhead(a, ctx):
     c = synth.lmhead_case(rows=a.rows, hidden=a.hidden, vocab=a.vocab, seed=1, w_seed=0,
                           mask_id=min(126336, a.vocab - 1))
     h, w = _bf16(c.h), _bf16(c.w)
     bt, bv = torch.from_numpy(c.bias_tok).cuda(), torch.from_numpy(c.bias_val).cuda()
     conf, tok = ctx.lmhead_confidence(h, w, bt, bv)
-    for _ in range(a.warmup):
-        ctx.lmhead_confidence(h, w, bt, bv, conf=conf, tok=tok)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.iters):
-        ctx.lmhead_confidence(h, w, bt, bv, conf=conf, tok=tok)
-    e1.record()
-    torch.cuda.synchronize()
+    us = _timed(a, lambda i: ctx.lmhead_confidence(h, w, bt, bv, conf=conf, tok=tok))
     ctx.device_status()
-    us = e0.elapsed_time(e1) * 1e3 / a.iters
     nbytes = a.vocab * a.hidden * 2 + a.rows * a.hidden * 2 + a.rows * 16
     flops = 2.0 * a.rows * a.hidden * a.vocab
     return {"op": "lmhead_confidence", "rows": a.rows, "hidden": a.hidden, "vocab": a.vocab,
-            "us": us, "GBps": nbytes / us / 1e3, "TFLOPs": flops / us / 1e6}
+            "graph": a.graph, "us": us, "GBps": nbytes / us / 1e3, "TFLOPs": flops / us / 1e6}
 
 
 def run_attention(a, ctx):
@@ -55,24 +74,15 @@ def run_attention(a, ctx):
     vc = [_bf16(c.v_cache) for c in cases]
     out = torch.empty_like(q[0])
     s = a.prefix
-    for l in range(a.layers):
-        ctx.dualcache_attention(q[l], kc[l], vc[l], s, out=out)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for it in range(a.iters):
-        l = it % a.layers
-        ctx.dualcache_attention(q[l], kc[l], vc[l], s, out=out)
-    e1.record()
-    torch.cuda.synchronize()
+    us = _timed(a, lambda i: ctx.dualcache_attention(q[i % a.layers], kc[i % a.layers],
+                                                     vc[i % a.layers], s, out=out))
     ctx.device_status()
-    us = e0.elapsed_time(e1) * 1e3 / a.iters
     L = a.prefix + a.block + a.suffix
     nbytes = (2 * a.batch * a.kv_heads * L * a.head_dim * 2
               + 2 * a.batch * a.block * a.heads * a.head_dim * 2)
     flops = 4.0 * a.batch * a.heads * a.block * L * a.head_dim
     return {"op": "dualcache_attention", "heads": a.heads, "kv_heads": a.kv_heads, "L": L,
-            "block": a.block, "batch": a.batch, "us": us, "GBps": nbytes / us / 1e3,
+            "block": a.block, "batch": a.batch, "graph": a.graph, "us": us, "GBps": nbytes / us / 1e3,
             "TFLOPs": flops / us / 1e6}
 
 
@@ -92,6 +102,8 @@ def main():
     p.add_argument("--layers", type=int, default=32)
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--graph", action="store_true", help="replay the timed calls as a CUDA graph")
+    p.add_argument("--reps", type=int, default=5, help="graph replays timed (with --graph)")
     a = p.parse_args()
     ctx = fdllm.Context(0)
     r = run_lmhead(a, ctx) if a.op == "lmhead" else run_attention(a, ctx)
