@@ -287,3 +287,141 @@ namespace fdl {
 // Record `msg` as the calling thread's last error and return `code`.
 int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
 }  // namespace fdl
+
+// ----------------------------------------------------------------------------
+// transformer scaffold
+// ----------------------------------------------------------------------------
+#include <cmath>
+
+#include "gemm.h"
+
+extern "C" {
+
+int fdl_rope_table(double theta, int max_pos, int head_dim, float* out_host) {
+    if (!out_host || max_pos < 1 || head_dim < 2 || head_dim % 2 || !(theta > 0.0))
+        return fail(FDL_EINVAL, "rope_table: need out, max_pos >= 1, even head_dim, theta > 0");
+    const int half = head_dim / 2;
+    for (int p = 0; p < max_pos; ++p)
+        for (int i = 0; i < half; ++i) {
+            const double ang = (double)p * std::pow(theta, -2.0 * i / head_dim);
+            out_host[((size_t)p * half + i) * 2 + 0] = (float)std::cos(ang);
+            out_host[((size_t)p * half + i) * 2 + 1] = (float)std::sin(ang);
+        }
+    return FDL_OK;
+}
+
+int fdl_rmsnorm(fdl_ctx* ctx, int rows, int hidden, const float* h, const int32_t* row_map,
+                const float* weight, float eps, void* out, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "rmsnorm: ctx is NULL");
+    if (rows < 1 || hidden < 8 || hidden % 8)
+        return fail(FDL_EINVAL, "rmsnorm: rows >= 1 and hidden a multiple of 8 required");
+    if (!h || !weight || !out || !(eps >= 0.f))
+        return fail(FDL_EINVAL, "rmsnorm: NULL buffer or bad eps");
+    if (!aligned16(h) || !aligned16(weight) || !aligned16(out))
+        return fail(FDL_EINVAL, "rmsnorm: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    cudaError_t e = fdl::launch_rmsnorm(rows, hidden, h, row_map, weight, eps, (fdl::bf16*)out,
+                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "rmsnorm launch");
+}
+
+int fdl_embed(fdl_ctx* ctx, int rows, int hidden, const int32_t* ids, const int32_t* row_map,
+              const void* table, float* h, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "embed: ctx is NULL");
+    if (rows < 1 || hidden < 2 || hidden % 2)
+        return fail(FDL_EINVAL, "embed: rows >= 1 and even hidden required");
+    if (!ids || !table || !h) return fail(FDL_EINVAL, "embed: NULL buffer");
+    DeviceGuard g(ctx->device);
+    cudaError_t e = fdl::launch_embed(rows, hidden, ids, row_map, (const fdl::bf16*)table, h,
+                                      (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "embed launch");
+}
+
+int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+                       const float* bias, const float* rope, void* q_out, void* k_cache,
+                       void* v_cache, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "qkv: ctx is NULL");
+    if (!d) return fail(FDL_EINVAL, "qkv: desc is NULL");
+    if (d->head_dim != 128) return fail(FDL_EUNSUPPORTED, "qkv: head_dim must be 128");
+    if (d->rows < 1 || d->hidden < 64 || d->hidden % 64 || d->n_q_heads < 1 ||
+        d->n_kv_heads < 1 || d->batch < 1 || d->seq_len < 1 || d->rows_per_seq < 1 ||
+        d->pos0 < 0 || d->max_pos < 1)
+        return fail(FDL_EINVAL, "qkv: bad shape");
+    if ((d->rows + d->rows_per_seq - 1) / d->rows_per_seq > d->batch)
+        return fail(FDL_EINVAL, "qkv: rows span more than batch sequences");
+    const int last_pos = d->pos0 + (d->rows < d->rows_per_seq ? d->rows : d->rows_per_seq) - 1;
+    if (last_pos >= d->seq_len || last_pos >= d->max_pos)
+        return fail(FDL_EINVAL, "qkv: position %d beyond seq_len %d or rope rows %d", last_pos,
+                    d->seq_len, d->max_pos);
+    if (!x || !w || !rope || !q_out || !k_cache || !v_cache)
+        return fail(FDL_EINVAL, "qkv: NULL buffer");
+    if (!aligned16(x) || !aligned16(w) || !aligned16(q_out) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || !aligned16(rope))
+        return fail(FDL_EINVAL, "qkv: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    fdl::GemmShape gs{d->rows, (d->n_q_heads + 2 * d->n_kv_heads) * 128, d->hidden};
+    fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
+                  (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
+                  d->rows_per_seq, d->pos0};
+    cudaError_t e = fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err,
+                                         (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv launch");
+}
+
+int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_features,
+                        const void* x, const void* w, float* h, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "linear_residual: ctx is NULL");
+    if (rows < 1 || out_features < 64 || out_features % 64 || in_features < 64 ||
+        in_features % 64)
+        return fail(FDL_EINVAL, "linear_residual: rows >= 1, in and out multiples of 64");
+    if (!x || !w || !h) return fail(FDL_EINVAL, "linear_residual: NULL buffer");
+    if (!aligned16(x) || !aligned16(w) || !aligned16(h))
+        return fail(FDL_EINVAL, "linear_residual: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    fdl::GemmShape gs{rows, out_features, in_features};
+    cudaError_t e = fdl::launch_gemm_resid(gs, x, w, fdl::EpiResid{h, out_features},
+                                           ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_residual launch");
+}
+
+int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features, const void* x,
+                      const void* w_gu, void* out, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "linear_swiglu: ctx is NULL");
+    if (rows < 1 || out_features < 32 || out_features % 32 || in_features < 64 ||
+        in_features % 64)
+        return fail(FDL_EINVAL, "linear_swiglu: rows >= 1, out % 32 == 0, in % 64 == 0");
+    if (!x || !w_gu || !out) return fail(FDL_EINVAL, "linear_swiglu: NULL buffer");
+    if (!aligned16(x) || !aligned16(w_gu) || !aligned16(out))
+        return fail(FDL_EINVAL, "linear_swiglu: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    fdl::GemmShape gs{rows, 2 * out_features, in_features};
+    cudaError_t e = fdl::launch_gemm_swiglu(gs, x, w_gu, fdl::EpiSwiGLU{(fdl::bf16*)out,
+                                            out_features}, ctx->sm_count, ctx->d_err,
+                                            (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_swiglu launch");
+}
+
+int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
+                       const void* k_cache, const void* v_cache, void* out, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "full_attention: ctx is NULL");
+    if (!desc) return fail(FDL_EINVAL, "full_attention: desc is NULL");
+    if (desc->dtype != FDL_BF16) return fail(FDL_EUNSUPPORTED, "full_attention: bf16 only");
+    if (desc->head_dim != 64 && desc->head_dim != 128)
+        return fail(FDL_EUNSUPPORTED, "full_attention: head_dim %d", desc->head_dim);
+    if (desc->batch < 1 || desc->n_q_heads < 1 || desc->n_kv_heads < 1 ||
+        desc->n_q_heads % desc->n_kv_heads || desc->seq_len < 32 || desc->seq_len % 32)
+        return fail(FDL_EINVAL, "full_attention: bad shape (seq_len a multiple of 32)");
+    if (!q || !k_cache || !v_cache || !out) return fail(FDL_EINVAL, "full_attention: NULL");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(FDL_EINVAL, "full_attention: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    const float scale = desc->scale == 0.f ? 1.0f / sqrtf((float)desc->head_dim) : desc->scale;
+    cudaError_t e = fdl::launch_full_attention_bf16(desc->batch, desc->n_q_heads,
+                                                    desc->n_kv_heads, desc->head_dim,
+                                                    desc->seq_len, scale, q, k_cache, v_cache,
+                                                    out, ctx->sm_count, ctx->d_err,
+                                                    (cudaStream_t)stream);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "full_attention launch");
+}
+
+}  // extern "C"

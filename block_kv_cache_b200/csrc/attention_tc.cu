@@ -143,7 +143,7 @@ __device__ __forceinline__ float ex2(float x) {
 struct AttnArgs {
     bf16* out;
     float* lse;         // optional
-    int B, Hq, Hkv, L, hc, n_chunks, rows, tiles, tps, n_splits;
+    int B, Hq, Hkv, L, hc, n_chunks, rows, tiles, tps, n_splits, q_per_kv;
     float scale_log2;
     int* err;
 };
@@ -219,7 +219,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int dc = 0; dc < S::DC; ++dc)
                 tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
                             bb * a.B);
-            const int krow0 = (bb * a.Hkv + g) * a.L + k_begin;
+            const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
             int t = 0;
             for (; ok && t < nt; ++t) {
                 const int st = t % STAGES;
@@ -518,7 +518,7 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
     const uint32_t qbox[3] = {64, (uint32_t)p.hc, (uint32_t)s.block_len};
     cudaError_t e = make_tmap_bf16(&tq, q, 3, qdims, qstr, qbox);
     if (e != cudaSuccess) return e;
-    const uint64_t kv_rows = (uint64_t)s.batch * s.n_kv_heads * s.seq_len;
+    const uint64_t kv_rows = (uint64_t)(s.batch / s.q_per_kv) * s.n_kv_heads * s.seq_len;
     e = make_tmap_bf16_2d(&tk, k, kv_rows, D, ATT_KT, 64);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_2d(&tv, v, kv_rows, D, ATT_KT, 64);
@@ -536,6 +536,7 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
     a.tiles = p.tiles;
     a.tps = p.tps;
     a.n_splits = p.n_splits;
+    a.q_per_kv = s.q_per_kv;
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
     if (D == 128)
@@ -543,6 +544,20 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
                          : run_tc<128, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
     return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st)
                      : run_tc<64, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
+}
+
+cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                       int seq_len, float scale, const void* q, const void* k,
+                                       const void* v, void* out, int sm_count, int* dev_err,
+                                       cudaStream_t st) {
+    // query blocks of Bq rows: as many whole heads of a GQA group per 256 rows
+    const int grp = n_q_heads / n_kv_heads;
+    int bq = grp == 1 ? 128 : grp == 2 ? 128 : grp <= 4 ? 64 : 32;
+    while (bq > 32 && seq_len % bq) bq /= 2;
+    if (seq_len % bq) return cudaErrorInvalidValue;
+    AttnShape s{batch * (seq_len / bq), n_q_heads, n_kv_heads, head_dim, seq_len, 0, bq, scale,
+                1, seq_len / bq};
+    return launch_attention_bf16(s, q, k, v, out, nullptr, nullptr, sm_count, dev_err, st);
 }
 
 }  // namespace fdl

@@ -1,0 +1,49 @@
+// Host-side interface of the fused-epilogue GEMMs (gemm_bf16.cu) and the
+// row-wise kernels of the transformer scaffold (norm.cu).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace fdl {
+
+struct GemmShape { int M, N, K; };
+
+struct EpiResid {            // h[M, N] (f32, row stride ldh) += A W^T
+    float* h;
+    int ldh;
+};
+
+struct EpiSwiGLU {           // out[M, N/2] (bf16, row stride ldo)
+    bf16* out;
+    int ldo;
+};
+
+struct EpiQKV {              // N = (n_q_heads + 2 n_kv_heads) * 128
+    bf16* q;                 // [M, n_q_heads, 128]
+    bf16* k_cache;           // [b, n_kv_heads, seq_len, 128]
+    bf16* v_cache;
+    const float* bias;       // [N] or null
+    const float2* rope;      // [max_pos, 64] (cos, sin)
+    int n_q_heads, n_kv_heads, seq_len;
+    int rows_per_seq;        // row r belongs to sequence r / rows_per_seq ...
+    int pos0;                // ... at position pos0 + r % rows_per_seq
+};
+
+cudaError_t launch_gemm_resid(const GemmShape& g, const void* a, const void* w,
+                              const EpiResid& p, int sm_count, int* err, cudaStream_t st);
+cudaError_t launch_gemm_swiglu(const GemmShape& g, const void* a, const void* w,
+                               const EpiSwiGLU& p, int sm_count, int* err, cudaStream_t st);
+cudaError_t launch_gemm_qkv(const GemmShape& g, const void* a, const void* w, const EpiQKV& p,
+                            int sm_count, int* err, cudaStream_t st);
+
+// out[i, :] = bf16(h[src_i, :] / sqrt(mean(h[src_i]^2) + eps) * weight), src_i =
+// row_map ? row_map[i] : i.
+cudaError_t launch_rmsnorm(int rows, int hidden, const float* h, const int32_t* row_map,
+                           const float* weight, float eps, bf16* out, cudaStream_t st);
+// h[i, :] = f32(table[ids[j], :]), j = row_map ? row_map[i] : i
+cudaError_t launch_embed(int rows, int hidden, const int32_t* ids, const int32_t* row_map,
+                         const bf16* table, float* h, cudaStream_t st);
+
+}  // namespace fdl

@@ -10,6 +10,8 @@ struct AttnShape {
     int batch, n_q_heads, n_kv_heads, head_dim, seq_len, block_start, block_len;
     float scale;  // resolved (never 0)
     int bf16;     // 1: bf16 tensors (tcgen05 kernel), 0: f32 (SIMT kernel)
+    int q_per_kv = 1;   // query blocks per sequence: batch counts query blocks,
+                        // sequence index = batch index / q_per_kv (full attention)
 };
 
 // Scratch for the split-KV partials of either attention kernel.
@@ -22,6 +24,13 @@ cudaError_t launch_attention_f32(const AttnShape& s, const float* q, const float
 cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
                                   const void* v, void* out, float* lse, void* ws,
                                   int sm_count, int* dev_err, cudaStream_t st);
+
+// Full bidirectional attention of every position of every sequence (the
+// refresh forward): q, out [b, L, Hq, d] bf16; caches [b, Hkv, L, d].
+cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                       int seq_len, float scale, const void* q, const void* k,
+                                       const void* v, void* out, int sm_count, int* dev_err,
+                                       cudaStream_t st);
 
 cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len,
                             int elem_bytes, const void* k_new, const void* v_new,

@@ -27,7 +27,9 @@ EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
            "fdl_get_device_status", "fdl_attention_workspace_bytes",
            "fdl_dualcache_attention", "fdl_kv_store", "fdl_lmhead_workspace_bytes",
            "fdl_lmhead_confidence", "fdl_threshold_unmask",
-           "fdl_lmhead_confidence_noalloc")
+           "fdl_lmhead_confidence_noalloc", "fdl_rope_table", "fdl_rmsnorm", "fdl_embed",
+           "fdl_qkv_rope_store", "fdl_linear_residual", "fdl_linear_swiglu",
+           "fdl_full_attention")
 
 
 class AttnDesc(ctypes.Structure):
@@ -47,6 +49,14 @@ class UnmaskDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("seq_len", ctypes.c_int),
                 ("block_start", ctypes.c_int), ("block_len", ctypes.c_int),
                 ("tau", ctypes.c_float)]
+
+
+class QKVDesc(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("hidden", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("batch", ctypes.c_int), ("seq_len", ctypes.c_int),
+                ("rows_per_seq", ctypes.c_int), ("pos0", ctypes.c_int),
+                ("max_pos", ctypes.c_int)]
 
 
 class FdlError(RuntimeError):
@@ -85,6 +95,13 @@ def load() -> ctypes.CDLL:
                                                 vp, vp, vp]
     L.fdl_threshold_unmask.argtypes = [vp, ctypes.POINTER(UnmaskDesc), vp, vp, vp, vp, vp,
                                        vp, vp]
+    L.fdl_rope_table.argtypes = [ctypes.c_double, i, i, vp]
+    L.fdl_rmsnorm.argtypes = [vp, i, i, vp, vp, vp, ctypes.c_float, vp, vp]
+    L.fdl_embed.argtypes = [vp, i, i, vp, vp, vp, vp, vp]
+    L.fdl_qkv_rope_store.argtypes = [vp, ctypes.POINTER(QKVDesc), vp, vp, vp, vp, vp, vp, vp, vp]
+    L.fdl_linear_residual.argtypes = [vp, i, i, i, vp, vp, vp, vp]
+    L.fdl_linear_swiglu.argtypes = [vp, i, i, i, vp, vp, vp, vp]
+    L.fdl_full_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -122,6 +139,16 @@ def _need(t: torch.Tensor, name: str, dtype=None, ndim=None):
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def rope_table(theta: float, max_pos: int, head_dim: int):
+    """(cos, sin) table of rotate-half RoPE as a host float32 array [max_pos, head_dim/2, 2]
+    (computed by the library in double precision)."""
+    import numpy as np
+    out = np.empty((max_pos, head_dim // 2, 2), np.float32)
+    _check(load().fdl_rope_table(float(theta), int(max_pos), int(head_dim),
+                                 ctypes.c_void_p(out.ctypes.data)))
+    return out
 
 
 class Context:
@@ -260,3 +287,71 @@ class Context:
                                            _ptr(x), _ptr(masked), _ptr(remaining),
                                            _ptr(n_decoded), _stream(stream)))
         return remaining
+
+    # -- transformer scaffold ------------------------------------------------
+    def rmsnorm(self, h, weight, eps, *, out=None, row_map=None, rows=None, stream=None):
+        """bf16 RMSNorm of f32 rows of h (optionally gathered through row_map)."""
+        _need(h, "h", torch.float32, 2)
+        _need(weight, "weight", torch.float32, 1)
+        n = rows if rows is not None else (row_map.numel() if row_map is not None else h.shape[0])
+        if out is None:
+            out = torch.empty((n, h.shape[1]), dtype=torch.bfloat16, device=h.device)
+        _check(load().fdl_rmsnorm(self._h, int(n), h.shape[1], _ptr(h), _ptr(row_map),
+                                  _ptr(weight), float(eps), _ptr(out), _stream(stream)))
+        return out
+
+    def embed(self, ids, table, *, out=None, row_map=None, stream=None):
+        """f32 rows of the embedding table: table[ids[row_map[i]]] (or ids[i])."""
+        _need(ids, "ids", torch.int32, None)
+        _need(table, "table", torch.bfloat16, 2)
+        n = row_map.numel() if row_map is not None else ids.numel()
+        if out is None:
+            out = torch.empty((n, table.shape[1]), dtype=torch.float32, device=ids.device)
+        _check(load().fdl_embed(self._h, int(n), table.shape[1], _ptr(ids), _ptr(row_map),
+                                _ptr(table), _ptr(out), _stream(stream)))
+        return out
+
+    def qkv_rope_store(self, x, w, rope, q_out, k_cache, v_cache, *, n_q_heads, rows_per_seq,
+                       pos0, bias=None, stream=None):
+        """[q|k|v] = x w^T (+bias), RoPE on q and k, q -> q_out, k/v -> caches."""
+        _need(x, "x", torch.bfloat16, 2)
+        _need(w, "w", torch.bfloat16, 2)
+        b, hkv, L, d = k_cache.shape
+        d_ = QKVDesc(x.shape[0], x.shape[1], int(n_q_heads), hkv, d, b, L, int(rows_per_seq),
+                     int(pos0), rope.shape[0])
+        _check(load().fdl_qkv_rope_store(self._h, ctypes.byref(d_), _ptr(x), _ptr(w),
+                                         _ptr(bias), _ptr(rope), _ptr(q_out), _ptr(k_cache),
+                                         _ptr(v_cache), _stream(stream)))
+        return q_out
+
+    def linear_residual(self, x, w, h, *, stream=None):
+        """h += x w^T (h f32)."""
+        _need(x, "x", torch.bfloat16, 2)
+        _need(w, "w", torch.bfloat16, 2)
+        _need(h, "h", torch.float32, 2)
+        _check(load().fdl_linear_residual(self._h, x.shape[0], w.shape[0], x.shape[1], _ptr(x),
+                                          _ptr(w), _ptr(h), _stream(stream)))
+        return h
+
+    def linear_swiglu(self, x, w_gu, *, out=None, stream=None):
+        """silu(x Wg^T) * (x Wu^T) with gate/up rows interleaved in w_gu."""
+        _need(x, "x", torch.bfloat16, 2)
+        _need(w_gu, "w_gu", torch.bfloat16, 2)
+        F = w_gu.shape[0] // 2
+        if out is None:
+            out = torch.empty((x.shape[0], F), dtype=torch.bfloat16, device=x.device)
+        _check(load().fdl_linear_swiglu(self._h, x.shape[0], F, x.shape[1], _ptr(x), _ptr(w_gu),
+                                        _ptr(out), _stream(stream)))
+        return out
+
+    def full_attention(self, q, k_cache, v_cache, *, out=None, scale=0.0, stream=None):
+        """Bidirectional attention of every position: q, out [b, L, Hq, d]."""
+        _need(q, "q", torch.bfloat16, 4)
+        b, L, Hq, d = q.shape
+        hkv = k_cache.shape[1]
+        desc = AttnDesc(b, Hq, hkv, d, L, 0, 1, FDL_BF16, float(scale))
+        if out is None:
+            out = torch.empty_like(q)
+        _check(load().fdl_full_attention(self._h, ctypes.byref(desc), _ptr(q), _ptr(k_cache),
+                                         _ptr(v_cache), _ptr(out), _stream(stream)))
+        return out

@@ -1,0 +1,252 @@
+"""Fast-dLLM block decoding of a LLaDA / Dream-shaped bidirectional
+transformer on the GPU, driven through the C-ABI library.
+
+Every arithmetic step runs in libfdllm.so kernels; this module only holds the
+device buffers (torch allocations) and issues the calls in order:
+
+  refresh (a full forward over all L positions; Fast-dLLM recomputes every
+  position's K/V once a block completes - ICLR reviews, review 4 question 2):
+      embed -> per layer [RMSNorm -> QKV + RoPE written into the K/V caches
+      (every row) -> full attention -> O proj + residual -> RMSNorm -> SwiGLU
+      -> down proj + residual] -> final RMSNorm of the current block's rows
+      -> LM head confidence -> threshold unmask
+  cached block step (DualCache; aibase news "Innovations" 1):
+      the same per layer, but only the block's B rows go through the layers:
+      their K/V overwrite the cache slot and the block attends over the whole
+      cache [prefix | block | masked suffix]
+
+Layouts: weights are stored [out, in] (K-major); the gate and up projections
+are interleaved by rows (row 2f = gate f, 2f+1 = up f) so the SwiGLU
+epilogue finds both halves of a feature in one tile.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import fdllm
+
+
+@dataclass
+class ModelShape:
+    vocab: int
+    hidden: int
+    n_layers: int
+    n_q_heads: int
+    n_kv_heads: int
+    ffn: int
+    mask_id: int
+    head_dim: int = 128
+    rope_theta: float = 10000.0
+    rms_eps: float = 1e-5
+    qkv_bias: bool = False
+
+
+def _bf16(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).to(dev)
+
+
+def _f32(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+
+
+class DeviceWeights:
+    """bf16 weights (f32 norms and biases) on one device."""
+
+    def __init__(self, shape: ModelShape, layers, embed, final_norm, lm_head):
+        self.shape = shape
+        self.layers = layers
+        self.embed = embed
+        self.final_norm = final_norm
+        self.lm_head = lm_head
+
+    @staticmethod
+    def from_params(P, device="cuda") -> "DeviceWeights":
+        """From synth.ModelParams (host float32 values exact in bf16)."""
+        sh = ModelShape(P.vocab, P.hidden, P.n_layers, P.n_q_heads, P.n_kv_heads, P.ffn,
+                        P.mask_id, P.head_dim, P.rope_theta, P.rms_eps, P.qkv_bias)
+        layers = []
+        for Lw in P.layers:
+            wgu = np.empty((2 * P.ffn, P.hidden), np.float32)
+            wgu[0::2] = Lw["wg"]
+            wgu[1::2] = Lw["wu"]
+            d = dict(attn_norm=_f32(Lw["attn_norm"], device),
+                     w_qkv=_bf16(np.concatenate([Lw["wq"], Lw["wk"], Lw["wv"]]), device),
+                     wo=_bf16(Lw["wo"], device), ffn_norm=_f32(Lw["ffn_norm"], device),
+                     w_gu=_bf16(wgu, device), wd=_bf16(Lw["wd"], device), bias=None)
+            if P.qkv_bias:
+                d["bias"] = _f32(np.concatenate([Lw["bq"], Lw["bk"], Lw["bv"]]), device)
+            layers.append(d)
+        return DeviceWeights(sh, layers, _bf16(P.embed, device), _f32(P.final_norm, device),
+                             _bf16(P.lm_head, device))
+
+    @staticmethod
+    def random(shape: ModelShape, seed=0, device="cuda", w_std=0.02) -> "DeviceWeights":
+        """Seeded random-init weights drawn on the device (for full-size runs whose
+        weights would take minutes to draw on the host). Norm weights are 1."""
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        D, F, d = shape.hidden, shape.ffn, shape.head_dim
+        nqkv = (shape.n_q_heads + 2 * shape.n_kv_heads) * d
+
+        def rnd(*sz):
+            return (torch.randn(*sz, generator=g, device=device, dtype=torch.float32)
+                    * w_std).to(torch.bfloat16)
+
+        layers = []
+        for _ in range(shape.n_layers):
+            layers.append(dict(
+                attn_norm=torch.ones(D, device=device), w_qkv=rnd(nqkv, D),
+                wo=rnd(D, shape.n_q_heads * d), ffn_norm=torch.ones(D, device=device),
+                w_gu=rnd(2 * F, D), wd=rnd(D, F),
+                bias=(torch.randn(nqkv, generator=g, device=device) * w_std)
+                if shape.qkv_bias else None))
+        embed = (torch.randn(shape.vocab, D, generator=g, device=device)).to(torch.bfloat16)
+        return DeviceWeights(shape, layers, embed, torch.ones(D, device=device),
+                             rnd(shape.vocab, D))
+
+    def nbytes(self) -> int:
+        n = self.embed.numel() * 2 + self.lm_head.numel() * 2
+        for L in self.layers:
+            n += sum(t.numel() * t.element_size() for t in L.values() if t is not None)
+        return n
+
+
+class BlockDecoder:
+    """DualCache + threshold decoding of `batch` sequences of length seq_len."""
+
+    def __init__(self, ctx: fdllm.Context, w: DeviceWeights, batch: int, seq_len: int,
+                 block: int = 32, device="cuda"):
+        sh = w.shape
+        self.ctx, self.w, self.sh = ctx, w, sh
+        self.b, self.L, self.B = batch, seq_len, block
+        dev = device
+        D, d = sh.hidden, sh.head_dim
+        self.rope = torch.from_numpy(fdllm.rope_table(sh.rope_theta, seq_len, d)).to(dev)
+        self.kc = [torch.zeros((batch, sh.n_kv_heads, seq_len, d), dtype=torch.bfloat16,
+                               device=dev) for _ in range(sh.n_layers)]
+        self.vc = [torch.zeros_like(k) for k in self.kc]
+        rows_full = batch * seq_len
+        self.h_full = torch.empty((rows_full, D), dtype=torch.float32, device=dev)
+        self.x_full = torch.empty((rows_full, D), dtype=torch.bfloat16, device=dev)
+        self.q_full = torch.empty((rows_full, sh.n_q_heads, d), dtype=torch.bfloat16, device=dev)
+        self.o_full = torch.empty_like(self.q_full)
+        self.f_full = torch.empty((rows_full, sh.ffn), dtype=torch.bfloat16, device=dev)
+        rb = batch * block
+        self.h_blk = torch.empty((rb, D), dtype=torch.float32, device=dev)
+        self.x_blk = torch.empty((rb, D), dtype=torch.bfloat16, device=dev)
+        self.q_blk = torch.empty((rb, sh.n_q_heads, d), dtype=torch.bfloat16, device=dev)
+        self.o_blk = torch.empty_like(self.q_blk)
+        self.f_blk = torch.empty((rb, sh.ffn), dtype=torch.bfloat16, device=dev)
+        self.xn = torch.empty((rb, D), dtype=torch.bfloat16, device=dev)
+        self.conf = torch.empty(rb, dtype=torch.float32, device=dev)
+        self.tok = torch.empty(rb, dtype=torch.int32, device=dev)
+        self.remaining = torch.empty(batch, dtype=torch.int32, device=dev)
+        self.n_decoded = torch.empty(batch, dtype=torch.int32, device=dev)
+        # rows of block k of every sequence in the flattened [b * L] token rows
+        nblk = (seq_len + block - 1) // block
+        i = np.arange(block)
+        maps = np.stack([(np.arange(batch)[:, None] * seq_len + k * block + i[None, :]).reshape(-1)
+                         for k in range(nblk)]).astype(np.int32)
+        self.row_maps = torch.from_numpy(np.minimum(maps, batch * seq_len - 1)).to(dev)
+        lmd = fdllm.LMHeadDesc(rb, D, sh.vocab, fdllm.FDL_BF16)
+        self.ws_lm = torch.empty(max(ctx.lmhead_workspace_bytes(lmd), 16), dtype=torch.uint8,
+                                 device=dev)
+        ad = fdllm.AttnDesc(batch, sh.n_q_heads, sh.n_kv_heads, d, seq_len, 0, block,
+                            fdllm.FDL_BF16, 0.0)
+        self.ws_att = torch.empty(max(ctx.attention_workspace_bytes(ad), 16), dtype=torch.uint8,
+                                  device=dev)
+
+    # ------------------------------------------------------------------ layers
+    def _layers(self, h, x, q, o, f, rows, rows_per_seq, pos0, full):
+        ctx, sh = self.ctx, self.sh
+        for li, Lw in enumerate(self.w.layers):
+            ctx.rmsnorm(h, Lw["attn_norm"], sh.rms_eps, out=x)
+            ctx.qkv_rope_store(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
+                               n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
+                               bias=Lw["bias"])
+            if full:
+                ctx.full_attention(q.view(self.b, self.L, sh.n_q_heads, sh.head_dim),
+                                   self.kc[li], self.vc[li],
+                                   out=o.view(self.b, self.L, sh.n_q_heads, sh.head_dim))
+            else:
+                ctx.dualcache_attention(q.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
+                                        self.kc[li], self.vc[li], pos0,
+                                        out=o.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
+                                        ws=self.ws_att)
+            ctx.linear_residual(o.view(rows, -1), Lw["wo"], h)
+            ctx.rmsnorm(h, Lw["ffn_norm"], sh.rms_eps, out=x)
+            ctx.linear_swiglu(x, Lw["w_gu"], out=f)
+            ctx.linear_residual(f, Lw["wd"], h)
+
+    def refresh(self, x_ids, s):
+        """Full forward over all positions of x_ids [b, L] (int32, device): rewrites
+        every layer's K/V cache and leaves conf/tok for the rows of block [s, s+B)."""
+        rows = self.b * self.L
+        self.ctx.embed(x_ids.view(-1), self.w.embed, out=self.h_full)
+        self._layers(self.h_full, self.x_full, self.q_full, self.o_full, self.f_full, rows,
+                     self.L, 0, True)
+        self.ctx.rmsnorm(self.h_full, self.w.final_norm, self.sh.rms_eps, out=self.xn,
+                         row_map=self._row_map(s))
+        self._confidence()
+
+    def block_step(self, x_ids, s):
+        """Cached DualCache step for block [s, s+B) of x_ids [b, L]."""
+        rows = self.b * self.B
+        self.ctx.embed(x_ids, self.w.embed, out=self.h_blk, row_map=self._row_map(s))
+        self._layers(self.h_blk, self.x_blk, self.q_blk, self.o_blk, self.f_blk, rows, self.B,
+                     s, False)
+        self.ctx.rmsnorm(self.h_blk, self.w.final_norm, self.sh.rms_eps, out=self.xn)
+        self._confidence()
+
+    def _row_map(self, s):
+        assert s % self.B == 0, "blocks start at multiples of the block size"
+        return self.row_maps[s // self.B]
+
+    def _confidence(self):
+        self.ctx.lmhead_confidence(self.xn, self.w.lm_head, conf=self.conf, tok=self.tok,
+                                   ws=self.ws_lm)
+
+    def unmask(self, x_ids, masked, s, tau):
+        self.ctx.threshold_unmask(self.conf.view(self.b, self.B), self.tok.view(self.b, self.B),
+                                  x_ids, masked, s, tau, remaining=self.remaining,
+                                  n_decoded=self.n_decoded)
+
+    # ------------------------------------------------------------------ decode
+    def generate(self, prompt, gen_len, tau=0.9, record=None):
+        """Decode gen_len tokens after prompt [b, P] (host or device int32) with
+        DualCache and the threshold rule. Returns (x [b, L] int32 device, steps).
+        If `record` is a list, each step appends (kind, s, x_before, masked_before,
+        conf, tok) as host arrays (for step-wise checks)."""
+        b, P = prompt.shape
+        assert P + gen_len == self.L and gen_len % self.B == 0
+        dev = self.h_full.device
+        x = torch.full((b, self.L), self.sh.mask_id, dtype=torch.int32, device=dev)
+        x[:, :P] = torch.as_tensor(prompt, dtype=torch.int32, device=dev)
+        masked = torch.zeros((b, self.L), dtype=torch.uint8, device=dev)
+        masked[:, P:] = 1
+        steps = 0
+        host_rem = torch.empty(b, dtype=torch.int32).pin_memory()
+        for blk in range(gen_len // self.B):
+            s = P + blk * self.B
+            kind = "refresh"
+            while True:
+                if record is not None:
+                    xb, mb = x.cpu().numpy(), masked.cpu().numpy()
+                if kind == "refresh":
+                    self.refresh(x, s)
+                else:
+                    self.block_step(x, s)
+                if record is not None:
+                    record.append((kind, s, xb, mb, self.conf.cpu().numpy().copy(),
+                                   self.tok.cpu().numpy().copy()))
+                self.unmask(x, masked, s, tau)
+                steps += 1
+                host_rem.copy_(self.remaining, non_blocking=True)
+                torch.cuda.current_stream().synchronize()
+                if int(host_rem.max()) == 0:
+                    break
+                kind = "cached"
+        return x, steps

@@ -236,6 +236,85 @@ FDL_API int fdl_threshold_unmask(fdl_ctx* ctx, const fdl_unmask_desc* desc,
                          uint8_t* masked, int32_t* remaining,
                          int32_t* n_decoded, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Transformer scaffold of the LLaDA / Dream family (pre-norm, bidirectional):
+ * the projections that produce the block's K/V (a cached step) or every
+ * position's K/V (a refresh), RMSNorm, SwiGLU FFN, residual stream. All GEMMs
+ * are bf16 on tcgen05 with f32 accumulation; the residual stream is f32.
+ * ------------------------------------------------------------------------ */
+
+/* Rotary table for rotate-half RoPE: out_host[p][i] = (cos, sin) of
+ * p * theta^(-2i/head_dim), p in [0, max_pos), i in [0, head_dim/2), computed
+ * in double and rounded to float. out_host holds max_pos*head_dim floats.
+ * Host-only; errors: FDL_EINVAL. */
+FDL_API int fdl_rope_table(double theta, int max_pos, int head_dim, float* out_host);
+
+/* out[i, :] = bf16( h[src, :] / sqrt(mean(h[src, :]^2) + eps) * weight ),
+ * src = row_map ? row_map[i] : i.
+ *   h [*, hidden] f32 device; row_map [rows] int32 device or NULL;
+ *   weight [hidden] f32 device; out [rows, hidden] bf16 device.
+ * hidden % 8 == 0. Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_rmsnorm(fdl_ctx* ctx, int rows, int hidden, const float* h,
+                        const int32_t* row_map, const float* weight, float eps, void* out,
+                        void* stream);
+
+/* h[i, :] = f32(table[ids[j], :]), j = row_map ? row_map[i] : i (row_map
+ * lets a cached step embed the block's tokens straight out of x [b, L]).
+ * ids int32, row_map [rows] int32 or NULL, table [V, hidden] bf16,
+ * h [rows, hidden] f32 (all device). Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_embed(fdl_ctx* ctx, int rows, int hidden, const int32_t* ids,
+                      const int32_t* row_map, const void* table, float* h, void* stream);
+
+typedef struct {
+    int rows;          /* M token rows of x */
+    int hidden;        /* K, multiple of 64 */
+    int n_q_heads;     /* q heads; N = (n_q_heads + 2 n_kv_heads) * head_dim */
+    int n_kv_heads;
+    int head_dim;      /* 128 */
+    int batch;         /* sequences in the caches */
+    int seq_len;       /* L, cache rows per (sequence, kv head) */
+    int rows_per_seq;  /* row r is sequence r / rows_per_seq ... */
+    int pos0;          /* ... at position pos0 + r % rows_per_seq */
+    int max_pos;       /* rows of the rope table, > every position used */
+} fdl_qkv_desc;
+
+/* Block-slot (or, at a refresh, full) projection with rotary embedding and
+ * in-place cache write (Fast-dLLM DualCache: at a cached step only the
+ * current block is recomputed; aibase news "Innovations" 1; a refresh
+ * recomputes every position, ICLR reviews, review 4 question 2).
+ *   [q | k | v] = x w^T (+ bias); q, k rotated (rotate-half RoPE) at their
+ *   absolute positions; q -> q_out [rows, n_q_heads, head_dim];
+ *   k, v -> k_cache / v_cache [batch, n_kv_heads, seq_len, head_dim] at rows
+ *   (sequence, position); other cache rows untouched.
+ *   x [rows, hidden] bf16; w [N, hidden] bf16 (q heads, then k, then v);
+ *   bias [N] f32 or NULL; rope = fdl_rope_table output on the device.
+ * Errors: FDL_EINVAL (shapes, positions beyond seq_len or max_pos,
+ * alignment), FDL_EUNSUPPORTED (head_dim != 128), FDL_ECUDA. */
+FDL_API int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* desc, const void* x,
+                               const void* w, const float* bias, const float* rope,
+                               void* q_out, void* k_cache, void* v_cache, void* stream);
+
+/* h[rows, out_features] += x w^T  (f32 residual stream; x bf16 [rows, in],
+ * w bf16 [out, in]). in % 64 == 0, out % 64 == 0. Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_features,
+                                const void* x, const void* w, float* h, void* stream);
+
+/* out[rows, out_features] = silu(x Wg^T) * (x Wu^T), bf16, with the gate and
+ * up weights interleaved by rows: w_gu [2*out_features, in], row 2f = gate
+ * row f, row 2f+1 = up row f. in % 64 == 0, out_features % 32 == 0.
+ * Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
+                              const void* x, const void* w_gu, void* out, void* stream);
+
+/* Full bidirectional attention of every position (the refresh forward after
+ * a block completes): out[b, i, h, :] = softmax over all j of q_i . k_j.
+ *   q, out [b, L, Hq, d] bf16; caches [b, Hkv, L, d] bf16 (desc->dtype must
+ *   be FDL_BF16; block_start/block_len are ignored). L % 32 == 0.
+ * Errors: FDL_EINVAL, FDL_EUNSUPPORTED, FDL_ECUDA. */
+FDL_API int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
+                               const void* k_cache, const void* v_cache, void* out,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

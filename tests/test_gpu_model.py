@@ -1,0 +1,233 @@
+"""Parity of the transformer scaffold and of whole DualCache decodes with the
+CPU oracle, through the C-ABI.
+
+Per-op tolerances: bf16 outputs max|gpu - ref| / max|ref| <= 2e-2 (one bf16
+rounding, 2^-9 relative, plus f32 accumulation); f32 outputs (the residual
+stream) <= 1e-4 relative; copies and gathers bit-exact.
+
+Whole decodes are checked step by step with the oracle replaying the GPU's
+own trajectory (same tokens before every step, caches refreshed at the same
+points): confidences agree within CONF_MODEL_TOL, which allows for the bf16
+rounding of activations between kernels that the float64 oracle does not
+have; token ids agree wherever the oracle's top-2 logit gap exceeds 0.05;
+the unmask decisions are bit-exact given the GPU's confidences.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from block_kv_cache_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 2e-2
+CONF_MODEL_TOL = 2e-2
+TOK_GAP = 0.05
+
+
+@pytest.fixture(scope="module")
+def ctx():
+    from block_kv_cache_b200 import fdllm
+    c = fdllm.Context(0)
+    yield c
+    c.close()
+
+
+def bf(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).cuda()
+
+
+def f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def rel(g, r):
+    return float(np.abs(g - r).max() / max(np.abs(r).max(), 1e-30))
+
+
+def bf_vals(a):
+    return synth.bf16_value(synth.bf16_bits(np.asarray(a, np.float32)))
+
+
+# ------------------------------------------------------------------ single ops
+def test_rmsnorm_with_row_map(ctx):
+    g = synth.rng(1)
+    h = (g.standard_normal((300, 1024)) * 3).astype(np.float32)
+    w = g.uniform(0.5, 1.5, 1024).astype(np.float32)
+    rm = g.integers(0, 300, 77).astype(np.int32)
+    out = ctx.rmsnorm(f32(h), f32(w), 1e-5, row_map=torch.from_numpy(rm).cuda())
+    ref = O.rms_norm(h[rm], w, 1e-5)
+    assert rel(out.float().cpu().numpy(), ref) <= BF16_TOL
+
+
+def test_embed_gather_exact(ctx):
+    g = synth.rng(2)
+    table = bf_vals(g.standard_normal((500, 256)))
+    ids = g.integers(0, 500, (3, 40)).astype(np.int32)
+    rm = np.array([0, 5, 39, 40, 119, 7], np.int32)
+    out = ctx.embed(torch.from_numpy(ids).cuda(), bf(table), row_map=torch.from_numpy(rm).cuda())
+    assert np.array_equal(out.cpu().numpy(), table[ids.reshape(-1)[rm]])
+
+
+@pytest.mark.parametrize("M,N,K", [(32, 4096, 4096), (300, 512, 256), (1, 64, 64), (129, 320, 192)])
+def test_linear_residual(ctx, M, N, K):
+    g = synth.rng(M + N)
+    x = bf_vals(g.standard_normal((M, K)))
+    w = bf_vals(g.standard_normal((N, K)) * 0.02)
+    h0 = g.standard_normal((M, N)).astype(np.float32)
+    h = f32(h0)
+    ctx.linear_residual(bf(x), bf(w), h)
+    ref = h0.astype(np.float64) + x.astype(np.float64) @ w.astype(np.float64).T
+    assert rel(h.cpu().numpy(), ref) <= 1e-4
+
+
+@pytest.mark.parametrize("M,F,K", [(32, 1024, 512), (257, 96, 128)])
+def test_linear_swiglu(ctx, M, F, K):
+    g = synth.rng(M + F)
+    x = bf_vals(g.standard_normal((M, K)))
+    wg = bf_vals(g.standard_normal((F, K)) * 0.05)
+    wu = bf_vals(g.standard_normal((F, K)) * 0.05)
+    wgu = np.empty((2 * F, K), np.float32)
+    wgu[0::2], wgu[1::2] = wg, wu
+    out = ctx.linear_swiglu(bf(x), bf(wgu))
+    x64 = x.astype(np.float64)
+    ref = O.silu(x64 @ wg.T) * (x64 @ wu.T)
+    assert rel(out.float().cpu().numpy(), ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("Hq,Hkv,bias,rows_per_seq,pos0,batch,L", [
+    (4, 4, False, 32, 64, 2, 128),     # block slot of 2 sequences
+    (4, 2, True, 128, 0, 2, 128),      # refresh: every position, GQA, Qwen-style bias
+    (7, 1, True, 32, 96, 1, 160),
+])
+def test_qkv_rope_store(ctx, Hq, Hkv, bias, rows_per_seq, pos0, batch, L):
+    g = synth.rng(Hq * 10 + pos0)
+    D, d = 256, 128
+    M = rows_per_seq * batch
+    N = (Hq + 2 * Hkv) * d
+    x = bf_vals(g.standard_normal((M, D)))
+    w = bf_vals(g.standard_normal((N, D)) * 0.06)
+    b = (g.standard_normal(N) * 0.1).astype(np.float32) if bias else None
+    k0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
+    v0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
+    from block_kv_cache_b200 import fdllm
+    rope = torch.from_numpy(fdllm.rope_table(10000.0, L, d)).cuda()
+    kc, vc = bf(k0), bf(v0)
+    q = torch.empty((M, Hq, d), dtype=torch.bfloat16, device="cuda")
+    ctx.qkv_rope_store(bf(x), bf(w), rope, q, kc, vc, n_q_heads=Hq, rows_per_seq=rows_per_seq,
+                       pos0=pos0, bias=None if b is None else f32(b))
+    y = x.astype(np.float64) @ w.astype(np.float64).T
+    if b is not None:
+        y = y + b
+    pos = pos0 + np.arange(M) % rows_per_seq
+    qr = O.apply_rope(y[:, :Hq * d].reshape(M, Hq, d), pos)
+    kr = O.apply_rope(y[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d), pos)
+    vr = y[:, (Hq + Hkv) * d:].reshape(M, Hkv, d)
+    assert rel(q.float().cpu().numpy(), qr) <= BF16_TOL
+    kg, vg = kc.float().cpu().numpy(), vc.float().cpu().numpy()
+    written = np.zeros((batch, L), bool)
+    for r in range(M):
+        sq, p = r // rows_per_seq, pos[r]
+        written[sq, p] = True
+        assert np.abs(kg[sq, :, p] - kr[r]).max() <= BF16_TOL * np.abs(kr).max()
+        assert np.abs(vg[sq, :, p] - vr[r]).max() <= BF16_TOL * np.abs(vr).max()
+    # rows outside the written positions untouched
+    for sq in range(batch):
+        keep = ~written[sq]
+        assert np.array_equal(kg[sq][:, keep], k0[sq][:, keep])
+        assert np.array_equal(vg[sq][:, keep], v0[sq][:, keep])
+
+
+@pytest.mark.parametrize("b,Hq,Hkv,L", [(1, 32, 32, 256), (2, 28, 4, 128), (2, 8, 2, 96)])
+def test_full_attention(ctx, b, Hq, Hkv, L):
+    g = synth.rng(b * Hq + L)
+    d = 128
+    q = bf_vals(g.standard_normal((b, L, Hq, d)))
+    k = bf_vals(g.standard_normal((b, Hkv, L, d)))
+    v = bf_vals(g.standard_normal((b, Hkv, L, d)))
+    out = ctx.full_attention(bf(q), bf(k), bf(v)).float().cpu().numpy()
+    for s in range(b):
+        o, _ = O.attention(q[s], k[s], v[s])
+        assert rel(out[s], o) <= BF16_TOL
+
+
+# ------------------------------------------------------------------ whole decodes
+def _small_params(seed, n_layers=2, hq=2, hkv=2, bias=False):
+    return synth.model_params(vocab=512, hidden=256, n_layers=n_layers, n_q_heads=hq,
+                              n_kv_heads=hkv, head_dim=128, ffn=512, seed=seed, dtype="bf16",
+                              qkv_bias=bias, w_std=0.06, lm_std=0.15)
+
+
+def _replay_check(P, rec, x_final, B, tau):
+    """Oracle replay of a recorded GPU decode (see module docstring)."""
+    b = rec[0][2].shape[0]
+    caches = [None] * b
+    max_err = 0.0
+    for n, (kind, s, xb, mb, conf, tok) in enumerate(rec):
+        conf = conf.reshape(b, B)
+        tok = tok.reshape(b, B)
+        for i in range(b):
+            if kind == "refresh":
+                logits, kv = O.full_forward(P, xb[i])
+                caches[i] = [(k.copy(), v.copy()) for k, v in kv]
+                lg = logits[s:s + B]
+            else:
+                lg = O.block_forward(P, xb[i, s:s + B], s, caches[i])
+            c = O.confidence_from_logits(lg)
+            max_err = max(max_err, float(np.abs(conf[i] - c.conf).max()))
+            sure = c.gap > TOK_GAP
+            assert np.array_equal(tok[i][sure], c.tok[sure]), (n, i)
+        # decisions on the GPU's confidences, bit-exact
+        xa, ma, _, nd = O.threshold_unmask(xb, mb, conf, tok, s, B, tau)
+        x_next = rec[n + 1][2] if n + 1 < len(rec) else x_final
+        m_next = rec[n + 1][3] if n + 1 < len(rec) else None
+        assert np.array_equal(xa, x_next), n
+        if m_next is not None:
+            assert np.array_equal(ma, m_next), n
+    assert max_err <= CONF_MODEL_TOL, max_err
+    return max_err
+
+
+@pytest.mark.parametrize("seed,tau,hq,hkv,bias", [(0, 0.9, 2, 2, False), (1, 0.5, 4, 2, True),
+                                                  (2, 1.0, 2, 1, False)])
+def test_decode_matches_oracle_step_by_step(ctx, seed, tau, hq, hkv, bias):
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(seed, hq=hq, hkv=hkv, bias=bias)
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B = 2, 64, 64, 32
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B)
+    prompt = synth.prompt_ids(seed, b, Lp, P.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
+    ctx.device_status()
+    xf = x.cpu().numpy()
+    assert steps == len(rec)
+    if tau == 1.0:
+        assert steps == gen                              # one token per step
+    _replay_check(P, rec, xf, B, tau)
+
+
+def test_tau_one_single_layer_gpu_equals_sequential(ctx):
+    """tau = 1 and one layer: the GPU's DualCache decode equals sequential
+    greedy decoding of the oracle wherever the oracle's choices are not
+    near-ties (checked token by token along the GPU's own trajectory)."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(5, n_layers=1)
+    w = DeviceWeights.from_params(P)
+    dec = BlockDecoder(ctx, w, 1, 96, 32)
+    prompt = synth.prompt_ids(5, 1, 32, P.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, 64, tau=1.0, record=rec)
+    assert steps == 64
+    # each step decodes exactly the position the sequential rule picks
+    for kind, s, xb, mb, conf, tok in rec:
+        logits, _ = O.full_forward(P, xb[0])
+        c = O.confidence_from_logits(logits[s:s + 32])
+        cand = mb[0, s:s + 32] != 0
+        order = np.argsort(-np.where(cand, c.conf, -1.0), kind="stable")
+        top, second = order[0], order[1] if cand.sum() > 1 else None
+        if second is not None and c.conf[top] - c.conf[second] < 2 * CONF_MODEL_TOL:
+            continue                                   # near tie: either choice is correct
+        gpu_pick = int(np.argmax(np.where(cand, conf, -1.0)))
+        assert gpu_pick == top
