@@ -15,7 +15,13 @@ struct fdl_ctx {
     int device;
     int sm_count;
     int* d_err;              // device error word (4 bytes)
+    float* d_acc;            // split-K accumulator of the projections, kept all zeros
+    size_t acc_bytes;
 };
+
+// Split-K accumulator of the few-token projections (zeroed at creation; every
+// kernel that adds into it leaves it zeroed again): room for 256 rows x 32768.
+static const size_t kAccBytes = (size_t)256 * 32768 * 4;
 
 namespace {
 
@@ -117,12 +123,18 @@ int fdl_create(fdl_ctx** out, int device) {
     c->device = device;
     c->sm_count = prop.multiProcessorCount;
     c->d_err = nullptr;
+    c->d_acc = nullptr;
+    c->acc_bytes = kAccBytes;
     e = cudaMalloc(&c->d_err, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(int));
+    if (e == cudaSuccess) e = cudaMalloc(&c->d_acc, kAccBytes);
+    if (e == cudaSuccess) e = cudaMemset(c->d_acc, 0, kAccBytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         if (c->d_err) cudaFree(c->d_err);
+        if (c->d_acc) cudaFree(c->d_acc);
         delete c;
-        return cuda_fail(e, "fdl_create: error word");
+        return cuda_fail(e, "fdl_create: device buffers");
     }
     *out = c;
     return FDL_OK;
@@ -132,6 +144,7 @@ int fdl_destroy(fdl_ctx* ctx) {
     if (!ctx) return FDL_OK;
     DeviceGuard g(ctx->device);
     if (ctx->d_err) cudaFree(ctx->d_err);
+    if (ctx->d_acc) cudaFree(ctx->d_acc);
     delete ctx;
     return FDL_OK;
 }
@@ -363,8 +376,10 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
     fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
                   (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
                   d->rows_per_seq, d->pos0};
-    cudaError_t e = fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err,
-                                         (cudaStream_t)stream);
+    cudaError_t e = fdl::skinny_ok(gs)
+        ? fdl::launch_skinny_qkv(gs, x, w, p, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
+                                 ctx->d_err, (cudaStream_t)stream)
+        : fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv launch");
 }
 
@@ -379,8 +394,11 @@ int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_feature
         return fail(FDL_EINVAL, "linear_residual: buffers must be 16-byte aligned");
     DeviceGuard g(ctx->device);
     fdl::GemmShape gs{rows, out_features, in_features};
-    cudaError_t e = fdl::launch_gemm_resid(gs, x, w, fdl::EpiResid{h, out_features},
-                                           ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
+    const fdl::EpiResid ep{h, out_features};
+    cudaError_t e = fdl::skinny_ok(gs)
+        ? fdl::launch_skinny_resid(gs, x, w, ep, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
+                                   ctx->d_err, (cudaStream_t)stream)
+        : fdl::launch_gemm_resid(gs, x, w, ep, ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_residual launch");
 }
 
@@ -395,9 +413,12 @@ int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
         return fail(FDL_EINVAL, "linear_swiglu: buffers must be 16-byte aligned");
     DeviceGuard g(ctx->device);
     fdl::GemmShape gs{rows, 2 * out_features, in_features};
-    cudaError_t e = fdl::launch_gemm_swiglu(gs, x, w_gu, fdl::EpiSwiGLU{(fdl::bf16*)out,
-                                            out_features}, ctx->sm_count, ctx->d_err,
-                                            (cudaStream_t)stream);
+    const fdl::EpiSwiGLU ep{(fdl::bf16*)out, out_features};
+    cudaError_t e = fdl::skinny_ok(gs)
+        ? fdl::launch_skinny_swiglu(gs, x, w_gu, ep, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
+                                    ctx->d_err, (cudaStream_t)stream)
+        : fdl::launch_gemm_swiglu(gs, x, w_gu, ep, ctx->sm_count, ctx->d_err,
+                                  (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_swiglu launch");
 }
 

@@ -205,6 +205,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
 
@@ -484,19 +486,8 @@ cudaError_t run_tc(const AttnPlan& p, const CUtensorMap& tq, const CUtensorMap& 
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S::TOTAL);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.n_splits, hkv * p.n_chunks, batch);
-    cfg.blockDim = dim3(S::THREADS);
-    cfg.dynamicSmemBytes = S::TOTAL;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.n_splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kfn, tq, tk, tv, a);
+    return launch_pdl(kfn, dim3(p.n_splits, hkv * p.n_chunks, batch), dim3(S::THREADS), S::TOTAL,
+                      st, p.n_splits, tq, tk, tv, a);
 }
 
 }  // namespace

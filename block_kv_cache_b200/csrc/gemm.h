@@ -38,6 +38,20 @@ cudaError_t launch_gemm_swiglu(const GemmShape& g, const void* a, const void* w,
 cudaError_t launch_gemm_qkv(const GemmShape& g, const void* a, const void* w, const EpiQKV& p,
                             int sm_count, int* err, cudaStream_t st);
 
+// Token-few variants (M <= 256, N % 128 == 0): weight rows on the MMA's M side.
+bool skinny_ok(const GemmShape& g);
+cudaError_t launch_skinny_resid(const GemmShape& g, const void* x, const void* w,
+                                const EpiResid& p, float* acc, size_t acc_bytes, int sm_count,
+                                int* err, cudaStream_t st);
+// acc: f32 scratch of acc_bytes, all zeros; split-K partial sums go there and
+// the finishing kernel restores the zeros. Too small or NULL: no K split.
+cudaError_t launch_skinny_swiglu(const GemmShape& g, const void* x, const void* w,
+                                 const EpiSwiGLU& p, float* acc, size_t acc_bytes, int sm_count,
+                                 int* err, cudaStream_t st);
+cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, const EpiQKV& p,
+                              float* acc, size_t acc_bytes, int sm_count, int* err,
+                              cudaStream_t st);
+
 // out[i, :] = bf16(h[src_i, :] / sqrt(mean(h[src_i]^2) + eps) * weight), src_i =
 // row_map ? row_map[i] : i.
 cudaError_t launch_rmsnorm(int rows, int hidden, const float* h, const int32_t* row_map,

@@ -182,6 +182,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
     const int k_iters = K / BK;
 
@@ -274,9 +276,8 @@ cudaError_t run_gemm(const GemmShape& g, const void* a, const void* w, const Epi
     e = cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    gemm_tc_kernel<Epi><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, g.M, g.N, g.K, num_m, items,
-                                                           err, epi);
-    return cudaGetLastError();
+    return launch_pdl(gemm_tc_kernel<Epi>, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 0, ta, tb,
+                      g.M, g.N, g.K, num_m, items, err, epi);
 }
 
 }  // namespace

@@ -1,0 +1,414 @@
+// Weight-streaming GEMMs of the cached block step (few token rows, M <= 256):
+//   C^T[N, M] = W[N, K] . X[M, K]^T      ("swap AB": the weight is the MMA's
+// A operand, 128 weight rows per tile; the tokens are its N dimension).
+//
+// At a cached DualCache step only the block's rows (32 per sequence) pass
+// through the layers (Fast-dLLM; aibase news "Innovations" 1), so every
+// projection is a stream of the weight matrix past a handful of activation
+// rows: HBM-bound, N*K*2 bytes per call. Putting the weight rows on the MMA's
+// M side keeps the tensor-core work per weight byte at the token count
+// instead of padding the tokens to 128 rows, and gives twice as many tiles as
+// 256-wide token-major tiles; the residual projections also split K so that
+// every SM streams (partial sums added atomically into the f32 residual).
+//
+// Persistent, warp-specialised: warp 0 TMA (ring of 128-wide K steps, each two
+// 64-column boxes of the 128-row weight tile and of the NT activation rows,
+// 128-byte swizzle), warp 1 TMEM owner + single-thread tcgen05.mma (M=128,
+// N=NT, K=16) into two NT-column accumulators, warps 2-5 epilogue with
+// thread = weight row (output feature), columns = tokens.
+#include "common.cuh"
+#include "gemm.h"
+#include "sm100.cuh"
+
+namespace fdl {
+namespace {
+
+constexpr int SK_BM = 128, SK_BK = 128, SK_THREADS = 192;
+
+template <int NT>
+struct Sk {
+    static constexpr int A_BYTES = SK_BM * SK_BK * 2;        // weight tile (2 chunks of 64)
+    static constexpr int B_BYTES = NT * SK_BK * 2;           // activation tile (2 chunks)
+    static constexpr int A_CHUNK = SK_BM * 128, B_CHUNK = NT * 128;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (176 * 1024) / STAGE > 8 ? 8 : (176 * 1024) / STAGE;
+    static constexpr int OFF_X = STAGES * STAGE;             // epilogue exchange (QKV)
+    static constexpr int X_BYTES = SK_BM * 33 * 4;           // 128 rows x 32 tokens (+1 pad)
+    static constexpr int OFF_BAR = OFF_X + X_BYTES;
+    static constexpr size_t TOTAL = 1024 + OFF_BAR + 256;
+    static constexpr uint32_t TMEM_COLS = 2 * NT < 32 ? 32 : 2 * NT;
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+    static_assert(TOTAL <= 227 * 1024, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Each epilogue gets (TMEM address of its lane's accumulator row, feature
+// index within [0, N), token count M, first token of the 32-token chunk, the
+// 32 accumulator values of the chunk).
+struct SkResid {
+    EpiResid p;
+    int split;          // > 1: partial sums are added atomically
+    static constexpr bool kSplitK = true;
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            if (t < M) {
+                float* dst = p.h + (size_t)t * p.ldh + f;
+                if (split > 1) atomicAdd(dst, v[j]);
+                else *dst += v[j];
+            }
+        }
+    }
+};
+
+// Split-K partial sums of a non-linear projection: acc[t][f] += C (f32,
+// token-major: for one token a warp's 32 features are one 128-byte line, so
+// each atomic instruction is a single coalesced L2 request); the epilogue
+// proper runs in a finish_* kernel that also restores the zeros.
+struct SkAccum {
+    float* acc;
+    int ldn;
+    static constexpr bool kSplitK = true;
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            if (t < M) atomicAdd(acc + (size_t)t * ldn + f, v[j]);
+        }
+    }
+};
+
+struct SkSwiGLU {
+    EpiSwiGLU p;
+    static constexpr bool kSplitK = false;
+    // rows 2g and 2g+1 of the tile are gate and up of feature g: adjacent lanes
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
+        const int lane = threadIdx.x & 31;
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+            const float up = __shfl_down_sync(0xffffffffu, v[j], 1);
+            const int t = j0 + j;
+            if (!(lane & 1) && t < M) {
+                const float g = v[j];
+                p.out[(size_t)t * p.ldo + (f >> 1)] =
+                    __float2bfloat16_rn(g / (1.f + __expf(-g)) * up);
+            }
+        }
+    }
+};
+
+struct SkQKV {
+    EpiQKV p;
+    static constexpr bool kSplitK = false;
+    // one tile = one head (128 dims); RoPE partners are 64 rows apart, so the
+    // chunk is exchanged through shared memory (row = dim, 32 tokens, +1 pad)
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t* xbuf, int n0) const {
+        constexpr int D = 128;
+        const int r = f - n0;                      // dim within the head
+        float* xs = reinterpret_cast<float*>(xbuf);
+        const int nq = p.n_q_heads * D, nk = p.n_kv_heads * D;
+        const bool rot = n0 < nq + nk;
+        if (rot) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xs[r * 33 + j] = v[j];
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const float bias = p.bias ? p.bias[f] : 0.f;
+        const float pb = (rot && p.bias) ? p.bias[n0 + (r ^ 64)] : 0.f;
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            if (t >= M) break;
+            const int seq = t / p.rows_per_seq, pos = p.pos0 + t % p.rows_per_seq;
+            float y = v[j] + bias;
+            if (rot) {
+                const float other = xs[(r ^ 64) * 33 + j] + pb;
+                const float2 cs = p.rope[(size_t)pos * (D / 2) + (r & 63)];
+                y = r < 64 ? y * cs.x - other * cs.y : other * cs.y + y * cs.x;
+            }
+            bf16* dst;
+            if (n0 < nq)
+                dst = p.q + ((size_t)t * p.n_q_heads + n0 / D) * D + r;
+            else if (n0 < nq + nk)
+                dst = p.k_cache + (((size_t)seq * p.n_kv_heads + (n0 - nq) / D) * p.seq_len + pos) *
+                                      D + r;
+            else
+                dst = p.v_cache +
+                      (((size_t)seq * p.n_kv_heads + (n0 - nq - nk) / D) * p.seq_len + pos) * D + r;
+            *dst = __float2bfloat16_rn(y);
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // exchange buffer free again
+    }
+};
+
+template <int NT, class Epi>
+__global__ void __launch_bounds__(SK_THREADS, 1)
+gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   int M, int N, int K, int splits, int num_items, int* err, const Epi epi) {
+    using namespace sm100;
+    using S = Sk<NT>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t sbase = raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S::STAGES + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    auto full_bar = [&](int s) { return smem_u32(bars + s); };
+    auto empty_bar = [&](int s) { return smem_u32(bars + S::STAGES + s); };
+    auto tfull_bar = [&](int a) { return smem_u32(bars + 2 * S::STAGES + a); };
+    auto tempty_bar = [&](int a) { return smem_u32(bars + 2 * S::STAGES + 2 + a); };
+    auto sA = [&](int s) { return sbase + s * S::STAGE; };
+    auto sB = [&](int s) { return sbase + s * S::STAGE + S::A_BYTES; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int k_iters = K / SK_BK;
+    const int kps = (k_iters + splits - 1) / splits;        // k iterations per split
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S::STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 128);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    pdl_wait();
+    pdl_trigger();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tmW);
+            prefetch_tmap(&tmX);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
+                const int n_tile = item / splits, ks = item % splits;
+                const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
+                for (int k = k0; k < k1; ++k) {
+                    if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
+                    mbar_arrive_expect_tx(full_bar(stage), S::STAGE);
+                    for (int c = 0; c < 2; ++c) {
+                        tma_load_2d(sA(stage) + c * S::A_CHUNK, &tmW, full_bar(stage),
+                                    k * SK_BK + c * 64, n_tile * SK_BM);
+                        tma_load_2d(sB(stage) + c * S::B_CHUNK, &tmX, full_bar(stage),
+                                    k * SK_BK + c * 64, 0);
+                    }
+                    if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            for (int s = 0; ok && s < S::STAGES; ++s) {
+                ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err);
+                if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32(SK_BM, NT);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int it = 0;
+            for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++it) {
+                const int ks = item % splits;
+                const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
+                const int acc = it & 1;
+                const uint32_t aphase = (it >> 1) & 1;
+                if (!(ok = mbar_wait(tempty_bar(acc), aphase ^ 1, abort_flag, err))) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * NT;
+                for (int k = k0; k < k1; ++k) {
+                    if (!(ok = mbar_wait(full_bar(stage), phase, abort_flag, err))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < SK_BK / 16; ++kk) {
+                        const uint64_t a0 = umma_desc_sw128(sA(stage) + (kk >> 2) * S::A_CHUNK);
+                        const uint64_t b0 = umma_desc_sw128(sB(stage) + (kk >> 2) * S::B_CHUNK);
+                        umma_bf16(d_tmem, a0 + (uint64_t)((kk & 3) * 2), b0 + (uint64_t)((kk & 3) * 2),
+                                  idesc, (k > k0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(empty_bar(stage));
+                    if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (ok) umma_commit(tfull_bar(acc));
+            }
+        }
+    } else {
+        const int q = warp & 3;                     // TMEM lane quarter = 32 weight rows
+        const int r = q * 32 + lane;
+        int it = 0;
+        for (int item = blockIdx.x; item < num_items; item += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t aphase = (it >> 1) & 1;
+            const int n0 = (item / splits) * SK_BM;
+            if (!mbar_wait_warp(tfull_bar(acc), aphase, abort_flag, err)) break;
+            tc_fence_after();
+            const uint32_t tacc = tmem_base + ((uint32_t)(q * 32) << 16) + acc * NT;
+#pragma unroll 1
+            for (int j0 = 0; j0 < NT; j0 += 32) {
+                float v[32];
+                tmem_ld32(tacc + j0, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_wait_ld();
+                if (j0 >= M) break;                           // no token left (uniform)
+                epi.chunk(n0 + r, M, j0, v, smem + S::OFF_X, n0);
+            }
+            tc_fence_before();
+            mbar_arrive(tempty_bar(acc));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+template <int NT, class Epi>
+cudaError_t run_skinny(const GemmShape& g, const void* x, const void* w, const Epi& epi,
+                       int splits, int sm_count, int* err, cudaStream_t st) {
+    using S = Sk<NT>;
+    CUtensorMap tw, tx;
+    cudaError_t e = make_tmap_bf16_2d(&tw, w, g.N, g.K, SK_BM, 64);
+    if (e != cudaSuccess) return e;
+    e = make_tmap_bf16_2d(&tx, x, g.M, g.K, NT, 64);
+    if (e != cudaSuccess) return e;
+    const int items = (g.N / SK_BM) * splits;
+    const int grid = items < sm_count ? items : sm_count;
+    e = cudaFuncSetAttribute(gemm_skinny_kernel<NT, Epi>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::TOTAL);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(gemm_skinny_kernel<NT, Epi>, dim3(grid), dim3(SK_THREADS), S::TOTAL, st, 0,
+                      tw, tx, g.M, g.N, g.K, splits, items, err, epi);
+}
+
+template <class Epi>
+cudaError_t dispatch_skinny(const GemmShape& g, const void* x, const void* w, const Epi& epi,
+                            int splits, int sm_count, int* err, cudaStream_t st) {
+    if (g.M <= 32) return run_skinny<32>(g, x, w, epi, splits, sm_count, err, st);
+    if (g.M <= 64) return run_skinny<64>(g, x, w, epi, splits, sm_count, err, st);
+    if (g.M <= 128) return run_skinny<128>(g, x, w, epi, splits, sm_count, err, st);
+    return run_skinny<256>(g, x, w, epi, splits, sm_count, err, st);
+}
+
+// K splits: the (tiles x splits) work items should fill whole waves of the
+// persistent grid (a partly filled last wave leaves SMs idle while the others
+// stream), with at least 4 K steps per split. Among splits with the best wave
+// efficiency the smallest wins (fewer partial-sum additions).
+int choose_splits(const GemmShape& g, int sm_count, int max_splits) {
+    const int tiles = g.N / SK_BM, k_iters = g.K / SK_BK;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int s = 1; s <= max_splits && s <= k_iters / 4; ++s) {
+        const int items = tiles * s;
+        const int waves = (items + sm_count - 1) / sm_count;
+        const double eff = (double)items / ((double)waves * sm_count);
+        if (eff > best_eff + 0.02) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    const int kps = (k_iters + best - 1) / best;
+    return (k_iters + kps - 1) / kps;            // every split gets at least one K step
+}
+
+// ---- epilogues of split-K projections: consume the f32 sums, leave zeros ----------
+__global__ void finish_swiglu_kernel(float* __restrict__ acc, int M, int F, bf16* __restrict__ out,
+                                     int ldo) {
+    pdl_wait();
+    pdl_trigger();
+    const size_t n = (size_t)M * F;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const size_t t = e / F, f = e % F;
+        float2* pg = reinterpret_cast<float2*>(acc + t * 2 * F + 2 * f);
+        const float2 gu = *pg;
+        *pg = make_float2(0.f, 0.f);
+        out[t * ldo + f] = __float2bfloat16_rn(gu.x / (1.f + __expf(-gu.x)) * gu.y);
+    }
+}
+
+// one CTA of 128 threads per (token, head of q, k or v); thread = dim
+__global__ void finish_qkv_kernel(float* __restrict__ acc, int M, EpiQKV p) {
+    pdl_wait();
+    pdl_trigger();
+    constexpr int D = 128;
+    const int heads = p.n_q_heads + 2 * p.n_kv_heads;
+    const int t = blockIdx.x / heads, h = blockIdx.x % heads, r = threadIdx.x;
+    const int N = heads * D;
+    float* row = acc + (size_t)t * N + h * D;
+    float y = row[r] + (p.bias ? p.bias[h * D + r] : 0.f);
+    const int seq = t / p.rows_per_seq, pos = p.pos0 + t % p.rows_per_seq;
+    if (h < p.n_q_heads + p.n_kv_heads) {
+        const float other = row[r ^ 64] + (p.bias ? p.bias[h * D + (r ^ 64)] : 0.f);
+        const float2 cs = p.rope[(size_t)pos * (D / 2) + (r & 63)];
+        y = r < 64 ? y * cs.x - other * cs.y : other * cs.y + y * cs.x;
+    }
+    __syncthreads();                               // both halves read before zeroing
+    row[r] = 0.f;
+    bf16* dst;
+    if (h < p.n_q_heads)
+        dst = p.q + ((size_t)t * p.n_q_heads + h) * D + r;
+    else if (h < p.n_q_heads + p.n_kv_heads)
+        dst = p.k_cache + (((size_t)seq * p.n_kv_heads + h - p.n_q_heads) * p.seq_len + pos) * D + r;
+    else
+        dst = p.v_cache +
+              (((size_t)seq * p.n_kv_heads + h - p.n_q_heads - p.n_kv_heads) * p.seq_len + pos) * D + r;
+    *dst = __float2bfloat16_rn(y);
+}
+
+}  // namespace
+
+bool skinny_ok(const GemmShape& g) { return g.M <= 256 && g.N % SK_BM == 0 && g.K % SK_BK == 0; }
+
+cudaError_t launch_skinny_resid(const GemmShape& g, const void* x, const void* w,
+                                const EpiResid& p, float* acc, size_t acc_bytes, int sm_count,
+                                int* err, cudaStream_t st) {
+    (void)acc;
+    (void)acc_bytes;
+    // partial sums go straight into the f32 residual stream (coalesced atomics)
+    const int splits = choose_splits(g, sm_count, 16);
+    return dispatch_skinny(g, x, w, SkResid{p, splits}, splits, sm_count, err, st);
+}
+
+cudaError_t launch_skinny_swiglu(const GemmShape& g, const void* x, const void* w,
+                                 const EpiSwiGLU& p, float* acc, size_t acc_bytes, int sm_count,
+                                 int* err, cudaStream_t st) {
+    const int splits = acc && (size_t)g.M * g.N * 4 <= acc_bytes
+                           ? choose_splits(g, sm_count, 8) : 1;
+    if (splits == 1) return dispatch_skinny(g, x, w, SkSwiGLU{p}, 1, sm_count, err, st);
+    cudaError_t e = dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st);
+    if (e != cudaSuccess) return e;
+    const size_t n = (size_t)g.M * (g.N / 2);
+    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    return launch_pdl(finish_swiglu_kernel, dim3(blocks), dim3(256), 0, st, 0, acc, g.M, g.N / 2,
+                      p.out, p.ldo);
+}
+
+cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, const EpiQKV& p,
+                              float* acc, size_t acc_bytes, int sm_count, int* err,
+                              cudaStream_t st) {
+    const int splits = acc && (size_t)g.M * g.N * 4 <= acc_bytes
+                           ? choose_splits(g, sm_count, 8) : 1;
+    if (splits == 1) return dispatch_skinny(g, x, w, SkQKV{p}, 1, sm_count, err, st);
+    cudaError_t e = dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(finish_qkv_kernel, dim3(g.M * (g.N / 128)), dim3(128), 0, st, 0, acc, g.M,
+                      p);
+}
+
+}  // namespace fdl

@@ -14,6 +14,8 @@ namespace fdl {
 __global__ void kv_store_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
                                 uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                                 long long total, int n, int Hkv, int chunks, int L, int start) {
+    pdl_wait();
+    pdl_trigger();
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
         const int c = (int)(idx % chunks);
@@ -38,10 +40,9 @@ cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len
     const int threads = 256;
     long long blocks = (total + threads - 1) / threads;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
-    kv_store_kernel<<<(int)blocks, threads, 0, st>>>(
-        (const uint4*)k_new, (const uint4*)v_new, (uint4*)k_cache, (uint4*)v_cache, total, n,
-        n_kv_heads, chunks, seq_len, start);
-    return cudaGetLastError();
+    return launch_pdl(kv_store_kernel, dim3((int)blocks), dim3(threads), 0, st, 0,
+                      (const uint4*)k_new, (const uint4*)v_new, (uint4*)k_cache, (uint4*)v_cache,
+                      total, n, n_kv_heads, chunks, seq_len, start);
 }
 
 }  // namespace fdl

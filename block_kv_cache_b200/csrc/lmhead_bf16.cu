@@ -78,6 +78,8 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    pdl_wait();
+    pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
     const int k_iters = D / BK;
 
@@ -221,9 +223,8 @@ cudaError_t launch_lmhead_bf16(const LMShape& s, const void* h, const void* w,
                              (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     LMPartial* part = (LMPartial*)ws;
-    lmhead_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, bias_tok, bias_val, part, s.rows,
-                                                        s.hidden, s.vocab, num_m, items, dev_err);
-    e = cudaGetLastError();
+    e = launch_pdl(lmhead_tc_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, st, 0, ta, tb,
+                   bias_tok, bias_val, part, s.rows, s.hidden, s.vocab, num_m, items, dev_err);
     if (e != cudaSuccess) return e;
     return launch_lmhead_combine(part, num_n, s.rows, conf, tok, st);
 }

@@ -9,6 +9,8 @@ namespace fdl {
 
 __global__ void lmhead_combine_kernel(const LMPartial* __restrict__ part, int n_tiles, int M,
                                       float* __restrict__ conf, int32_t* __restrict__ tok) {
+    pdl_wait();
+    pdl_trigger();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= M) return;
@@ -35,8 +37,8 @@ cudaError_t launch_lmhead_combine(const LMPartial* part, int n_tiles, int M, flo
                                   int32_t* tok, cudaStream_t st) {
     const int threads = 256;
     const int blocks = (M * 32 + threads - 1) / threads;
-    lmhead_combine_kernel<<<blocks, threads, 0, st>>>(part, n_tiles, M, conf, tok);
-    return cudaGetLastError();
+    return launch_pdl(lmhead_combine_kernel, dim3(blocks), dim3(threads), 0, st, 0, part, n_tiles,
+                      M, conf, tok);
 }
 
 }  // namespace fdl

@@ -12,6 +12,8 @@ constexpr int NORM_THREADS = 256;
 __global__ void __launch_bounds__(NORM_THREADS)
 rmsnorm_kernel(const float* __restrict__ h, const int32_t* __restrict__ row_map,
                const float* __restrict__ weight, float eps, bf16* __restrict__ out, int hidden) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float s_red[NORM_THREADS / 32];
     const int i = blockIdx.x;
     const int src = row_map ? row_map[i] : i;
@@ -44,6 +46,8 @@ rmsnorm_kernel(const float* __restrict__ h, const int32_t* __restrict__ row_map,
 __global__ void __launch_bounds__(NORM_THREADS)
 embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ row_map,
              const bf16* __restrict__ table, float* __restrict__ h, int hidden) {
+    pdl_wait();
+    pdl_trigger();
     const int i = blockIdx.x;
     const int id = ids[row_map ? row_map[i] : i];
     const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(table + (size_t)id * hidden);
@@ -53,14 +57,14 @@ embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ row_ma
 
 cudaError_t launch_rmsnorm(int rows, int hidden, const float* h, const int32_t* row_map,
                            const float* weight, float eps, bf16* out, cudaStream_t st) {
-    rmsnorm_kernel<<<rows, NORM_THREADS, 0, st>>>(h, row_map, weight, eps, out, hidden);
-    return cudaGetLastError();
+    return launch_pdl(rmsnorm_kernel, dim3(rows), dim3(NORM_THREADS), 0, st, 0, h, row_map, weight,
+                      eps, out, hidden);
 }
 
 cudaError_t launch_embed(int rows, int hidden, const int32_t* ids, const int32_t* row_map,
                          const bf16* table, float* h, cudaStream_t st) {
-    embed_kernel<<<rows, NORM_THREADS, 0, st>>>(ids, row_map, table, h, hidden);
-    return cudaGetLastError();
+    return launch_pdl(embed_kernel, dim3(rows), dim3(NORM_THREADS), 0, st, 0, ids, row_map, table,
+                      h, hidden);
 }
 
 }  // namespace fdl

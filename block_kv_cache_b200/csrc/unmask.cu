@@ -20,6 +20,8 @@ threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restric
                         int32_t* __restrict__ x, uint8_t* __restrict__ masked,
                         int32_t* __restrict__ remaining, int32_t* __restrict__ n_decoded,
                         int L, int s, int B, float tau, int* err) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ float s_val[32];
     __shared__ int s_idx[32];
     __shared__ int s_win;
@@ -79,10 +81,9 @@ cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
                                     int32_t* remaining, int32_t* n_decoded,
                                     int* dev_err, cudaStream_t st) {
     int threads = ((block_len + 31) / 32) * 32;
-    threshold_unmask_kernel<<<batch, threads, 0, st>>>(conf, tok, x, masked, remaining,
-                                                       n_decoded, seq_len, block_start,
-                                                       block_len, tau, dev_err);
-    return cudaGetLastError();
+    return launch_pdl(threshold_unmask_kernel, dim3(batch), dim3(threads), 0, st, 0, conf, tok, x,
+                      masked, remaining, n_decoded, seq_len, block_start, block_len, tau,
+                      dev_err);
 }
 
 }  // namespace fdl

@@ -3,6 +3,7 @@
     python -m block_kv_cache_b200.kernel_cases lmhead --rows 32 [--iters 20]
     python -m block_kv_cache_b200.kernel_cases attention --heads 32 --kv-heads 32 \
         --prefix 512 --block 32 --suffix 224 [--layers 32]
+    python -m block_kv_cache_b200.kernel_cases swiglu|resid|qkv --rows 32 --n 24576 --k 4096
 
 Used to profile a single kernel (e.g. under ncu with -k/-c) and to time it
 with CUDA events. With --graph the timed calls are captured once in a CUDA
@@ -86,9 +87,43 @@ def run_attention(a, ctx):
             "TFLOPs": flops / us / 1e6}
 
 
+def run_linear(a, ctx):
+    """One projection of the transformer at (rows, n, k); `layers` distinct weight
+    matrices are cycled so the weight stream comes from HBM, not L2."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    ws = [(torch.randn(a.n, a.k, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+          for _ in range(a.layers)]
+    x = torch.randn(a.rows, a.k, generator=g, device="cuda").to(torch.bfloat16)
+    if a.op == "swiglu":
+        out = torch.empty((a.rows, a.n // 2), dtype=torch.bfloat16, device="cuda")
+        call = lambda i: ctx.linear_swiglu(x, ws[i % a.layers], out=out)
+    elif a.op == "resid":
+        h = torch.zeros((a.rows, a.n), dtype=torch.float32, device="cuda")
+        call = lambda i: ctx.linear_residual(x, ws[i % a.layers], h)
+    else:
+        from block_kv_cache_b200 import fdllm as F
+        nq = a.heads
+        nkv = (a.n // 128 - nq) // 2
+        L = 2048
+        rope = torch.from_numpy(F.rope_table(10000.0, L, 128)).cuda()
+        q = torch.empty((a.rows, nq, 128), dtype=torch.bfloat16, device="cuda")
+        kc = torch.zeros((1, nkv, L, 128), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        call = lambda i: ctx.qkv_rope_store(x, ws[i % a.layers], rope, q, kc, vc, n_q_heads=nq,
+                                            rows_per_seq=a.rows, pos0=a.prefix)
+    us = _timed(a, call)
+    ctx.device_status()
+    nbytes = a.n * a.k * 2 + a.rows * a.k * 2
+    return {"op": a.op, "rows": a.rows, "n": a.n, "k": a.k, "graph": a.graph, "us": us,
+            "GBps": nbytes / us / 1e3, "TFLOPs": 2.0 * a.rows * a.n * a.k / us / 1e6}
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["lmhead", "attention"])
+    p.add_argument("op", choices=["lmhead", "attention", "swiglu", "resid", "qkv"])
+    p.add_argument("--n", type=int, default=24576)
+    p.add_argument("--k", type=int, default=4096)
     p.add_argument("--rows", type=int, default=32)
     p.add_argument("--hidden", type=int, default=4096)
     p.add_argument("--vocab", type=int, default=126464)
@@ -106,7 +141,12 @@ def main():
     p.add_argument("--reps", type=int, default=5, help="graph replays timed (with --graph)")
     a = p.parse_args()
     ctx = fdllm.Context(0)
-    r = run_lmhead(a, ctx) if a.op == "lmhead" else run_attention(a, ctx)
+    if a.op == "lmhead":
+        r = run_lmhead(a, ctx)
+    elif a.op == "attention":
+        r = run_attention(a, ctx)
+    else:
+        r = run_linear(a, ctx)
     print(json.dumps(r), flush=True)
     ctx.close()
 

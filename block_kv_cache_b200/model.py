@@ -143,8 +143,17 @@ class BlockDecoder:
         self.xn = torch.empty((rb, D), dtype=torch.bfloat16, device=dev)
         self.conf = torch.empty(rb, dtype=torch.float32, device=dev)
         self.tok = torch.empty(rb, dtype=torch.int32, device=dev)
-        self.remaining = torch.empty(batch, dtype=torch.int32, device=dev)
-        self.n_decoded = torch.empty(batch, dtype=torch.int32, device=dev)
+        # per-step counters (remaining masked in the block, decoded this step),
+        # read back by the host after every step
+        self.counts = torch.zeros((2, batch), dtype=torch.int32, device=dev)
+        self.remaining, self.n_decoded = self.counts[0], self.counts[1]
+        self.counts_host = torch.zeros((2, batch), dtype=torch.int32).pin_memory()
+        # decode state (device-resident for the whole decode)
+        self.x = torch.empty((batch, seq_len), dtype=torch.int32, device=dev)
+        self.masked = torch.empty((batch, seq_len), dtype=torch.uint8, device=dev)
+        self.graphs = {}
+        self.graph_timers = {}          # graph key -> [(event, event)] around SwiGLU GEMMs
+        self._timers = None
         # rows of block k of every sequence in the flattened [b * L] token rows
         nblk = (seq_len + block - 1) // block
         i = np.arange(block)
@@ -178,7 +187,14 @@ class BlockDecoder:
                                         ws=self.ws_att)
             ctx.linear_residual(o.view(rows, -1), Lw["wo"], h)
             ctx.rmsnorm(h, Lw["ffn_norm"], sh.rms_eps, out=x)
+            if self._timers is not None:
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record()
             ctx.linear_swiglu(x, Lw["w_gu"], out=f)
+            if self._timers is not None:
+                e1.record()
+                self._timers.append((e0, e1))
             ctx.linear_residual(f, Lw["wd"], h)
 
     def refresh(self, x_ids, s):
@@ -250,3 +266,68 @@ class BlockDecoder:
                     break
                 kind = "cached"
         return x, steps
+
+    # ------------------------------------------------------- graph-replayed decode
+    def _step_calls(self, kind, s, tau):
+        if kind == "refresh":
+            self.refresh(self.x, s)
+        else:
+            self.block_step(self.x, s)
+        self.unmask(self.x, self.masked, s, tau)
+        self.counts_host.copy_(self.counts, non_blocking=True)
+
+    def capture(self, kind, s, tau, time_swiglu=False):
+        """CUDA graph of one decode step (forward, unmask, counter read-back) for
+        block start s; kernels read and write the decoder's own x / masked. With
+        time_swiglu, timing events bracket every layer's SwiGLU GEMM."""
+        key = (kind, s, float(tau))
+        if key not in self.graphs:
+            g = torch.cuda.CUDAGraph()
+            self._timers = [] if time_swiglu else None
+            with torch.cuda.graph(g):
+                self._step_calls(kind, s, tau)
+            self.graph_timers[key] = self._timers or []
+            self._timers = None
+            self.graphs[key] = g
+        return self.graphs[key]
+
+    def last_timers(self):
+        """Event pairs of the graph replayed by the last step()."""
+        return self.graph_timers.get(self._last_key, [])
+
+    def capture_all(self, prompt_len, gen_len, tau, time_swiglu=False):
+        for blk in range(gen_len // self.B):
+            s = prompt_len + blk * self.B
+            self.capture("refresh", s, tau, time_swiglu)
+            self.capture("cached", s, tau, time_swiglu)
+        torch.cuda.synchronize()
+
+    def begin(self, prompt, tau):
+        """Start a decode of prompt [b, P] (host or device int32)."""
+        b, P = prompt.shape
+        self.P, self.tau = P, float(tau)
+        self.x.fill_(self.sh.mask_id)
+        self.x[:, :P].copy_(torch.as_tensor(prompt, dtype=torch.int32), non_blocking=True)
+        self.masked.zero_()
+        self.masked[:, P:] = 1
+        self.blk, self.kind, self.done = 0, "refresh", False
+        self.steps = 0
+
+    def step(self):
+        """One decode step (graph replay). Returns tokens decoded by this step."""
+        s = self.P + self.blk * self.B
+        self._last_key = (self.kind, s, self.tau)
+        self.last_kind = self.kind
+        self.capture(self.kind, s, self.tau).replay()
+        torch.cuda.current_stream().synchronize()
+        rem = int(self.counts_host[0].max())
+        nd = int(self.counts_host[1].sum())
+        self.steps += 1
+        if rem == 0:
+            self.blk += 1
+            self.kind = "refresh"
+            if self.P + self.blk * self.B >= self.L:
+                self.done = True
+        else:
+            self.kind = "cached"
+        return nd

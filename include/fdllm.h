@@ -65,10 +65,14 @@ typedef struct fdl_ctx fdl_ctx;   /* opaque: device id, device error word, launc
 /* ABI version of the loaded library (FDL_ABI_VERSION it was built with). */
 FDL_API int fdl_abi_version(void);
 
-/* Create a context on CUDA device `device`. Allocates the 4-byte device error
- * word (the only allocation the library makes, once, here) and reads the
- * device's properties. Fails with FDL_EUNSUPPORTED unless the device is
- * compute capability 10.0 (B200). *out is set to NULL on failure. */
+/* Create a context on CUDA device `device`. Allocates, once, here (the only
+ * allocations the library makes): the 4-byte device error word and a 32 MiB
+ * zero-filled f32 accumulator used by the few-token projections to add
+ * split-K partial sums (every kernel that adds into it leaves it zeroed).
+ * Because of that shared accumulator, the calls made on one context must be
+ * ordered on the GPU (one stream, or streams ordered by events); use one
+ * context per concurrent stream. Fails with FDL_EUNSUPPORTED unless the device
+ * is compute capability 10.0 (B200). *out is set to NULL on failure. */
 FDL_API int fdl_create(fdl_ctx** out, int device);
 
 /* Free the context and its error word. NULL is accepted. */

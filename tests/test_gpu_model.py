@@ -70,7 +70,9 @@ def test_embed_gather_exact(ctx):
     assert np.array_equal(out.cpu().numpy(), table[ids.reshape(-1)[rm]])
 
 
-@pytest.mark.parametrize("M,N,K", [(32, 4096, 4096), (300, 512, 256), (1, 64, 64), (129, 320, 192)])
+@pytest.mark.parametrize("M,N,K", [(32, 4096, 4096), (300, 512, 256), (1, 64, 64), (129, 320, 192),
+                                   (32, 4096, 12288), (200, 1024, 512), (1, 128, 64),
+                                   (64, 12288, 4096)])
 def test_linear_residual(ctx, M, N, K):
     g = synth.rng(M + N)
     x = bf_vals(g.standard_normal((M, K)))
@@ -82,7 +84,8 @@ def test_linear_residual(ctx, M, N, K):
     assert rel(h.cpu().numpy(), ref) <= 1e-4
 
 
-@pytest.mark.parametrize("M,F,K", [(32, 1024, 512), (257, 96, 128)])
+@pytest.mark.parametrize("M,F,K", [(32, 1024, 512), (257, 96, 128), (32, 12288, 4096),
+                                   (100, 256, 256)])
 def test_linear_swiglu(ctx, M, F, K):
     g = synth.rng(M + F)
     x = bf_vals(g.standard_normal((M, K)))
