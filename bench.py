@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=40)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-steps", action="store_true",
+                   help="also print the per-call time of a cached step and of a refresh")
     return p.parse_args()
 
 
@@ -251,6 +253,10 @@ def run_gpu(args):
             "cpu_baseline": cpu,
         }
         print(json.dumps(out), flush=True)
+    if args.profile_steps and rank == 0:
+        s0 = c["prompt"] + dec.blk * c["block"] if not dec.done else c["prompt"]
+        prof = {k: dec.profile_step(k, s0, c["tau"]) for k in ("cached", "refresh")}
+        print(json.dumps({"profile_us_per_step": prof}), flush=True)
     dec.graphs.clear()
     ctx.close()
     if world > 1:

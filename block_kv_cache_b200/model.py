@@ -331,3 +331,47 @@ class BlockDecoder:
         else:
             self.kind = "cached"
         return nd
+
+    # ------------------------------------------------------------------ profiling
+    def profile_step(self, kind, s, tau, reps=5):
+        """Per-call GPU time of one decode step: the step is captured in a CUDA
+        graph with timing events around every library call and replayed (the
+        events serialise neighbouring kernels, so this shows where a step's time
+        goes rather than the overlapped total). Returns {call: mean us per step}."""
+        ctx = self.ctx
+        pairs = []
+        orig = {}
+
+        def wrap(name):
+            fn = getattr(ctx, name)
+            orig[name] = fn
+
+            def timed(*a, **k):
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record()
+                r = fn(*a, **k)
+                e1.record()
+                pairs.append((name, e0, e1))
+                return r
+            setattr(ctx, name, timed)
+
+        calls = ["rmsnorm", "embed", "qkv_rope_store", "full_attention", "dualcache_attention",
+                 "linear_residual", "linear_swiglu", "lmhead_confidence", "threshold_unmask"]
+        for n in calls:
+            wrap(n)
+        g = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(g):
+                self._step_calls(kind, s, tau)
+        finally:
+            for n, fn in orig.items():
+                setattr(ctx, n, fn)
+        tot = {}
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            for name, a, b in pairs:
+                tot[name] = tot.get(name, 0.0) + a.elapsed_time(b) * 1e3
+        del g
+        return {n: v / reps for n, v in tot.items()}
