@@ -1,7 +1,7 @@
 // C-ABI entry points of the Fast-dLLM step library: argument validation,
 // device selection, workspace checks and dispatch to the kernels. See
 // include/fdllm.h for the contract of every function.
-#include "../../include/fdllm.h"
+#include "fdllm.h"
 #include "launch.h"
 #include "common.cuh"
 
@@ -396,8 +396,8 @@ int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_feature
     fdl::GemmShape gs{rows, out_features, in_features};
     const fdl::EpiResid ep{h, out_features};
     cudaError_t e = fdl::skinny_ok(gs)
-        ? fdl::launch_skinny_resid(gs, x, w, ep, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
-                                   ctx->d_err, (cudaStream_t)stream)
+        ? fdl::launch_skinny_resid(gs, x, w, ep, ctx->sm_count, ctx->d_err,
+                                   (cudaStream_t)stream)
         : fdl::launch_gemm_resid(gs, x, w, ep, ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_residual launch");
 }

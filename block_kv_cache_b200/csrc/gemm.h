@@ -41,8 +41,7 @@ cudaError_t launch_gemm_qkv(const GemmShape& g, const void* a, const void* w, co
 // Token-few variants (M <= 256, N % 128 == 0): weight rows on the MMA's M side.
 bool skinny_ok(const GemmShape& g);
 cudaError_t launch_skinny_resid(const GemmShape& g, const void* x, const void* w,
-                                const EpiResid& p, float* acc, size_t acc_bytes, int sm_count,
-                                int* err, cudaStream_t st);
+                                const EpiResid& p, int sm_count, int* err, cudaStream_t st);
 // acc: f32 scratch of acc_bytes, all zeros; split-K partial sums go there and
 // the finishing kernel restores the zeros. Too small or NULL: no K split.
 cudaError_t launch_skinny_swiglu(const GemmShape& g, const void* x, const void* w,

@@ -16,6 +16,10 @@
 // 128-byte swizzle), warp 1 TMEM owner + single-thread tcgen05.mma (M=128,
 // N=NT, K=16) into two NT-column accumulators, warps 2-5 epilogue with
 // thread = weight row (output feature), columns = tokens.
+//
+// The weights never depend on the kernel before this one, so under
+// programmatic dependent launch the TMA warp requests the first ring of weight
+// tiles before it waits for that kernel; only the activation boxes wait.
 #include "common.cuh"
 #include "gemm.h"
 #include "sm100.cuh"
@@ -52,7 +56,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
 struct SkResid {
     EpiResid p;
     int split;          // > 1: partial sums are added atomically
-    static constexpr bool kSplitK = true;
     __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
 #pragma unroll 4
         for (int j = 0; j < 32; ++j) {
@@ -66,26 +69,8 @@ struct SkResid {
     }
 };
 
-// Split-K partial sums of a non-linear projection: acc[t][f] += C (f32,
-// token-major: for one token a warp's 32 features are one 128-byte line, so
-// each atomic instruction is a single coalesced L2 request); the epilogue
-// proper runs in a finish_* kernel that also restores the zeros.
-struct SkAccum {
-    float* acc;
-    int ldn;
-    static constexpr bool kSplitK = true;
-    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
-#pragma unroll 4
-        for (int j = 0; j < 32; ++j) {
-            const int t = j0 + j;
-            if (t < M) atomicAdd(acc + (size_t)t * ldn + f, v[j]);
-        }
-    }
-};
-
 struct SkSwiGLU {
     EpiSwiGLU p;
-    static constexpr bool kSplitK = false;
     // rows 2g and 2g+1 of the tile are gate and up of feature g: adjacent lanes
     __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
         const int lane = threadIdx.x & 31;
@@ -104,7 +89,6 @@ struct SkSwiGLU {
 
 struct SkQKV {
     EpiQKV p;
-    static constexpr bool kSplitK = false;
     // one tile = one head (128 dims); RoPE partners are 64 rows apart, so the
     // chunk is exchanged through shared memory (row = dim, 32 tokens, +1 pad)
     __device__ void chunk(int f, int M, int j0, const float* v, uint8_t* xbuf, int n0) const {
@@ -120,6 +104,15 @@ struct SkQKV {
         asm volatile("bar.sync 1, 128;" ::: "memory");
         const float bias = p.bias ? p.bias[f] : 0.f;
         const float pb = (rot && p.bias) ? p.bias[n0 + (r ^ 64)] : 0.f;
+        float2 cs[32];                             // all table loads in flight at once
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            cs[j] = rot && t < M
+                        ? __ldg(p.rope + (size_t)(p.pos0 + t % p.rows_per_seq) * (D / 2) + (r & 63))
+                        : make_float2(1.f, 0.f);
+        }
+#pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int t = j0 + j;
             if (t >= M) break;
@@ -127,8 +120,7 @@ struct SkQKV {
             float y = v[j] + bias;
             if (rot) {
                 const float other = xs[(r ^ 64) * 33 + j] + pb;
-                const float2 cs = p.rope[(size_t)pos * (D / 2) + (r & 63)];
-                y = r < 64 ? y * cs.x - other * cs.y : other * cs.y + y * cs.x;
+                y = r < 64 ? y * cs[j].x - other * cs[j].y : other * cs[j].y + y * cs[j].x;
             }
             bf16* dst;
             if (n0 < nq)
@@ -142,6 +134,22 @@ struct SkQKV {
             *dst = __float2bfloat16_rn(y);
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");   // exchange buffer free again
+    }
+};
+
+// Split-K partial sums of a non-linear projection: acc[t][f] += C (f32,
+// token-major: for one token a warp's 32 features are one 128-byte line, so
+// each atomic instruction is a single coalesced L2 request); the epilogue
+// proper runs in a finish_* kernel that also restores the zeros.
+struct SkAccum {
+    float* acc;
+    int ldn;
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            if (t < M) atomicAdd(acc + (size_t)t * ldn + f, v[j]);
+        }
     }
 };
 
@@ -185,7 +193,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    pdl_wait();
+    if (warp != 0) pdl_wait();
     pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -193,21 +201,37 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         if (lane == 0) {
             prefetch_tmap(&tmW);
             prefetch_tmap(&tmX);
-            int stage = 0;
+            // (item, k) steps of this CTA in order; the first npre of them get
+            // their weight boxes before the dependency wait
+            int npre = 0;
+            for (int item = blockIdx.x; npre < S::STAGES && item < num_items; item += gridDim.x) {
+                const int n_tile = item / splits, ks = item % splits;
+                const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
+                for (int k = k0; npre < S::STAGES && k < k1; ++k, ++npre) {
+                    mbar_arrive_expect_tx(full_bar(npre), S::STAGE);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_2d(sA(npre) + c * S::A_CHUNK, &tmW, full_bar(npre),
+                                    k * SK_BK + c * 64, n_tile * SK_BM);
+                }
+            }
+            pdl_wait();
+            int stage = 0, n = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
                 const int n_tile = item / splits, ks = item % splits;
                 const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
-                for (int k = k0; k < k1; ++k) {
-                    if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
-                    mbar_arrive_expect_tx(full_bar(stage), S::STAGE);
-                    for (int c = 0; c < 2; ++c) {
-                        tma_load_2d(sA(stage) + c * S::A_CHUNK, &tmW, full_bar(stage),
-                                    k * SK_BK + c * 64, n_tile * SK_BM);
+                for (int k = k0; k < k1; ++k, ++n) {
+                    if (n >= npre) {
+                        if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
+                        mbar_arrive_expect_tx(full_bar(stage), S::STAGE);
+                        for (int c = 0; c < 2; ++c)
+                            tma_load_2d(sA(stage) + c * S::A_CHUNK, &tmW, full_bar(stage),
+                                        k * SK_BK + c * 64, n_tile * SK_BM);
+                    }
+                    for (int c = 0; c < 2; ++c)
                         tma_load_2d(sB(stage) + c * S::B_CHUNK, &tmX, full_bar(stage),
                                     k * SK_BK + c * 64, 0);
-                    }
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -327,18 +351,24 @@ int choose_splits(const GemmShape& g, int sm_count, int max_splits) {
 }
 
 // ---- epilogues of split-K projections: consume the f32 sums, leave zeros ----------
+// SwiGLU: thread = 4 consecutive features of one token (two float4 of
+// interleaved gate/up sums in, 8 bytes of bf16 out).
 __global__ void finish_swiglu_kernel(float* __restrict__ acc, int M, int F, bf16* __restrict__ out,
                                      int ldo) {
     pdl_wait();
     pdl_trigger();
-    const size_t n = (size_t)M * F;
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
-         e += (size_t)gridDim.x * blockDim.x) {
-        const size_t t = e / F, f = e % F;
-        float2* pg = reinterpret_cast<float2*>(acc + t * 2 * F + 2 * f);
-        const float2 gu = *pg;
-        *pg = make_float2(0.f, 0.f);
-        out[t * ldo + f] = __float2bfloat16_rn(gu.x / (1.f + __expf(-gu.x)) * gu.y);
+    const int fq = F / 4;
+    const int n = M * fq;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+        const int t = e / fq, f = (e - t * fq) * 4;
+        float4* pg = reinterpret_cast<float4*>(acc + (size_t)t * 2 * F + 2 * f);
+        const float4 a = __ldcs(pg), b = __ldcs(pg + 1);
+        __stcs(pg, make_float4(0.f, 0.f, 0.f, 0.f));
+        __stcs(pg + 1, make_float4(0.f, 0.f, 0.f, 0.f));
+        uint2 o;
+        o.x = pack2(a.x / (1.f + __expf(-a.x)) * a.y, a.z / (1.f + __expf(-a.z)) * a.w);
+        o.y = pack2(b.x / (1.f + __expf(-b.x)) * b.y, b.z / (1.f + __expf(-b.z)) * b.w);
+        *reinterpret_cast<uint2*>(out + (size_t)t * ldo + f) = o;
     }
 }
 
@@ -376,10 +406,7 @@ __global__ void finish_qkv_kernel(float* __restrict__ acc, int M, EpiQKV p) {
 bool skinny_ok(const GemmShape& g) { return g.M <= 256 && g.N % SK_BM == 0 && g.K % SK_BK == 0; }
 
 cudaError_t launch_skinny_resid(const GemmShape& g, const void* x, const void* w,
-                                const EpiResid& p, float* acc, size_t acc_bytes, int sm_count,
-                                int* err, cudaStream_t st) {
-    (void)acc;
-    (void)acc_bytes;
+                                const EpiResid& p, int sm_count, int* err, cudaStream_t st) {
     // partial sums go straight into the f32 residual stream (coalesced atomics)
     const int splits = choose_splits(g, sm_count, 16);
     return dispatch_skinny(g, x, w, SkResid{p, splits}, splits, sm_count, err, st);
@@ -393,8 +420,8 @@ cudaError_t launch_skinny_swiglu(const GemmShape& g, const void* x, const void* 
     if (splits == 1) return dispatch_skinny(g, x, w, SkSwiGLU{p}, 1, sm_count, err, st);
     cudaError_t e = dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st);
     if (e != cudaSuccess) return e;
-    const size_t n = (size_t)g.M * (g.N / 2);
-    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+    const int n = g.M * (g.N / 8);                 // 4 output features per thread
+    const int blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
     return launch_pdl(finish_swiglu_kernel, dim3(blocks), dim3(256), 0, st, 0, acc, g.M, g.N / 2,
                       p.out, p.ldo);
 }

@@ -14,7 +14,7 @@
 
 #include <mutex>
 
-#include "../../include/fdllm.h"
+#include "fdllm.h"
 #include "launch.h"
 #include "lmhead_common.cuh"
 
