@@ -227,14 +227,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 const int st = t % STAGES;
                 if (!(ok = mbar_wait(kv_empty(st), ((t / STAGES) & 1) ^ 1, abort_flag, a.err)))
                     break;
+                // one copy per tile and operand: all D columns as DC sub-tiles
                 mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
-                for (int dc = 0; dc < S::DC; ++dc)
-                    tma_load_2d(sb + S::OFF_K + st * S::KV_TILE + dc * S::KV_CHUNK, &tmK,
-                                k_full(st), dc * 64, krow0 + t * KT);
+                tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0, krow0 + t * KT, 0);
                 mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
-                for (int dc = 0; dc < S::DC; ++dc)
-                    tma_load_2d(sb + S::OFF_V + st * S::KV_TILE + dc * S::KV_CHUNK, &tmV,
-                                v_full(st), dc * 64, krow0 + t * KT);
+                tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0, krow0 + t * KT, 0);
             }
             // tail: every stage handed out has been released again
             for (int u = t; ok && u < t + STAGES; ++u)
@@ -510,9 +507,9 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
     cudaError_t e = make_tmap_bf16(&tq, q, 3, qdims, qstr, qbox);
     if (e != cudaSuccess) return e;
     const uint64_t kv_rows = (uint64_t)(s.batch / s.q_per_kv) * s.n_kv_heads * s.seq_len;
-    e = make_tmap_bf16_2d(&tk, k, kv_rows, D, ATT_KT, 64);
+    e = make_tmap_bf16_rows(&tk, k, kv_rows, D, ATT_KT, D / 64);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_2d(&tv, v, kv_rows, D, ATT_KT, 64);
+    e = make_tmap_bf16_rows(&tv, v, kv_rows, D, ATT_KT, D / 64);
     if (e != cudaSuccess) return e;
     AttnArgs a;
     a.out = (bf16*)out;

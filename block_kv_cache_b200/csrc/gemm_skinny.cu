@@ -11,9 +11,9 @@
 // 256-wide token-major tiles; the residual projections also split K so that
 // every SM streams (partial sums added atomically into the f32 residual).
 //
-// Persistent, warp-specialised: warp 0 TMA (ring of 128-wide K steps, each two
-// 64-column boxes of the 128-row weight tile and of the NT activation rows,
-// 128-byte swizzle), warp 1 TMEM owner + single-thread tcgen05.mma (M=128,
+// Persistent, warp-specialised: warp 0 TMA (ring of 128-wide K steps, each one
+// copy of the 128-row weight tile and one of the NT activation rows, landing
+// as two 64-column 128-byte-swizzled sub-tiles), warp 1 TMEM owner + single-thread tcgen05.mma (M=128,
 // N=NT, K=16) into two NT-column accumulators, warps 2-5 epilogue with
 // thread = weight row (output feature), columns = tokens.
 //
@@ -37,7 +37,8 @@ struct Sk {
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int STAGES = (176 * 1024) / STAGE > 8 ? 8 : (176 * 1024) / STAGE;
     static constexpr int OFF_X = STAGES * STAGE;             // epilogue exchange (QKV)
-    static constexpr int X_BYTES = SK_BM * 33 * 4;           // 128 rows x 32 tokens (+1 pad)
+    // exchange buffer: RoPE partners (128 rows x 33) or the split-K transpose (32 x 132)
+    static constexpr int X_BYTES = SK_BM * 33 * 4;
     static constexpr int OFF_BAR = OFF_X + X_BYTES;
     static constexpr size_t TOTAL = 1024 + OFF_BAR + 256;
     static constexpr uint32_t TMEM_COLS = 2 * NT < 32 ? 32 : 2 * NT;
@@ -50,21 +51,45 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Each epilogue gets (TMEM address of its lane's accumulator row, feature
-// index within [0, N), token count M, first token of the 32-token chunk, the
-// 32 accumulator values of the chunk).
+// Each epilogue gets (feature index within [0, N), token count M, first token
+// of the 32-token chunk, the 32 accumulator values of the chunk, the shared
+// exchange buffer, first feature of the tile).
+
+// dst[t * ld + n0 + c] += C[c][t] for the tile's 128 features c and the chunk's
+// tokens t < M, with 16-byte vector atomics: the chunk is transposed through
+// shared memory (token-major, rows of 132 floats) so that a thread adds 4
+// consecutive features of one token and a warp instruction covers 128
+// consecutive features (512 bytes): a quarter of the atomic operations of one
+// per element, which the L2 has to absorb when several splits add into a tile.
+__device__ __forceinline__ void add_tile_v4(float* dst, int ld, int n0, int M, int j0, int r,
+                                            const float* v, uint8_t* xbuf) {
+    float* xs = reinterpret_cast<float*>(xbuf);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) xs[j * 132 + r] = v[j];
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int et = threadIdx.x - 64;                 // epilogue thread 0..127
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = et + 128 * k, g4 = i & 31, tl = i >> 5;
+        if (j0 + tl < M)
+            atomicAdd(reinterpret_cast<float4*>(dst + (size_t)(j0 + tl) * ld + n0 + 4 * g4),
+                      *reinterpret_cast<const float4*>(xs + tl * 132 + 4 * g4));
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // exchange buffer free again
+}
+
 struct SkResid {
     EpiResid p;
     int split;          // > 1: partial sums are added atomically
-    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t* xbuf, int n0) const {
+        if (split > 1) {
+            add_tile_v4(p.h, p.ldh, n0, M, j0, f - n0, v, xbuf);
+            return;
+        }
 #pragma unroll 4
         for (int j = 0; j < 32; ++j) {
             const int t = j0 + j;
-            if (t < M) {
-                float* dst = p.h + (size_t)t * p.ldh + f;
-                if (split > 1) atomicAdd(dst, v[j]);
-                else *dst += v[j];
-            }
+            if (t < M) p.h[(size_t)t * p.ldh + f] += v[j];
         }
     }
 };
@@ -138,18 +163,13 @@ struct SkQKV {
 };
 
 // Split-K partial sums of a non-linear projection: acc[t][f] += C (f32,
-// token-major: for one token a warp's 32 features are one 128-byte line, so
-// each atomic instruction is a single coalesced L2 request); the epilogue
-// proper runs in a finish_* kernel that also restores the zeros.
+// token-major); the epilogue proper runs in a finish_* kernel that also
+// restores the zeros.
 struct SkAccum {
     float* acc;
     int ldn;
-    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t*, int) const {
-#pragma unroll 4
-        for (int j = 0; j < 32; ++j) {
-            const int t = j0 + j;
-            if (t < M) atomicAdd(acc + (size_t)t * ldn + f, v[j]);
-        }
+    __device__ void chunk(int f, int M, int j0, const float* v, uint8_t* xbuf, int n0) const {
+        add_tile_v4(acc, ldn, n0, M, j0, f - n0, v, xbuf);
     }
 };
 
@@ -209,9 +229,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
                 for (int k = k0; npre < S::STAGES && k < k1; ++k, ++npre) {
                     mbar_arrive_expect_tx(full_bar(npre), S::STAGE);
-                    for (int c = 0; c < 2; ++c)
-                        tma_load_2d(sA(npre) + c * S::A_CHUNK, &tmW, full_bar(npre),
-                                    k * SK_BK + c * 64, n_tile * SK_BM);
+                    tma_load_3d(sA(npre), &tmW, full_bar(npre), 0, n_tile * SK_BM, k * 2);
                 }
             }
             pdl_wait();
@@ -225,13 +243,9 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                     if (n >= npre) {
                         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
                         mbar_arrive_expect_tx(full_bar(stage), S::STAGE);
-                        for (int c = 0; c < 2; ++c)
-                            tma_load_2d(sA(stage) + c * S::A_CHUNK, &tmW, full_bar(stage),
-                                        k * SK_BK + c * 64, n_tile * SK_BM);
+                        tma_load_3d(sA(stage), &tmW, full_bar(stage), 0, n_tile * SK_BM, k * 2);
                     }
-                    for (int c = 0; c < 2; ++c)
-                        tma_load_2d(sB(stage) + c * S::B_CHUNK, &tmX, full_bar(stage),
-                                    k * SK_BK + c * 64, 0);
+                    tma_load_3d(sB(stage), &tmX, full_bar(stage), 0, 0, k * 2);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -307,9 +321,10 @@ cudaError_t run_skinny(const GemmShape& g, const void* x, const void* w, const E
                        int splits, int sm_count, int* err, cudaStream_t st) {
     using S = Sk<NT>;
     CUtensorMap tw, tx;
-    cudaError_t e = make_tmap_bf16_2d(&tw, w, g.N, g.K, SK_BM, 64);
+    // one copy per K step and operand: 128 columns as two 64-column sub-tiles
+    cudaError_t e = make_tmap_bf16_rows(&tw, w, g.N, g.K, SK_BM, 2);
     if (e != cudaSuccess) return e;
-    e = make_tmap_bf16_2d(&tx, x, g.M, g.K, NT, 64);
+    e = make_tmap_bf16_rows(&tx, x, g.M, g.K, NT, 2);
     if (e != cudaSuccess) return e;
     const int items = (g.N / SK_BM) * splits;
     const int grid = items < sm_count ? items : sm_count;

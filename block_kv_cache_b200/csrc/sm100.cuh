@@ -258,6 +258,14 @@ __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
 cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                               uint32_t box_rows, uint32_t box_cols);
 
+// Tensor map over a row-major [rows, cols] bf16 matrix (cols % 64 == 0) whose
+// box is box_rows rows x (n_chunks * 64) columns, delivered as n_chunks
+// consecutive [box_rows][64] sub-tiles of 128-byte rows (128-byte swizzle):
+// the K-major operand layout of the MMAs, fetched with one copy instead of
+// one per 64 columns. Copy coordinates: (0, row, first chunk).
+cudaError_t make_tmap_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                uint32_t box_rows, uint32_t n_chunks);
+
 // General rank-2..5 bf16 tensor map, 128-byte swizzle: dims[0] is the
 // contiguous dimension (box[0] must be 64 elements = 128 bytes);
 // strides_bytes[i] is the byte stride of dimension i+1 (multiple of 16).

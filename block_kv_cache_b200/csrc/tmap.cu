@@ -62,4 +62,15 @@ cudaError_t make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows,
     return make_tmap_bf16(map, base, 2, dims, strides, box);
 }
 
+cudaError_t make_tmap_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                                uint32_t box_rows, uint32_t n_chunks) {
+    if (cols % 64 || n_chunks < 1 || n_chunks * 64 > cols) return cudaErrorInvalidValue;
+    // (element within a 64-wide chunk, row, chunk): one copy lands as n_chunks
+    // consecutive [box_rows][64] sub-tiles
+    const uint64_t dims[3] = {64, rows, cols / 64};
+    const uint64_t strides[2] = {cols * 2, 128};
+    const uint32_t box[3] = {64, box_rows, n_chunks};
+    return make_tmap_bf16(map, base, 3, dims, strides, box);
+}
+
 }  // namespace fdl

@@ -40,6 +40,9 @@ class AttnDesc(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
+ABI_VERSION = 1
+
+
 class LMHeadDesc(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int), ("hidden", ctypes.c_int),
                 ("vocab", ctypes.c_int), ("dtype", ctypes.c_int)]
@@ -78,6 +81,9 @@ def load() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.fdl_abi_version.restype = i
+    if L.fdl_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"{LIB_PATH} has ABI {L.fdl_abi_version()}, this binding expects "
+                           f"{ABI_VERSION}: rebuild with `python -m block_kv_cache_b200.build`")
     L.fdl_create.argtypes = [ctypes.POINTER(vp), i]
     L.fdl_destroy.argtypes = [vp]
     L.fdl_last_error.restype = ctypes.c_char_p

@@ -29,7 +29,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     for name in declared:
         assert hasattr(L, name), name
     assert set(fdllm.EXPORTS) <= set(declared)
-    assert L.fdl_abi_version() == 1
+    assert L.fdl_abi_version() == fdllm.ABI_VERSION
 
 
 def test_null_arguments_rejected_without_device():
