@@ -17,11 +17,13 @@ struct fdl_ctx {
     int* d_err;              // device error word (4 bytes)
     float* d_acc;            // split-K accumulator of the projections, kept all zeros
     size_t acc_bytes;
+    unsigned* d_sync;        // grid-barrier words of the fused kernels (zeroed)
 };
 
 // Split-K accumulator of the few-token projections (zeroed at creation; every
 // kernel that adds into it leaves it zeroed again): room for 256 rows x 32768.
 static const size_t kAccBytes = (size_t)256 * 32768 * 4;
+static const size_t kSyncBytes = 256;
 
 namespace {
 
@@ -124,15 +126,19 @@ int fdl_create(fdl_ctx** out, int device) {
     c->sm_count = prop.multiProcessorCount;
     c->d_err = nullptr;
     c->d_acc = nullptr;
+    c->d_sync = nullptr;
     c->acc_bytes = kAccBytes;
     e = cudaMalloc(&c->d_err, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(int));
     if (e == cudaSuccess) e = cudaMalloc(&c->d_acc, kAccBytes);
     if (e == cudaSuccess) e = cudaMemset(c->d_acc, 0, kAccBytes);
+    if (e == cudaSuccess) e = cudaMalloc(&c->d_sync, kSyncBytes);
+    if (e == cudaSuccess) e = cudaMemset(c->d_sync, 0, kSyncBytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {
         if (c->d_err) cudaFree(c->d_err);
         if (c->d_acc) cudaFree(c->d_acc);
+        if (c->d_sync) cudaFree(c->d_sync);
         delete c;
         return cuda_fail(e, "fdl_create: device buffers");
     }
@@ -145,6 +151,7 @@ int fdl_destroy(fdl_ctx* ctx) {
     DeviceGuard g(ctx->device);
     if (ctx->d_err) cudaFree(ctx->d_err);
     if (ctx->d_acc) cudaFree(ctx->d_acc);
+    if (ctx->d_sync) cudaFree(ctx->d_sync);
     delete ctx;
     return FDL_OK;
 }
@@ -420,6 +427,38 @@ int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
         : fdl::launch_gemm_swiglu(gs, x, w_gu, ep, ctx->sm_count, ctx->d_err,
                                   (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_swiglu launch");
+}
+
+int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const void* x, const void* w_gu,
+            const void* w_down, void* f, float* h, void* stream) {
+    if (!ctx) return fail(FDL_EINVAL, "ffn: ctx is NULL");
+    if (rows < 1 || hidden < 64 || hidden % 64 || ffn < 64 || ffn % 64)
+        return fail(FDL_EINVAL, "ffn: rows >= 1, hidden % 64 == 0, ffn % 64 == 0");
+    if (!x || !w_gu || !w_down || !f || !h) return fail(FDL_EINVAL, "ffn: NULL buffer");
+    if (!aligned16(x) || !aligned16(w_gu) || !aligned16(w_down) || !aligned16(f) ||
+        !aligned16(h))
+        return fail(FDL_EINVAL, "ffn: buffers must be 16-byte aligned");
+    DeviceGuard g(ctx->device);
+    cudaStream_t st = (cudaStream_t)stream;
+    const fdl::GemmShape gu{rows, 2 * ffn, hidden}, dn{rows, hidden, ffn};
+    cudaError_t e;
+    if (fdl::skinny_ok(gu) && fdl::skinny_ok(dn)) {
+        e = fdl::launch_skinny_ffn(gu, x, w_gu, w_down, (fdl::bf16*)f, h, hidden, ctx->d_acc,
+                                   ctx->acc_bytes, ctx->d_sync, ctx->sm_count, ctx->d_err, st);
+    } else {
+        const fdl::EpiSwiGLU es{(fdl::bf16*)f, ffn};
+        e = fdl::skinny_ok(gu)
+            ? fdl::launch_skinny_swiglu(gu, x, w_gu, es, ctx->d_acc, ctx->acc_bytes,
+                                        ctx->sm_count, ctx->d_err, st)
+            : fdl::launch_gemm_swiglu(gu, x, w_gu, es, ctx->sm_count, ctx->d_err, st);
+        if (e == cudaSuccess) {
+            const fdl::EpiResid er{h, hidden};
+            e = fdl::skinny_ok(dn)
+                ? fdl::launch_skinny_resid(dn, f, w_down, er, ctx->sm_count, ctx->d_err, st)
+                : fdl::launch_gemm_resid(dn, f, w_down, er, ctx->sm_count, ctx->d_err, st);
+        }
+    }
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "ffn launch");
 }
 
 int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,

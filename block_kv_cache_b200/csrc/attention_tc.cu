@@ -222,6 +222,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
                             bb * a.B);
             const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
+            const uint64_t kv_policy = l2_evict_first();
             int t = 0;
             for (; ok && t < nt; ++t) {
                 const int st = t % STAGES;
@@ -229,9 +230,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     break;
                 // one copy per tile and operand: all D columns as DC sub-tiles
                 mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
-                tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0, krow0 + t * KT, 0);
+                if (a.q_per_kv == 1)   // one query block: every K/V byte is read once
+                    tma_load_3d_hint(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
+                                     krow0 + t * KT, 0, kv_policy);
+                else
+                    tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
+                                krow0 + t * KT, 0);
                 mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
-                tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0, krow0 + t * KT, 0);
+                if (a.q_per_kv == 1)
+                    tma_load_3d_hint(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
+                                     krow0 + t * KT, 0, kv_policy);
+                else
+                    tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
+                                krow0 + t * KT, 0);
             }
             // tail: every stage handed out has been released again
             for (int u = t; ok && u < t + STAGES; ++u)

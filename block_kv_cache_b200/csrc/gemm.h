@@ -51,6 +51,15 @@ cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, 
                               float* acc, size_t acc_bytes, int sm_count, int* err,
                               cudaStream_t st);
 
+// Feed-forward block for M <= 256 rows: h[M, ld_h] += down(SwiGLU(x W_gu^T)),
+// w_gu [2F, K] interleaved (row 2f gate, 2f + 1 up), w_down [ld_h, F], f [M, F]
+// bf16 scratch (the down projection's operand). acc/acc_bytes as above; bar:
+// two zeroed words for the grid barrier of the down projection.
+cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* w_gu,
+                              const void* w_down, bf16* f, float* h, int ld_h, float* acc,
+                              size_t acc_bytes, unsigned* bar, int sm_count, int* err,
+                              cudaStream_t st);
+
 // out[i, :] = bf16(h[src_i, :] / sqrt(mean(h[src_i]^2) + eps) * weight), src_i =
 // row_map ? row_map[i] : i.
 cudaError_t launch_rmsnorm(int rows, int hidden, const float* h, const int32_t* row_map,

@@ -173,10 +173,65 @@ struct SkAccum {
     }
 };
 
-template <int NT, class Epi>
+// ---- prologues: work every CTA does after the preceding kernel, before the GEMM --
+struct NoPro {
+    static constexpr bool kActive = false;
+    unsigned* bar = nullptr;
+    __device__ void work(int, int) const {}
+};
+
+// The SwiGLU of a split-K gate/up projection, done by the CTAs of the GEMM that
+// consumes it (the down projection) instead of a kernel of its own: the CTAs
+// share out[t, f] = bf16(silu(g) * u) over the f32 sums acc[t, 2f + {0, 1}]
+// (restoring the zeros), then meet at a grid barrier before the TMA reads
+// `out` as the activation operand. Thread item = 4 consecutive features of
+// one token (two float4 of interleaved sums in, 8 bytes out).
+struct ProSwiGLU {
+    static constexpr bool kActive = true;
+    unsigned* bar;           // grid barrier words
+    float* acc;
+    int M, F;                // tokens, features
+    bf16* out;               // [M, F] row stride F: the GEMM's X
+    __device__ void work(int part, int nparts) const {
+        constexpr int U = 4;                         // items in flight per thread
+        const int fq = F / 4, n = M * fq, stride = nparts * blockDim.x;
+        for (int e0 = part * blockDim.x + threadIdx.x; e0 < n; e0 += U * stride) {
+            float4 a[U], b[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {           // every load first, then the math
+                const int e = e0 + u * stride;
+                if (e < n) {
+                    const int t = e / fq, f = (e - t * fq) * 4;
+                    const float4* pg = reinterpret_cast<const float4*>(acc + (size_t)t * 2 * F + 2 * f);
+                    a[u] = __ldcg(pg);
+                    b[u] = __ldcg(pg + 1);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * stride;
+                if (e < n) {
+                    const int t = e / fq, f = (e - t * fq) * 4;
+                    float4* pg = reinterpret_cast<float4*>(acc + (size_t)t * 2 * F + 2 * f);
+                    __stcg(pg, make_float4(0.f, 0.f, 0.f, 0.f));
+                    __stcg(pg + 1, make_float4(0.f, 0.f, 0.f, 0.f));
+                    uint2 o;
+                    o.x = pack2(a[u].x / (1.f + __expf(-a[u].x)) * a[u].y,
+                                a[u].z / (1.f + __expf(-a[u].z)) * a[u].w);
+                    o.y = pack2(b[u].x / (1.f + __expf(-b[u].x)) * b[u].y,
+                                b[u].z / (1.f + __expf(-b[u].z)) * b[u].w);
+                    *reinterpret_cast<uint2*>(out + (size_t)t * F + f) = o;
+                }
+            }
+        }
+    }
+};
+
+template <int NT, class Epi, class Pro>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   int M, int N, int K, int splits, int num_items, int* err, const Epi epi) {
+                   int M, int N, int K, int splits, int num_items, int* err, const Epi epi,
+                   const Pro pro) {
     using namespace sm100;
     using S = Sk<NT>;
     extern __shared__ uint8_t smem_raw[];
@@ -213,29 +268,42 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp != 0) pdl_wait();
-    pdl_trigger();
     const uint32_t tmem_base = *tmem_slot;
+
+    // (item, k) steps of this CTA in order; the first npre of them get their
+    // weight boxes before the dependency wait (the weights never depend on the
+    // preceding kernel)
+    int npre = 0;
+    int pre_k[S::STAGES];                            // K step of each of them
+    const uint64_t w_policy = l2_evict_first();      // weights: read once per call
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmW);
+        prefetch_tmap(&tmX);
+        for (int item = blockIdx.x; npre < S::STAGES && item < num_items; item += gridDim.x) {
+            const int n_tile = item / splits, ks = item % splits;
+            const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
+            for (int k = k0; npre < S::STAGES && k < k1; ++k, ++npre) {
+                pre_k[npre] = k;
+                mbar_arrive_expect_tx(full_bar(npre), S::STAGE);
+                tma_load_3d_hint(sA(npre), &tmW, full_bar(npre), 0, n_tile * SK_BM, k * 2,
+                                 w_policy);
+            }
+        }
+    }
+    pdl_wait();
+    if constexpr (Pro::kActive) {
+        pro.work(blockIdx.x, gridDim.x);
+        fence_proxy_async_global();                 // the TMA below reads what was written
+        grid_barrier(pro.bar, abort_flag, err);
+    }
+    pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tmap(&tmW);
-            prefetch_tmap(&tmX);
-            // (item, k) steps of this CTA in order; the first npre of them get
-            // their weight boxes before the dependency wait
-            int npre = 0;
-            for (int item = blockIdx.x; npre < S::STAGES && item < num_items; item += gridDim.x) {
-                const int n_tile = item / splits, ks = item % splits;
-                const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
-                for (int k = k0; npre < S::STAGES && k < k1; ++k, ++npre) {
-                    mbar_arrive_expect_tx(full_bar(npre), S::STAGE);
-                    tma_load_3d(sA(npre), &tmW, full_bar(npre), 0, n_tile * SK_BM, k * 2);
-                }
-            }
-            pdl_wait();
+            if constexpr (Pro::kActive) fence_proxy_async_global();
             int stage = 0, n = 0;
             uint32_t phase = 0;
-            bool ok = true;
+            bool ok = *abort_flag == 0;
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
                 const int n_tile = item / splits, ks = item % splits;
                 const int k0 = ks * kps, k1 = min(k_iters, k0 + kps);
@@ -243,15 +311,31 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                     if (n >= npre) {
                         if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
                         mbar_arrive_expect_tx(full_bar(stage), S::STAGE);
-                        tma_load_3d(sA(stage), &tmW, full_bar(stage), 0, n_tile * SK_BM, k * 2);
+                        tma_load_3d_hint(sA(stage), &tmW, full_bar(stage), 0, n_tile * SK_BM,
+                                         k * 2, w_policy);
                     }
                     tma_load_3d(sB(stage), &tmX, full_bar(stage), 0, 0, k * 2);
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
                 }
+                if (!ok) break;
             }
             for (int s = 0; ok && s < S::STAGES; ++s) {
                 ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err);
                 if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
+            }
+            if (!ok) {
+                // gave up: wait (bounded) until every copy issued into this
+                // CTA's shared memory has landed before the CTA may exit; a
+                // step whose weights went out early gets its activation box
+                // now, so that its barrier phase completes
+                for (int j = n; j < npre; ++j)
+                    tma_load_3d(sB(j), &tmX, full_bar(j), 0, 0, pre_k[j] * 2);
+                volatile int no_abort = 0;
+                const int issued = n > npre ? n : npre;
+                for (int s = 0; s < S::STAGES && s < issued; ++s) {
+                    const int j = s + ((issued - 1 - s) / S::STAGES) * S::STAGES;
+                    mbar_wait(full_bar(s), (uint32_t)((j / S::STAGES) & 1), &no_abort, err);
+                }
             }
         }
     } else if (warp == 1) {
@@ -316,9 +400,9 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
 }
 
-template <int NT, class Epi>
+template <int NT, class Epi, class Pro = NoPro>
 cudaError_t run_skinny(const GemmShape& g, const void* x, const void* w, const Epi& epi,
-                       int splits, int sm_count, int* err, cudaStream_t st) {
+                       int splits, int sm_count, int* err, cudaStream_t st, const Pro& pro = Pro{}) {
     using S = Sk<NT>;
     CUtensorMap tw, tx;
     // one copy per K step and operand: 128 columns as two 64-column sub-tiles
@@ -328,20 +412,21 @@ cudaError_t run_skinny(const GemmShape& g, const void* x, const void* w, const E
     if (e != cudaSuccess) return e;
     const int items = (g.N / SK_BM) * splits;
     const int grid = items < sm_count ? items : sm_count;
-    e = cudaFuncSetAttribute(gemm_skinny_kernel<NT, Epi>,
+    e = cudaFuncSetAttribute(gemm_skinny_kernel<NT, Epi, Pro>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::TOTAL);
     if (e != cudaSuccess) return e;
-    return launch_pdl(gemm_skinny_kernel<NT, Epi>, dim3(grid), dim3(SK_THREADS), S::TOTAL, st, 0,
-                      tw, tx, g.M, g.N, g.K, splits, items, err, epi);
+    return launch_pdl(gemm_skinny_kernel<NT, Epi, Pro>, dim3(grid), dim3(SK_THREADS), S::TOTAL, st,
+                      0, tw, tx, g.M, g.N, g.K, splits, items, err, epi, pro);
 }
 
-template <class Epi>
+template <class Epi, class Pro = NoPro>
 cudaError_t dispatch_skinny(const GemmShape& g, const void* x, const void* w, const Epi& epi,
-                            int splits, int sm_count, int* err, cudaStream_t st) {
-    if (g.M <= 32) return run_skinny<32>(g, x, w, epi, splits, sm_count, err, st);
-    if (g.M <= 64) return run_skinny<64>(g, x, w, epi, splits, sm_count, err, st);
-    if (g.M <= 128) return run_skinny<128>(g, x, w, epi, splits, sm_count, err, st);
-    return run_skinny<256>(g, x, w, epi, splits, sm_count, err, st);
+                            int splits, int sm_count, int* err, cudaStream_t st,
+                            const Pro& pro = Pro{}) {
+    if (g.M <= 32) return run_skinny<32>(g, x, w, epi, splits, sm_count, err, st, pro);
+    if (g.M <= 64) return run_skinny<64>(g, x, w, epi, splits, sm_count, err, st, pro);
+    if (g.M <= 128) return run_skinny<128>(g, x, w, epi, splits, sm_count, err, st, pro);
+    return run_skinny<256>(g, x, w, epi, splits, sm_count, err, st, pro);
 }
 
 // K splits: the (tiles x splits) work items should fill whole waves of the
@@ -451,6 +536,32 @@ cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, 
     if (e != cudaSuccess) return e;
     return launch_pdl(finish_qkv_kernel, dim3(g.M * (g.N / 128)), dim3(128), 0, st, 0, acc, g.M,
                       p);
+}
+
+// h += down(SwiGLU(x W_gu^T)) for few rows: the gate/up projection with split-K
+// partial sums in acc, then the down projection whose CTAs first turn the
+// sums into f = bf16(silu(g) * u) (grid barrier, no kernel in between).
+cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* w_gu,
+                              const void* w_down, bf16* f, float* h, int ld_h, float* acc,
+                              size_t acc_bytes, unsigned* bar, int sm_count, int* err,
+                              cudaStream_t st) {
+    const int F = g_gu.N / 2;
+    const GemmShape g_dn{g_gu.M, ld_h, F};
+    const int splits = acc && (size_t)g_gu.M * g_gu.N * 4 <= acc_bytes
+                           ? choose_splits(g_gu, sm_count, 8) : 1;
+    const EpiResid pr{h, ld_h};
+    const int dn_splits = choose_splits(g_dn, sm_count, 16);
+    cudaError_t e;
+    if (splits == 1) {
+        e = dispatch_skinny(g_gu, x, w_gu, SkSwiGLU{EpiSwiGLU{f, F}}, 1, sm_count, err, st);
+        if (e != cudaSuccess) return e;
+        return dispatch_skinny(g_dn, f, w_down, SkResid{pr, dn_splits}, dn_splits, sm_count, err,
+                               st);
+    }
+    e = dispatch_skinny(g_gu, x, w_gu, SkAccum{acc, g_gu.N}, splits, sm_count, err, st);
+    if (e != cudaSuccess) return e;
+    return dispatch_skinny(g_dn, f, w_down, SkResid{pr, dn_splits}, dn_splits, sm_count, err, st,
+                           ProSwiGLU{bar, acc, g_gu.M, F, f});
 }
 
 }  // namespace fdl

@@ -90,13 +90,18 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            const uint64_t w_policy = l2_evict_first();
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
                 const int m_tile = item % num_m, n_tile = item / num_m;
                 for (int k = 0; k < k_iters; ++k) {
                     if (!(ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err))) break;
                     mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
                     tma_load_2d(sA(stage), &tmA, full_bar(stage), k * BK, m_tile * BM);
-                    tma_load_2d(sB(stage), &tmB, full_bar(stage), k * BK, n_tile * BN);
+                    if (num_m == 1)                      // the vocabulary matrix is read once
+                        tma_load_2d_hint(sB(stage), &tmB, full_bar(stage), k * BK, n_tile * BN,
+                                         w_policy);
+                    else
+                        tma_load_2d(sB(stage), &tmB, full_bar(stage), k * BK, n_tile * BN);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }

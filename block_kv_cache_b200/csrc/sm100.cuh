@@ -36,6 +36,11 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's generic-proxy global accesses with later async-proxy
+// (TMA) accesses to global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -91,6 +96,46 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
     return __all_sync(0xffffffffu, ok);
 }
 
+// Barrier over every CTA of the grid. Only for grids whose CTAs are all
+// resident at once (persistent grids of at most one CTA per SM, launched when
+// nothing else can hold an SM indefinitely). bar[0] counts arrivals and bar[1]
+// is the generation; both start at zero and are left consistent for the next
+// use (the last CTA to arrive resets the count before it releases the
+// others). Bounded: a CTA that waits longer than the timeout raises *abort,
+// records DEV_TIMEOUT and returns false; afterwards the two words are no
+// longer consistent, so the caller's context has to be recreated.
+__device__ __forceinline__ bool grid_barrier(unsigned* bar, volatile int* abort, int* err) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        volatile unsigned* gen = bar + 1;
+        const unsigned g = *gen;                     // before arriving
+        __threadfence();
+        if (atomicAdd(bar, 1u) == gridDim.x * gridDim.y * gridDim.z - 1) {
+            atomicExch(bar, 0u);
+            __threadfence();
+            atomicAdd(bar + 1, 1u);
+        } else {
+            uint32_t n = 0;
+            uint64_t t0 = 0;
+            while (*gen == g) {
+                if ((++n & 63u) == 0) {
+                    const uint64_t now = globaltimer();
+                    if (t0 == 0) {
+                        t0 = now;
+                    } else if (now - t0 > kWaitTimeoutNs) {
+                        *abort = 1;
+                        record_error(err, DEV_TIMEOUT);
+                        break;
+                    }
+                }
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return *abort == 0;
+}
+
 // 2-D TMA tile load global -> shared, completion counted on `bar` in bytes.
 // c0 is the innermost (contiguous) coordinate in elements; c0 * elem_size must
 // be a multiple of 16 bytes.
@@ -110,6 +155,37 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// L2 policy for data read once per pass (weights, K/V caches streamed past a
+// handful of rows): such lines are the first to be evicted, so a stream far
+// larger than L2 does not push out the small tensors that the next kernels
+// read back (split-K sums, the residual stream, activations).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// tma_load_2d with an L2 cache policy (l2_evict_first()).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int c0, int c1, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+// tma_load_3d with an L2 cache policy (l2_evict_first()).
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int c0, int c1, int c2,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
         : "memory");
 }
 

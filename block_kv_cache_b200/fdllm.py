@@ -29,7 +29,7 @@ EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
            "fdl_lmhead_confidence", "fdl_threshold_unmask",
            "fdl_lmhead_confidence_noalloc", "fdl_rope_table", "fdl_rmsnorm", "fdl_embed",
            "fdl_qkv_rope_store", "fdl_linear_residual", "fdl_linear_swiglu",
-           "fdl_full_attention")
+           "fdl_full_attention", "fdl_ffn")
 
 
 class AttnDesc(ctypes.Structure):
@@ -108,6 +108,7 @@ def load() -> ctypes.CDLL:
     L.fdl_linear_residual.argtypes = [vp, i, i, i, vp, vp, vp, vp]
     L.fdl_linear_swiglu.argtypes = [vp, i, i, i, vp, vp, vp, vp]
     L.fdl_full_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp]
+    L.fdl_ffn.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -349,6 +350,20 @@ class Context:
         _check(load().fdl_linear_swiglu(self._h, x.shape[0], F, x.shape[1], _ptr(x), _ptr(w_gu),
                                         _ptr(out), _stream(stream)))
         return out
+
+    def ffn(self, x, w_gu, w_down, h, *, f=None, stream=None):
+        """h += (silu(x Wg^T) * (x Wu^T)) Wd^T; returns f, the SwiGLU output."""
+        _need(x, "x", torch.bfloat16, 2)
+        _need(w_gu, "w_gu", torch.bfloat16, 2)
+        _need(w_down, "w_down", torch.bfloat16, 2)
+        _need(h, "h", torch.float32, 2)
+        rows, hidden = x.shape
+        F = w_gu.shape[0] // 2
+        if f is None:
+            f = torch.empty((rows, F), dtype=torch.bfloat16, device=x.device)
+        _check(load().fdl_ffn(self._h, rows, hidden, F, _ptr(x), _ptr(w_gu), _ptr(w_down),
+                              _ptr(f), _ptr(h), _stream(stream)))
+        return f
 
     def full_attention(self, q, k_cache, v_cache, *, out=None, scale=0.0, stream=None):
         """Bidirectional attention of every position: q, out [b, L, Hq, d]."""

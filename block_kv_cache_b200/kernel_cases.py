@@ -119,9 +119,28 @@ def run_linear(a, ctx):
             "GBps": nbytes / us / 1e3, "TFLOPs": 2.0 * a.rows * a.n * a.k / us / 1e6}
 
 
+def run_ffn(a, ctx):
+    """The feed-forward call at (rows, hidden = k, ffn = n): gate/up [2n, k] and
+    down [k, n] weights, `layers` distinct sets cycled."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    wgu = [(torch.randn(2 * a.n, a.k, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+           for _ in range(a.layers)]
+    wd = [(torch.randn(a.k, a.n, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+          for _ in range(a.layers)]
+    x = torch.randn(a.rows, a.k, generator=g, device="cuda").to(torch.bfloat16)
+    h = torch.zeros((a.rows, a.k), dtype=torch.float32, device="cuda")
+    f = torch.empty((a.rows, a.n), dtype=torch.bfloat16, device="cuda")
+    us = _timed(a, lambda i: ctx.ffn(x, wgu[i % a.layers], wd[i % a.layers], h, f=f))
+    ctx.device_status()
+    nbytes = 3 * a.n * a.k * 2 + a.rows * a.k * 2 + 2 * a.rows * a.n * 2 + 2 * a.rows * a.k * 4
+    return {"op": "ffn", "rows": a.rows, "hidden": a.k, "ffn": a.n, "graph": a.graph, "us": us,
+            "GBps": nbytes / us / 1e3, "TFLOPs": 6.0 * a.rows * a.n * a.k / us / 1e6}
+
+
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["lmhead", "attention", "swiglu", "resid", "qkv"])
+    p.add_argument("op", choices=["lmhead", "attention", "swiglu", "resid", "qkv", "ffn"])
     p.add_argument("--n", type=int, default=24576)
     p.add_argument("--k", type=int, default=4096)
     p.add_argument("--rows", type=int, default=32)
@@ -145,6 +164,8 @@ def main():
         r = run_lmhead(a, ctx)
     elif a.op == "attention":
         r = run_attention(a, ctx)
+    elif a.op == "ffn":
+        r = run_ffn(a, ctx)
     else:
         r = run_linear(a, ctx)
     print(json.dumps(r), flush=True)

@@ -152,7 +152,7 @@ class BlockDecoder:
         self.x = torch.empty((batch, seq_len), dtype=torch.int32, device=dev)
         self.masked = torch.empty((batch, seq_len), dtype=torch.uint8, device=dev)
         self.graphs = {}
-        self.graph_timers = {}          # graph key -> [(event, event)] around SwiGLU GEMMs
+        self.graph_timers = {}          # graph key -> [(event, event)] around the FFN calls
         self._timers = None
         # rows of block k of every sequence in the flattened [b * L] token rows
         nblk = (seq_len + block - 1) // block
@@ -191,11 +191,10 @@ class BlockDecoder:
                 e0 = torch.cuda.Event(enable_timing=True, external=True)
                 e1 = torch.cuda.Event(enable_timing=True, external=True)
                 e0.record()
-            ctx.linear_swiglu(x, Lw["w_gu"], out=f)
+            ctx.ffn(x, Lw["w_gu"], Lw["wd"], h, f=f)
             if self._timers is not None:
                 e1.record()
                 self._timers.append((e0, e1))
-            ctx.linear_residual(f, Lw["wd"], h)
 
     def refresh(self, x_ids, s):
         """Full forward over all positions of x_ids [b, L] (int32, device): rewrites
@@ -276,14 +275,14 @@ class BlockDecoder:
         self.unmask(self.x, self.masked, s, tau)
         self.counts_host.copy_(self.counts, non_blocking=True)
 
-    def capture(self, kind, s, tau, time_swiglu=False):
+    def capture(self, kind, s, tau, time_ffn=False):
         """CUDA graph of one decode step (forward, unmask, counter read-back) for
         block start s; kernels read and write the decoder's own x / masked. With
-        time_swiglu, timing events bracket every layer's SwiGLU GEMM."""
+        time_ffn, timing events bracket every layer's FFN call."""
         key = (kind, s, float(tau))
         if key not in self.graphs:
             g = torch.cuda.CUDAGraph()
-            self._timers = [] if time_swiglu else None
+            self._timers = [] if time_ffn else None
             with torch.cuda.graph(g):
                 self._step_calls(kind, s, tau)
             self.graph_timers[key] = self._timers or []
@@ -295,11 +294,11 @@ class BlockDecoder:
         """Event pairs of the graph replayed by the last step()."""
         return self.graph_timers.get(self._last_key, [])
 
-    def capture_all(self, prompt_len, gen_len, tau, time_swiglu=False):
+    def capture_all(self, prompt_len, gen_len, tau, time_ffn=False):
         for blk in range(gen_len // self.B):
             s = prompt_len + blk * self.B
-            self.capture("refresh", s, tau, time_swiglu)
-            self.capture("cached", s, tau, time_swiglu)
+            self.capture("refresh", s, tau, time_ffn)
+            self.capture("cached", s, tau, time_ffn)
         torch.cuda.synchronize()
 
     def begin(self, prompt, tau):
@@ -357,7 +356,7 @@ class BlockDecoder:
             setattr(ctx, name, timed)
 
         calls = ["rmsnorm", "embed", "qkv_rope_store", "full_attention", "dualcache_attention",
-                 "linear_residual", "linear_swiglu", "lmhead_confidence", "threshold_unmask"]
+                 "linear_residual", "ffn", "lmhead_confidence", "threshold_unmask"]
         for n in calls:
             wrap(n)
         g = torch.cuda.CUDAGraph()

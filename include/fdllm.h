@@ -66,9 +66,11 @@ typedef struct fdl_ctx fdl_ctx;   /* opaque: device id, device error word, launc
 FDL_API int fdl_abi_version(void);
 
 /* Create a context on CUDA device `device`. Allocates, once, here (the only
- * allocations the library makes): the 4-byte device error word and a 32 MiB
+ * allocations the library makes): the 4-byte device error word, a 32 MiB
  * zero-filled f32 accumulator used by the few-token projections to add
- * split-K partial sums (every kernel that adds into it leaves it zeroed).
+ * split-K partial sums (every kernel that adds into it leaves it zeroed), and
+ * 256 zeroed bytes for the grid-wide barriers of fused kernels. After a call
+ * has reported FDL_ETIMEOUT these may be inconsistent: destroy the context.
  * Because of that shared accumulator, the calls made on one context must be
  * ordered on the GPU (one stream, or streams ordered by events); use one
  * context per concurrent stream. Fails with FDL_EUNSUPPORTED unless the device
@@ -309,6 +311,20 @@ FDL_API int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in
  * Errors: FDL_EINVAL, FDL_ECUDA. */
 FDL_API int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
                               const void* x, const void* w_gu, void* out, void* stream);
+
+/* Feed-forward half of a layer with its residual (SwiGLU MLP):
+ *   f  = silu(x Wg^T) * (x Wu^T)      bf16 [rows, ffn], written
+ *   h += f Wd^T                        f32 [rows, hidden], updated
+ * x bf16 [rows, hidden]; w_gu bf16 [2*ffn, hidden] interleaved as for
+ * fdl_linear_swiglu; w_down bf16 [hidden, ffn]. hidden % 64 == 0,
+ * ffn % 64 == 0. The result equals fdl_linear_swiglu followed by
+ * fdl_linear_residual. For the few rows of a cached block step (rows <= 256,
+ * hidden and ffn multiples of 128) the SwiGLU of the split-K gate/up sums is
+ * applied by the CTAs of the down projection, between a grid-wide barrier
+ * and the projection itself, instead of by a kernel of its own.
+ * Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const void* x,
+                    const void* w_gu, const void* w_down, void* f, float* h, void* stream);
 
 /* Full bidirectional attention of every position (the refresh forward after
  * a block completes): out[b, i, h, :] = softmax over all j of q_i . k_j.

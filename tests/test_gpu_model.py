@@ -99,6 +99,34 @@ def test_linear_swiglu(ctx, M, F, K):
     assert rel(out.float().cpu().numpy(), ref) <= BF16_TOL
 
 
+@pytest.mark.parametrize("M,D,F", [(32, 4096, 12288), (32, 512, 1024), (7, 256, 640),
+                                   (64, 1024, 4096), (300, 256, 192), (1, 128, 128)])
+def test_ffn_block(ctx, M, D, F):
+    """h += SwiGLU(x) Wd^T in one call; for few rows the SwiGLU of the split-K
+    sums runs in the down projection's kernel behind a grid barrier. Called
+    twice so that the context's scratch (zeroed sums, barrier words) is
+    checked to be reusable."""
+    g = synth.rng(M * 7 + F)
+    x = bf_vals(g.standard_normal((M, D)))
+    wg = bf_vals(g.standard_normal((F, D)) * 0.05)
+    wu = bf_vals(g.standard_normal((F, D)) * 0.05)
+    wd = bf_vals(g.standard_normal((D, F)) * 0.03)
+    wgu = np.empty((2 * F, D), np.float32)
+    wgu[0::2], wgu[1::2] = wg, wu
+    h0 = g.standard_normal((M, D)).astype(np.float32)
+    x64 = x.astype(np.float64)
+    f_ref = O.silu(x64 @ wg.T) * (x64 @ wu.T)
+    xg, wgug, wdg = bf(x), bf(wgu), bf(wd)
+    for rep in range(2):
+        h = f32(h0)
+        f = ctx.ffn(xg, wgug, wdg, h)
+        assert rel(f.float().cpu().numpy(), f_ref) <= BF16_TOL, rep
+        # the down projection consumes the bf16 f the call wrote
+        ref = h0.astype(np.float64) + f.float().cpu().numpy().astype(np.float64) @ wd.astype(np.float64).T
+        assert rel(h.cpu().numpy(), ref) <= 1e-4, rep
+    ctx.device_status()
+
+
 @pytest.mark.parametrize("Hq,Hkv,bias,rows_per_seq,pos0,batch,L", [
     (4, 4, False, 32, 64, 2, 128),     # block slot of 2 sequences
     (4, 2, True, 128, 0, 2, 128),      # refresh: every position, GQA, Qwen-style bias
