@@ -357,9 +357,11 @@ int fdl_embed(fdl_ctx* ctx, int rows, int hidden, const int32_t* ids, const int3
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "embed launch");
 }
 
-int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
-                       const float* bias, const float* rope, void* q_out, void* k_cache,
-                       void* v_cache, void* stream) {
+}  // extern "C"
+
+namespace {
+int check_qkv(const fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+              const float* rope, const void* q_out, const void* k_cache, const void* v_cache) {
     if (!ctx) return fail(FDL_EINVAL, "qkv: ctx is NULL");
     if (!d) return fail(FDL_EINVAL, "qkv: desc is NULL");
     if (d->head_dim != 128) return fail(FDL_EUNSUPPORTED, "qkv: head_dim must be 128");
@@ -378,6 +380,17 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
     if (!aligned16(x) || !aligned16(w) || !aligned16(q_out) || !aligned16(k_cache) ||
         !aligned16(v_cache) || !aligned16(rope))
         return fail(FDL_EINVAL, "qkv: buffers must be 16-byte aligned");
+    return FDL_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+                       const float* bias, const float* rope, void* q_out, void* k_cache,
+                       void* v_cache, void* stream) {
+    const int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
+    if (rc) return rc;
     DeviceGuard g(ctx->device);
     fdl::GemmShape gs{d->rows, (d->n_q_heads + 2 * d->n_kv_heads) * 128, d->hidden};
     fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
@@ -388,6 +401,46 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
                                  ctx->d_err, (cudaStream_t)stream)
         : fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err, (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv launch");
+}
+
+int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+                      const float* bias, const float* rope, void* q_out, void* k_cache,
+                      void* v_cache, void* out, void* stream) {
+    int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
+    if (rc) return rc;
+    if (d->rows != d->batch * d->rows_per_seq || d->rows_per_seq > 128)
+        return fail(FDL_EINVAL, "qkv_attention: rows must be batch * rows_per_seq, "
+                    "rows_per_seq <= 128 (one block per sequence)");
+    if (d->n_q_heads % d->n_kv_heads)
+        return fail(FDL_EINVAL, "qkv_attention: n_q_heads must be a multiple of n_kv_heads");
+    if (!out || !aligned16(out)) return fail(FDL_EINVAL, "qkv_attention: out NULL or unaligned");
+    DeviceGuard g(ctx->device);
+    cudaStream_t st = (cudaStream_t)stream;
+    const fdl::GemmShape gs{d->rows, (d->n_q_heads + 2 * d->n_kv_heads) * 128, d->hidden};
+    const fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
+                        (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
+                        d->rows_per_seq, d->pos0};
+    fdl::AttnShape as{d->batch, d->n_q_heads, d->n_kv_heads, 128, d->seq_len, d->pos0,
+                      d->rows_per_seq, 1.0f / sqrtf(128.f), 1};
+    cudaError_t e;
+    const int splits = fdl::skinny_ok(gs) ? fdl::skinny_qkv_splits(gs, ctx->acc_bytes,
+                                                                   ctx->sm_count) : 1;
+    if (splits > 1 && fdl::qkv_attention_fusable(as, ctx->sm_count)) {
+        e = fdl::launch_skinny_qkv_sums(gs, x, w, ctx->d_acc, splits, ctx->sm_count, ctx->d_err,
+                                        st);
+        if (e == cudaSuccess)
+            e = fdl::launch_qkv_attention_bf16(as, ctx->d_acc, d->rows, p, ctx->d_sync + 2, out,
+                                               ctx->sm_count, ctx->d_err, st);
+    } else {
+        e = fdl::skinny_ok(gs)
+            ? fdl::launch_skinny_qkv(gs, x, w, p, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
+                                     ctx->d_err, st)
+            : fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err, st);
+        if (e == cudaSuccess)
+            e = fdl::launch_attention_bf16(as, q_out, k_cache, v_cache, out, nullptr, nullptr,
+                                           ctx->sm_count, ctx->d_err, st);
+    }
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv_attention launch");
 }
 
 int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_features,

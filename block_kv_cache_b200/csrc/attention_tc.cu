@@ -31,6 +31,7 @@
 // Roofline: HBM. Algorithmic bytes per call = K and V once (2*b*Hkv*L*d*2)
 // + q and out (2*b*B*Hq*d*2).
 #include "common.cuh"
+#include "gemm.h"
 #include "launch.h"
 #include "sm100.cuh"
 
@@ -144,14 +145,85 @@ struct AttnArgs {
     bf16* out;
     float* lse;         // optional
     int B, Hq, Hkv, L, hc, n_chunks, rows, tiles, tps, n_splits, q_per_kv;
+    int blk0, blk1;     // block slot [blk0, blk1) of every sequence
     float scale_log2;
     int* err;
 };
 
-template <int D, int MT>
+// ---- prologues: work every CTA does after the preceding kernel -----------------
+struct AttNoPro {
+    static constexpr bool kActive = false;
+    unsigned* bar = nullptr;
+    __device__ void work(int, int) const {}
+};
+
+// The epilogue of a split-K block-slot projection (bias, RoPE, q and the K/V
+// block slot written; the f32 sums zeroed again), shared by the CTAs of the
+// attention kernel that reads the result, followed by a grid barrier: no
+// kernel of its own. Item = one (token, head, dimension pair d / d + 64).
+struct ProQKV {
+    static constexpr bool kActive = true;
+    unsigned* bar;           // grid barrier words
+    float* acc;              // [M, N] sums, N = (Hq + 2 Hkv) * 128
+    int M;
+    EpiQKV p;
+    __device__ void work(int part, int nparts) const {
+        constexpr int D = 128, U = 4;
+        const int heads = p.n_q_heads + 2 * p.n_kv_heads, N = heads * D;
+        const int n = M * heads * 64, stride = nparts * blockDim.x;
+        for (int e0 = part * blockDim.x + threadIdx.x; e0 < n; e0 += U * stride) {
+            float lo[U], hi[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {           // every load first, then the math
+                const int e = e0 + u * stride;
+                if (e < n) {
+                    const int t = e / (heads * 64), r = e - t * heads * 64;
+                    const float* row = acc + (size_t)t * N + (r >> 6) * D + (r & 63);
+                    lo[u] = __ldcg(row);
+                    hi[u] = __ldcg(row + 64);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int e = e0 + u * stride;
+                if (e >= n) continue;
+                const int t = e / (heads * 64), r = e - t * heads * 64;
+                const int h = r >> 6, d = r & 63;
+                float* row = acc + (size_t)t * N + h * D + d;
+                __stcg(row, 0.f);
+                __stcg(row + 64, 0.f);
+                float y0 = lo[u], y1 = hi[u];
+                if (p.bias) {
+                    y0 += p.bias[h * D + d];
+                    y1 += p.bias[h * D + d + 64];
+                }
+                const int seq = t / p.rows_per_seq, pos = p.pos0 + t % p.rows_per_seq;
+                if (h < p.n_q_heads + p.n_kv_heads) {
+                    const float2 cs = p.rope[(size_t)pos * (D / 2) + d];
+                    const float r0 = y0 * cs.x - y1 * cs.y, r1 = y1 * cs.x + y0 * cs.y;
+                    y0 = r0;
+                    y1 = r1;
+                }
+                bf16* dst;
+                if (h < p.n_q_heads)
+                    dst = p.q + ((size_t)t * p.n_q_heads + h) * D;
+                else if (h < p.n_q_heads + p.n_kv_heads)
+                    dst = p.k_cache +
+                          (((size_t)seq * p.n_kv_heads + h - p.n_q_heads) * p.seq_len + pos) * D;
+                else
+                    dst = p.v_cache + (((size_t)seq * p.n_kv_heads + h - p.n_q_heads - p.n_kv_heads) *
+                                           p.seq_len + pos) * D;
+                dst[d] = __float2bfloat16_rn(y0);
+                dst[d + 64] = __float2bfloat16_rn(y1);
+            }
+        }
+    }
+};
+
+template <int D, int MT, class Pro>
 __global__ void __launch_bounds__(Att4<D, MT>::THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+               const __grid_constant__ CUtensorMap tmV, const AttnArgs a, const Pro pro) {
     using namespace sm100;
     using S = Att4<D, MT>;
     constexpr int KT = ATT_KT, STAGES = S::STAGES;
@@ -205,48 +277,83 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    pdl_wait();
-    pdl_trigger();
     const uint32_t tmem = *tmem_slot;
-    bool ok = true;
+    const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
+    const uint64_t kv_policy = l2_evict_first();
+    auto load_kv = [&](int t, int st) {
+        // one copy per tile and operand: all D columns as DC sub-tiles
+        mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
+        if (a.q_per_kv == 1)   // one query block: every K/V byte is read once
+            tma_load_3d_hint(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
+                             krow0 + t * KT, 0, kv_policy);
+        else
+            tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0, krow0 + t * KT, 0);
+        mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
+        if (a.q_per_kv == 1)
+            tma_load_3d_hint(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
+                             krow0 + t * KT, 0, kv_policy);
+        else
+            tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0, krow0 + t * KT, 0);
+    };
+    // With a prologue, the preceding kernel is this call's own projection,
+    // which writes no cache row: whole tiles outside the block slot can be
+    // requested before it ends (ring stages are fresh, so no empty wait).
+    uint32_t early = 0;
+    if constexpr (Pro::kActive) {
+        if (warp == S::TMA_WARP && lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            for (int t = 0; t < nt && t < STAGES; ++t) {
+                const int k0 = k_begin + t * KT, k1 = k0 + KT;
+                if (k1 <= a.L && (k1 <= a.blk0 || k0 >= a.blk1)) {
+                    load_kv(t, t);
+                    early |= 1u << t;
+                }
+            }
+        }
+    }
+    pdl_wait();
+    if constexpr (Pro::kActive) {
+        pro.work(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z),
+                 gridDim.x * gridDim.y * gridDim.z);
+        fence_proxy_async_global();                 // the TMA below reads what was written
+        grid_barrier(pro.bar, abort_flag, a.err);
+    }
+    pdl_trigger();
+    bool ok = *abort_flag == 0;
 
     if (warp == S::TMA_WARP) {
         // ---------------------------------------------------------------- TMA
         if (lane == 0) {
             prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
+            if constexpr (Pro::kActive) fence_proxy_async_global();
             const int head0 = g * grp + chunk * a.hc;
-            mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
-            for (int dc = 0; dc < S::DC; ++dc)
-                tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
-                            bb * a.B);
-            const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
-            const uint64_t kv_policy = l2_evict_first();
+            if (ok) {
+                mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
+                for (int dc = 0; dc < S::DC; ++dc)
+                    tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
+                                bb * a.B);
+            }
             int t = 0;
             for (; ok && t < nt; ++t) {
                 const int st = t % STAGES;
+                if (t < STAGES && ((early >> t) & 1u)) continue;
                 if (!(ok = mbar_wait(kv_empty(st), ((t / STAGES) & 1) ^ 1, abort_flag, a.err)))
                     break;
-                // one copy per tile and operand: all D columns as DC sub-tiles
-                mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
-                if (a.q_per_kv == 1)   // one query block: every K/V byte is read once
-                    tma_load_3d_hint(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
-                                     krow0 + t * KT, 0, kv_policy);
-                else
-                    tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
-                                krow0 + t * KT, 0);
-                mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
-                if (a.q_per_kv == 1)
-                    tma_load_3d_hint(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
-                                     krow0 + t * KT, 0, kv_policy);
-                else
-                    tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
-                                krow0 + t * KT, 0);
+                load_kv(t, st);
             }
             // tail: every stage handed out has been released again
             for (int u = t; ok && u < t + STAGES; ++u)
                 ok = mbar_wait(kv_empty(u % STAGES), ((u / STAGES) & 1) ^ 1, abort_flag, a.err);
+            if (!ok && early) {
+                // gave up: the tiles requested early must land before the CTA exits
+                volatile int no_abort = 0;
+                for (int u = 0; u < STAGES; ++u)
+                    if ((early >> u) & 1u) {
+                        mbar_wait(k_full(u), 0, &no_abort, a.err);
+                        mbar_wait(v_full(u), 0, &no_abort, a.err);
+                    }
+            }
         }
     } else if (warp == S::MMA_WARP) {
         // ---------------------------------------------------------------- MMA
@@ -485,17 +592,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
 }
 
-template <int D, int MT>
+template <int D, int MT, class Pro>
 cudaError_t run_tc(const AttnPlan& p, const CUtensorMap& tq, const CUtensorMap& tk,
                    const CUtensorMap& tv, const AttnArgs& a, int batch, int hkv,
-                   cudaStream_t st) {
+                   cudaStream_t st, const Pro& pro) {
     using S = Att4<D, MT>;
-    auto kfn = attn_tc_kernel<D, MT>;
+    auto kfn = attn_tc_kernel<D, MT, Pro>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S::TOTAL);
     if (e != cudaSuccess) return e;
     return launch_pdl(kfn, dim3(p.n_splits, hkv * p.n_chunks, batch), dim3(S::THREADS), S::TOTAL,
-                      st, p.n_splits, tq, tk, tv, a);
+                      st, p.n_splits, tq, tk, tv, a, pro);
 }
 
 }  // namespace
@@ -504,10 +611,12 @@ size_t attn_tc_workspace_bytes(const AttnShape&, int) {
     return 16;   // the splits merge on chip; no scratch is needed
 }
 
-cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
-                                  const void* v, void* out, float* lse, void* ws, int sm_count,
-                                  int* err, cudaStream_t st) {
-    (void)ws;
+namespace {
+
+template <class Pro>
+cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const void* v,
+                        void* out, float* lse, int sm_count, int* err, cudaStream_t st,
+                        const Pro& pro) {
     const AttnPlan p = attn_tc_plan(s, sm_count);
     const int D = s.head_dim;
     CUtensorMap tq, tk, tv;
@@ -536,13 +645,75 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
     a.tps = p.tps;
     a.n_splits = p.n_splits;
     a.q_per_kv = s.q_per_kv;
+    a.blk0 = s.block_start;
+    a.blk1 = s.block_start + s.block_len;
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
+    const int hb = s.batch, hk = s.n_kv_heads;
     if (D == 128)
-        return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st)
-                         : run_tc<128, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
-    return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st)
-                     : run_tc<64, 1>(p, tq, tk, tv, a, s.batch, s.n_kv_heads, st);
+        return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
+                         : run_tc<128, 1>(p, tq, tk, tv, a, hb, hk, st, pro);
+    return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
+                     : run_tc<64, 1>(p, tq, tk, tv, a, hb, hk, st, pro);
+}
+
+// Largest number of clusters of the given size that fit on the device at once
+// (queried once per kernel and size).
+template <int D, int MT>
+int max_active_clusters(int size, int sm_count) {
+    static int cache[ATT_MAX_SPLITS + 1] = {0};
+    if (size < 1 || size > ATT_MAX_SPLITS) return 0;
+    if (cache[size] == 0) {
+        using S = Att4<D, MT>;
+        auto kfn = attn_tc_kernel<D, MT, ProQKV>;
+        int n = 0;
+        if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)S::TOTAL) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(size * (sm_count / size));
+            cfg.blockDim = dim3(S::THREADS);
+            cfg.dynamicSmemBytes = S::TOTAL;
+            cudaLaunchAttribute at;
+            at.id = cudaLaunchAttributeClusterDimension;
+            at.val.clusterDim.x = size;
+            at.val.clusterDim.y = 1;
+            at.val.clusterDim.z = 1;
+            cfg.attrs = &at;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();
+        cache[size] = n > 0 ? n : -1;
+    }
+    return cache[size] > 0 ? cache[size] : 0;
+}
+
+}  // namespace
+
+cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void* k,
+                                  const void* v, void* out, float* lse, void* ws, int sm_count,
+                                  int* err, cudaStream_t st) {
+    (void)ws;
+    return launch_attn(s, q, k, v, out, lse, sm_count, err, st, AttNoPro{});
+}
+
+bool qkv_attention_fusable(const AttnShape& s, int sm_count) {
+    if (s.head_dim != 128 || !s.bf16 || s.q_per_kv != 1) return false;
+    const AttnPlan p = attn_tc_plan(s, sm_count);
+    const int ctas = p.n_splits * s.n_kv_heads * p.n_chunks * s.batch;
+    if (ctas > sm_count) return false;               // one CTA per SM: all resident
+    if (p.n_splits == 1) return true;
+    const int clusters = ctas / p.n_splits;
+    const int fit = p.mt == 2 ? max_active_clusters<128, 2>(p.n_splits, sm_count)
+                              : max_active_clusters<128, 1>(p.n_splits, sm_count);
+    return clusters <= fit;
+}
+
+cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, int rows, const EpiQKV& pq,
+                                      unsigned* bar, void* out, int sm_count, int* err,
+                                      cudaStream_t st) {
+    return launch_attn(s, pq.q, pq.k_cache, pq.v_cache, out, nullptr, sm_count, err, st,
+                       ProQKV{bar, acc, rows, pq});
 }
 
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,

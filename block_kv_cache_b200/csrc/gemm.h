@@ -51,6 +51,13 @@ cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, 
                               float* acc, size_t acc_bytes, int sm_count, int* err,
                               cudaStream_t st);
 
+// K splits the few-row q/k/v projection uses with an accumulator of acc_bytes
+// (1: none), and the projection alone leaving its split-K sums in acc (the
+// epilogue is then up to the caller: launch_qkv_attention_bf16).
+int skinny_qkv_splits(const GemmShape& g, size_t acc_bytes, int sm_count);
+cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void* w, float* acc,
+                                   int splits, int sm_count, int* err, cudaStream_t st);
+
 // Feed-forward block for M <= 256 rows: h[M, ld_h] += down(SwiGLU(x W_gu^T)),
 // w_gu [2F, K] interleaved (row 2f gate, 2f + 1 up), w_down [ld_h, F], f [M, F]
 // bf16 scratch (the down projection's operand). acc/acc_bytes as above; bar:

@@ -538,6 +538,15 @@ cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, 
                       p);
 }
 
+int skinny_qkv_splits(const GemmShape& g, size_t acc_bytes, int sm_count) {
+    return (size_t)g.M * g.N * 4 <= acc_bytes ? choose_splits(g, sm_count, 8) : 1;
+}
+
+cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void* w, float* acc,
+                                   int splits, int sm_count, int* err, cudaStream_t st) {
+    return dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st);
+}
+
 // h += down(SwiGLU(x W_gu^T)) for few rows: the gate/up projection with split-K
 // partial sums in acc, then the down projection whose CTAs first turn the
 // sums into f = bf16(silu(g) * u) (grid barrier, no kernel in between).

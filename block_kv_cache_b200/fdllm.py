@@ -29,7 +29,7 @@ EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
            "fdl_lmhead_confidence", "fdl_threshold_unmask",
            "fdl_lmhead_confidence_noalloc", "fdl_rope_table", "fdl_rmsnorm", "fdl_embed",
            "fdl_qkv_rope_store", "fdl_linear_residual", "fdl_linear_swiglu",
-           "fdl_full_attention", "fdl_ffn")
+           "fdl_full_attention", "fdl_ffn", "fdl_qkv_attention")
 
 
 class AttnDesc(ctypes.Structure):
@@ -109,6 +109,8 @@ def load() -> ctypes.CDLL:
     L.fdl_linear_swiglu.argtypes = [vp, i, i, i, vp, vp, vp, vp]
     L.fdl_full_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp]
     L.fdl_ffn.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
+    L.fdl_qkv_attention.argtypes = [vp, ctypes.POINTER(QKVDesc), vp, vp, vp, vp, vp, vp, vp, vp,
+                                    vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -330,6 +332,20 @@ class Context:
                                          _ptr(bias), _ptr(rope), _ptr(q_out), _ptr(k_cache),
                                          _ptr(v_cache), _stream(stream)))
         return q_out
+
+    def qkv_attention(self, x, w, rope, q_out, k_cache, v_cache, out, *, n_q_heads,
+                      rows_per_seq, pos0, bias=None, stream=None):
+        """qkv_rope_store of the block rows, then DualCache attention of the block
+        [pos0, pos0 + rows_per_seq) of every sequence over the caches -> out."""
+        _need(x, "x", torch.bfloat16, 2)
+        _need(w, "w", torch.bfloat16, 2)
+        b, hkv, L, d = k_cache.shape
+        d_ = QKVDesc(x.shape[0], x.shape[1], int(n_q_heads), hkv, d, b, L, int(rows_per_seq),
+                     int(pos0), rope.shape[0])
+        _check(load().fdl_qkv_attention(self._h, ctypes.byref(d_), _ptr(x), _ptr(w), _ptr(bias),
+                                        _ptr(rope), _ptr(q_out), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(out), _stream(stream)))
+        return out
 
     def linear_residual(self, x, w, h, *, stream=None):
         """h += x w^T (h f32)."""

@@ -163,28 +163,25 @@ class BlockDecoder:
         lmd = fdllm.LMHeadDesc(rb, D, sh.vocab, fdllm.FDL_BF16)
         self.ws_lm = torch.empty(max(ctx.lmhead_workspace_bytes(lmd), 16), dtype=torch.uint8,
                                  device=dev)
-        ad = fdllm.AttnDesc(batch, sh.n_q_heads, sh.n_kv_heads, d, seq_len, 0, block,
-                            fdllm.FDL_BF16, 0.0)
-        self.ws_att = torch.empty(max(ctx.attention_workspace_bytes(ad), 16), dtype=torch.uint8,
-                                  device=dev)
 
     # ------------------------------------------------------------------ layers
     def _layers(self, h, x, q, o, f, rows, rows_per_seq, pos0, full):
         ctx, sh = self.ctx, self.sh
         for li, Lw in enumerate(self.w.layers):
             ctx.rmsnorm(h, Lw["attn_norm"], sh.rms_eps, out=x)
-            ctx.qkv_rope_store(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
-                               n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
-                               bias=Lw["bias"])
             if full:
+                ctx.qkv_rope_store(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
+                                   n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
+                                   bias=Lw["bias"])
                 ctx.full_attention(q.view(self.b, self.L, sh.n_q_heads, sh.head_dim),
                                    self.kc[li], self.vc[li],
                                    out=o.view(self.b, self.L, sh.n_q_heads, sh.head_dim))
             else:
-                ctx.dualcache_attention(q.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
-                                        self.kc[li], self.vc[li], pos0,
-                                        out=o.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
-                                        ws=self.ws_att)
+                # block-slot projection + DualCache attention of the block rows
+                ctx.qkv_attention(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
+                                  o.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
+                                  n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
+                                  bias=Lw["bias"])
             ctx.linear_residual(o.view(rows, -1), Lw["wo"], h)
             ctx.rmsnorm(h, Lw["ffn_norm"], sh.rms_eps, out=x)
             if self._timers is not None:
@@ -355,7 +352,7 @@ class BlockDecoder:
                 return r
             setattr(ctx, name, timed)
 
-        calls = ["rmsnorm", "embed", "qkv_rope_store", "full_attention", "dualcache_attention",
+        calls = ["rmsnorm", "embed", "qkv_rope_store", "full_attention", "qkv_attention",
                  "linear_residual", "ffn", "lmhead_confidence", "threshold_unmask"]
         for n in calls:
             wrap(n)

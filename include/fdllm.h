@@ -300,6 +300,23 @@ FDL_API int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* desc, const voi
                                const void* w, const float* bias, const float* rope,
                                void* q_out, void* k_cache, void* v_cache, void* stream);
 
+/* The block-slot projection of a cached DualCache step followed by the block's
+ * attention: the result equals fdl_qkv_rope_store(desc, ...) and then
+ * fdl_dualcache_attention over the caches with block_start = desc->pos0,
+ * block_len = desc->rows_per_seq, scale 1/sqrt(128) and no LSE. Requires
+ * rows == batch * rows_per_seq (the block rows of every sequence) and
+ * rows_per_seq <= 128. out [batch, rows_per_seq, n_q_heads, 128] bf16 is
+ * written; q_out, k_cache, v_cache as for fdl_qkv_rope_store. When the
+ * attention grid fits on the device at once, the projection's epilogue
+ * (bias, RoPE, q and block-slot store) is done by the CTAs of the attention
+ * kernel between a grid-wide barrier and the attention, instead of by a
+ * kernel of its own. Errors: as fdl_qkv_rope_store, plus FDL_EINVAL for the
+ * row layout. */
+FDL_API int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* desc, const void* x,
+                              const void* w, const float* bias, const float* rope,
+                              void* q_out, void* k_cache, void* v_cache, void* out,
+                              void* stream);
+
 /* h[rows, out_features] += x w^T  (f32 residual stream; x bf16 [rows, in],
  * w bf16 [out, in]). in % 64 == 0, out % 64 == 0. Errors: FDL_EINVAL, FDL_ECUDA. */
 FDL_API int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_features,

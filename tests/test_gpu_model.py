@@ -170,6 +170,59 @@ def test_qkv_rope_store(ctx, Hq, Hkv, bias, rows_per_seq, pos0, batch, L):
         assert np.array_equal(vg[sq][:, keep], v0[sq][:, keep])
 
 
+@pytest.mark.parametrize("batch,Hq,Hkv,bias,B,pos0,L,D", [
+    (1, 32, 32, False, 32, 1024, 2048, 4096),   # LLaDA-8B layer: fused path
+    (1, 8, 8, False, 32, 96, 256, 1024),        # fused, several splits per head
+    (2, 28, 4, True, 32, 512, 1024, 3584),      # GQA 7:1 with bias (Dream / Qwen2.5 shape)
+    (2, 4, 2, True, 32, 64, 160, 256),          # no K split: separate calls
+])
+def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D):
+    """Block-slot projection + DualCache attention in one call equals the
+    oracle's projection, RoPE, cache store and attention over the cache."""
+    g = synth.rng(Hq * 3 + L + D)
+    d = 128
+    M = batch * B
+    N = (Hq + 2 * Hkv) * d
+    x = bf_vals(g.standard_normal((M, D)))
+    w = bf_vals(g.standard_normal((N, D)) * (1.0 / np.sqrt(D)))
+    bvec = (g.standard_normal(N) * 0.1).astype(np.float32) if bias else None
+    k0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
+    v0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
+    from block_kv_cache_b200 import fdllm
+    rope = torch.from_numpy(fdllm.rope_table(10000.0, L, d)).cuda()
+    kc, vc = bf(k0), bf(v0)
+    q = torch.empty((M, Hq, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((batch, B, Hq, d), dtype=torch.bfloat16, device="cuda")
+    xg, wg = bf(x), bf(w)
+    bg = None if bvec is None else f32(bvec)
+    for rep in range(2):                       # scratch and barrier words are reusable
+        ctx.qkv_attention(xg, wg, rope, q, kc, vc, out, n_q_heads=Hq, rows_per_seq=B,
+                          pos0=pos0, bias=bg)
+        ctx.device_status()
+        y = x.astype(np.float64) @ w.astype(np.float64).T
+        if bvec is not None:
+            y = y + bvec
+        pos = pos0 + np.arange(M) % B
+        qr = O.apply_rope(y[:, :Hq * d].reshape(M, Hq, d), pos)
+        kr = O.apply_rope(y[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d), pos)
+        vr = y[:, (Hq + Hkv) * d:].reshape(M, Hkv, d)
+        assert rel(q.float().cpu().numpy(), qr) <= BF16_TOL
+        kg, vg = kc.float().cpu().numpy(), vc.float().cpu().numpy()
+        og = out.float().cpu().numpy()
+        for sq in range(batch):
+            rows = slice(sq * B, (sq + 1) * B)
+            kref = k0[sq].astype(np.float64).copy()
+            vref = v0[sq].astype(np.float64).copy()
+            kref[:, pos0:pos0 + B] = kr[rows].transpose(1, 0, 2)
+            vref[:, pos0:pos0 + B] = vr[rows].transpose(1, 0, 2)
+            assert rel(kg[sq], kref) <= BF16_TOL and rel(vg[sq], vref) <= BF16_TOL
+            keep = np.ones(L, bool)
+            keep[pos0:pos0 + B] = False
+            assert np.array_equal(kg[sq][:, keep], k0[sq][:, keep])
+            o_ref, _ = O.attention(qr[rows], kref, vref)
+            assert rel(og[sq], o_ref) <= BF16_TOL, (rep, sq)
+
+
 @pytest.mark.parametrize("b,Hq,Hkv,L", [(1, 32, 32, 256), (2, 28, 4, 128), (2, 8, 2, 96)])
 def test_full_attention(ctx, b, Hq, Hkv, L):
     g = synth.rng(b * Hq + L)
