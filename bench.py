@@ -129,9 +129,10 @@ def read_peaks():
 
 
 # kernels per step: embed, final norm, LM head (2), unmask, and per layer
-#   cached:  norm, QKV GEMM, QKV finish, attention, O GEMM, norm, gate/up GEMM, down GEMM
+#   cached:  QKV GEMM (norm inside), attention (QKV epilogue inside), O GEMM,
+#            gate/up GEMM (norm inside), down GEMM (SwiGLU inside)
 #   refresh: norm, QKV GEMM, full attention, O GEMM, norm, gate/up GEMM, down GEMM
-LAUNCHES = {"cached": 32 * 8 + 5, "refresh": 32 * 7 + 5}
+LAUNCHES = {"cached": 32 * 5 + 5, "refresh": 32 * 7 + 5}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -225,9 +226,10 @@ def run_gpu(args):
         peak = peaks.get("hbm_gbs") or 6650.0
         M = c["batch"] * c["block"]
         D, F = c["hidden"], c["ffn"]
-        # algorithmic bytes of one FFN call: both weights once, x in, f out and
-        # back in, the f32 residual rows read and written
-        ffn_bytes = 3 * F * D * 2 + M * D * 2 + 2 * M * F * 2 + 2 * M * D * 4
+        # algorithmic bytes of one FFN call: both weights once, the f32 residual
+        # rows read for the norm and read + written by the down projection, x and
+        # f each written and read back
+        ffn_bytes = 3 * F * D * 2 + 2 * M * D * 2 + 2 * M * F * 2 + 3 * M * D * 4
         sw_avg_ms = sw_ms / max(sw_n, 1)
         ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
         out = {
@@ -247,8 +249,9 @@ def run_gpu(args):
                        "l2": "no flush: 16 GB of weights (> 126 MB L2) are streamed every step"},
             "gpu_launches": sum(LAUNCHES[k] * n for k, n in kinds.items()),
             "roofline": {"kernel": "ffn call of a cached step (M=32): gate/up GEMM 24576x4096 "
-                                   "with split-K sums, then the down GEMM 4096x12288 whose CTAs "
-                                   "apply the SwiGLU first; 40% of the step's weight bytes",
+                                   "whose CTAs apply the RMSNorm first, with split-K sums, then "
+                                   "the down GEMM 4096x12288 whose CTAs apply the SwiGLU first; "
+                                   "60% of the step's weight bytes",
                          "bytes_per_call": ffn_bytes,
                          "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": (ach / peak) if ach else None, "traffic": None,

@@ -403,11 +403,14 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv launch");
 }
 
-int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
-                      const float* bias, const float* rope, void* q_out, void* k_cache,
-                      void* v_cache, void* out, void* stream) {
+int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const float* norm_w,
+                      float eps, void* x, const void* w, const float* bias, const float* rope,
+                      void* q_out, void* k_cache, void* v_cache, void* out, void* stream) {
     int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
     if (rc) return rc;
+    if (norm_w && (!h || !aligned16(h) || !aligned16(norm_w) || !(eps > 0.f)))
+        return fail(FDL_EINVAL, "qkv_attention: with norm_w, h must be a 16-byte aligned f32 "
+                    "buffer and eps > 0");
     if (d->rows != d->batch * d->rows_per_seq || d->rows_per_seq > 128)
         return fail(FDL_EINVAL, "qkv_attention: rows must be batch * rows_per_seq, "
                     "rows_per_seq <= 128 (one block per sequence)");
@@ -422,20 +425,25 @@ int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const 
                         d->rows_per_seq, d->pos0};
     fdl::AttnShape as{d->batch, d->n_q_heads, d->n_kv_heads, 128, d->seq_len, d->pos0,
                       d->rows_per_seq, 1.0f / sqrtf(128.f), 1};
+    const fdl::NormIn ni{h, norm_w, eps};
     cudaError_t e;
     const int splits = fdl::skinny_ok(gs) ? fdl::skinny_qkv_splits(gs, ctx->acc_bytes,
                                                                    ctx->sm_count) : 1;
     if (splits > 1 && fdl::qkv_attention_fusable(as, ctx->sm_count)) {
-        e = fdl::launch_skinny_qkv_sums(gs, x, w, ctx->d_acc, splits, ctx->sm_count, ctx->d_err,
-                                        st);
+        e = fdl::launch_skinny_qkv_sums(gs, x, w, ctx->d_acc, splits, norm_w ? &ni : nullptr,
+                                        ctx->d_sync + 6, ctx->sm_count, ctx->d_err, st);
         if (e == cudaSuccess)
-            e = fdl::launch_qkv_attention_bf16(as, ctx->d_acc, d->rows, p, ctx->d_sync + 2, out,
+            e = fdl::launch_qkv_attention_bf16(as, ctx->d_acc, d->rows, p, ctx->d_sync + 4, out,
                                                ctx->sm_count, ctx->d_err, st);
     } else {
-        e = fdl::skinny_ok(gs)
-            ? fdl::launch_skinny_qkv(gs, x, w, p, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
-                                     ctx->d_err, st)
-            : fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err, st);
+        e = norm_w ? fdl::launch_rmsnorm(d->rows, d->hidden, h, nullptr, norm_w, eps,
+                                         (fdl::bf16*)x, st)
+                   : cudaSuccess;
+        if (e == cudaSuccess)
+            e = fdl::skinny_ok(gs)
+                ? fdl::launch_skinny_qkv(gs, x, w, p, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
+                                         ctx->d_err, st)
+                : fdl::launch_gemm_qkv(gs, x, w, p, ctx->sm_count, ctx->d_err, st);
         if (e == cudaSuccess)
             e = fdl::launch_attention_bf16(as, q_out, k_cache, v_cache, out, nullptr, nullptr,
                                            ctx->sm_count, ctx->d_err, st);
@@ -482,23 +490,29 @@ int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "linear_swiglu launch");
 }
 
-int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const void* x, const void* w_gu,
-            const void* w_down, void* f, float* h, void* stream) {
+int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const float* norm_w, float eps, void* x,
+            const void* w_gu, const void* w_down, void* f, float* h, void* stream) {
     if (!ctx) return fail(FDL_EINVAL, "ffn: ctx is NULL");
     if (rows < 1 || hidden < 64 || hidden % 64 || ffn < 64 || ffn % 64)
         return fail(FDL_EINVAL, "ffn: rows >= 1, hidden % 64 == 0, ffn % 64 == 0");
     if (!x || !w_gu || !w_down || !f || !h) return fail(FDL_EINVAL, "ffn: NULL buffer");
     if (!aligned16(x) || !aligned16(w_gu) || !aligned16(w_down) || !aligned16(f) ||
-        !aligned16(h))
+        !aligned16(h) || (norm_w && !aligned16(norm_w)))
         return fail(FDL_EINVAL, "ffn: buffers must be 16-byte aligned");
+    if (norm_w && !(eps > 0.f)) return fail(FDL_EINVAL, "ffn: eps must be > 0");
     DeviceGuard g(ctx->device);
     cudaStream_t st = (cudaStream_t)stream;
     const fdl::GemmShape gu{rows, 2 * ffn, hidden}, dn{rows, hidden, ffn};
+    const fdl::NormIn ni{h, norm_w, eps};
     cudaError_t e;
     if (fdl::skinny_ok(gu) && fdl::skinny_ok(dn)) {
         e = fdl::launch_skinny_ffn(gu, x, w_gu, w_down, (fdl::bf16*)f, h, hidden, ctx->d_acc,
-                                   ctx->acc_bytes, ctx->d_sync, ctx->sm_count, ctx->d_err, st);
+                                   ctx->acc_bytes, ctx->d_sync, norm_w ? &ni : nullptr,
+                                   ctx->sm_count, ctx->d_err, st);
     } else {
+        e = norm_w ? fdl::launch_rmsnorm(rows, hidden, h, nullptr, norm_w, eps, (fdl::bf16*)x, st)
+                   : cudaSuccess;
+        if (e != cudaSuccess) return cuda_fail(e, "ffn launch");
         const fdl::EpiSwiGLU es{(fdl::bf16*)f, ffn};
         e = fdl::skinny_ok(gu)
             ? fdl::launch_skinny_swiglu(gu, x, w_gu, es, ctx->d_acc, ctx->acc_bytes,

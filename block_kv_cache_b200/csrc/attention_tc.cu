@@ -168,19 +168,28 @@ struct ProQKV {
     int M;
     EpiQKV p;
     __device__ void work(int part, int nparts) const {
-        constexpr int D = 128, U = 4;
+        constexpr int D = 128, U = 8;
         const int heads = p.n_q_heads + 2 * p.n_kv_heads, N = heads * D;
         const int n = M * heads * 64, stride = nparts * blockDim.x;
         for (int e0 = part * blockDim.x + threadIdx.x; e0 < n; e0 += U * stride) {
-            float lo[U], hi[U];
+            // every load of the batch first (sums, bias, rotation), then the math
+            float lo[U], hi[U], b0[U], b1[U];
+            float2 cs[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {           // every load first, then the math
+            for (int u = 0; u < U; ++u) {
                 const int e = e0 + u * stride;
                 if (e < n) {
                     const int t = e / (heads * 64), r = e - t * heads * 64;
-                    const float* row = acc + (size_t)t * N + (r >> 6) * D + (r & 63);
+                    const int h = r >> 6, d = r & 63;
+                    const float* row = acc + (size_t)t * N + h * D + d;
                     lo[u] = __ldcg(row);
                     hi[u] = __ldcg(row + 64);
+                    b0[u] = p.bias ? __ldg(p.bias + h * D + d) : 0.f;
+                    b1[u] = p.bias ? __ldg(p.bias + h * D + d + 64) : 0.f;
+                    const int pos = p.pos0 + t % p.rows_per_seq;
+                    cs[u] = h < p.n_q_heads + p.n_kv_heads
+                                ? __ldg(p.rope + (size_t)pos * (D / 2) + d)
+                                : make_float2(1.f, 0.f);
                 }
             }
 #pragma unroll
@@ -192,18 +201,9 @@ struct ProQKV {
                 float* row = acc + (size_t)t * N + h * D + d;
                 __stcg(row, 0.f);
                 __stcg(row + 64, 0.f);
-                float y0 = lo[u], y1 = hi[u];
-                if (p.bias) {
-                    y0 += p.bias[h * D + d];
-                    y1 += p.bias[h * D + d + 64];
-                }
+                const float y0 = lo[u] + b0[u], y1 = hi[u] + b1[u];
+                const float r0 = y0 * cs[u].x - y1 * cs[u].y, r1 = y1 * cs[u].x + y0 * cs[u].y;
                 const int seq = t / p.rows_per_seq, pos = p.pos0 + t % p.rows_per_seq;
-                if (h < p.n_q_heads + p.n_kv_heads) {
-                    const float2 cs = p.rope[(size_t)pos * (D / 2) + d];
-                    const float r0 = y0 * cs.x - y1 * cs.y, r1 = y1 * cs.x + y0 * cs.y;
-                    y0 = r0;
-                    y1 = r1;
-                }
                 bf16* dst;
                 if (h < p.n_q_heads)
                     dst = p.q + ((size_t)t * p.n_q_heads + h) * D;
@@ -213,8 +213,8 @@ struct ProQKV {
                 else
                     dst = p.v_cache + (((size_t)seq * p.n_kv_heads + h - p.n_q_heads - p.n_kv_heads) *
                                            p.seq_len + pos) * D;
-                dst[d] = __float2bfloat16_rn(y0);
-                dst[d + 64] = __float2bfloat16_rn(y1);
+                dst[d] = __float2bfloat16_rn(r0);
+                dst[d + 64] = __float2bfloat16_rn(r1);
             }
         }
     }

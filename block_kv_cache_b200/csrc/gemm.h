@@ -51,21 +51,33 @@ cudaError_t launch_skinny_qkv(const GemmShape& g, const void* x, const void* w, 
                               float* acc, size_t acc_bytes, int sm_count, int* err,
                               cudaStream_t st);
 
+// RMSNorm applied by a fused kernel to its activation rows: x = bf16(h *
+// rsqrt(mean(h^2) + eps) * w), x then being the kernel's operand.
+struct NormIn {
+    const float* h;          // [rows, hidden] f32 residual stream
+    const float* w;          // [hidden]
+    float eps;
+};
+
 // K splits the few-row q/k/v projection uses with an accumulator of acc_bytes
 // (1: none), and the projection alone leaving its split-K sums in acc (the
 // epilogue is then up to the caller: launch_qkv_attention_bf16).
 int skinny_qkv_splits(const GemmShape& g, size_t acc_bytes, int sm_count);
+// With norm, the projection's CTAs first write x = RMSNorm(h) (grid barrier
+// on the two words at bar).
 cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void* w, float* acc,
-                                   int splits, int sm_count, int* err, cudaStream_t st);
+                                   int splits, const NormIn* norm, unsigned* bar, int sm_count,
+                                   int* err, cudaStream_t st);
 
 // Feed-forward block for M <= 256 rows: h[M, ld_h] += down(SwiGLU(x W_gu^T)),
 // w_gu [2F, K] interleaved (row 2f gate, 2f + 1 up), w_down [ld_h, F], f [M, F]
 // bf16 scratch (the down projection's operand). acc/acc_bytes as above; bar:
-// two zeroed words for the grid barrier of the down projection.
+// four zeroed words for the grid barriers. With norm, x is first written as
+// RMSNorm(norm->h) by the gate/up projection's CTAs.
 cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* w_gu,
                               const void* w_down, bf16* f, float* h, int ld_h, float* acc,
-                              size_t acc_bytes, unsigned* bar, int sm_count, int* err,
-                              cudaStream_t st);
+                              size_t acc_bytes, unsigned* bar, const NormIn* norm, int sm_count,
+                              int* err, cudaStream_t st);
 
 // out[i, :] = bf16(h[src_i, :] / sqrt(mean(h[src_i]^2) + eps) * weight), src_i =
 // row_map ? row_map[i] : i.

@@ -227,6 +227,75 @@ struct ProSwiGLU {
     }
 };
 
+// RMSNorm of the rows of the f32 residual stream that the GEMM consumes,
+// done by its own CTAs instead of a kernel of its own: CTA c normalises rows
+// c, c + grid, ... (a block reduction of the sum of squares, then
+// out = bf16(h * rsqrt(mean(h^2) + eps) * w)), then all CTAs meet at a grid
+// barrier before the TMA reads `out` as the activation operand.
+struct ProRMSNorm {
+    static constexpr bool kActive = true;
+    unsigned* bar;           // grid barrier words
+    const float* h;          // [M, D] f32
+    const float* w;          // [D]
+    float eps;
+    int M, D;
+    bf16* out;               // [M, D]: the GEMM's X
+    __device__ void work(int part, int nparts) const {
+        constexpr int RV = 8;                        // float4 of a row held per thread
+        __shared__ float red[SK_THREADS / 32];
+        const int n4 = D / 4;
+        const bool in_regs = n4 <= RV * (int)blockDim.x;
+        for (int r = part; r < M; r += nparts) {
+            const float4* x = reinterpret_cast<const float4*>(h + (size_t)r * D);
+            float4 v[RV];
+            float ss = 0.f;
+            if (in_regs) {                           // one pass: the row stays in registers
+#pragma unroll
+                for (int k = 0; k < RV; ++k) {
+                    const int j = threadIdx.x + k * blockDim.x;
+                    v[k] = j < n4 ? __ldcg(x + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int k = 0; k < RV; ++k)
+                    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+            } else {
+                for (int j = threadIdx.x; j < n4; j += blockDim.x) {
+                    const float4 u = __ldcg(x + j);
+                    ss += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w;
+                }
+            }
+            ss = warp_sum(ss);
+            if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+            __syncthreads();
+            float tot = 0.f;
+#pragma unroll
+            for (int k = 0; k < SK_THREADS / 32; ++k) tot += red[k];
+            const float inv = rsqrtf(tot / (float)D + eps);
+            const float4* w4 = reinterpret_cast<const float4*>(w);
+            __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + (size_t)r * D);
+            if (in_regs) {
+#pragma unroll
+                for (int k = 0; k < RV; ++k) {
+                    const int j = threadIdx.x + k * blockDim.x;
+                    if (j < n4) {
+                        const float4 g = __ldg(w4 + j);
+                        o2[2 * j] = __floats2bfloat162_rn(v[k].x * inv * g.x, v[k].y * inv * g.y);
+                        o2[2 * j + 1] =
+                            __floats2bfloat162_rn(v[k].z * inv * g.z, v[k].w * inv * g.w);
+                    }
+                }
+            } else {
+                for (int j = threadIdx.x; j < n4; j += blockDim.x) {
+                    const float4 u = __ldcg(x + j), g = __ldg(w4 + j);
+                    o2[2 * j] = __floats2bfloat162_rn(u.x * inv * g.x, u.y * inv * g.y);
+                    o2[2 * j + 1] = __floats2bfloat162_rn(u.z * inv * g.z, u.w * inv * g.w);
+                }
+            }
+            __syncthreads();                        // red[] is reused by the next row
+        }
+    }
+};
+
 template <int NT, class Epi, class Pro>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -543,7 +612,11 @@ int skinny_qkv_splits(const GemmShape& g, size_t acc_bytes, int sm_count) {
 }
 
 cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void* w, float* acc,
-                                   int splits, int sm_count, int* err, cudaStream_t st) {
+                                   int splits, const NormIn* norm, unsigned* bar, int sm_count,
+                                   int* err, cudaStream_t st) {
+    if (norm)
+        return dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st,
+                               ProRMSNorm{bar, norm->h, norm->w, norm->eps, g.M, g.K, (bf16*)x});
     return dispatch_skinny(g, x, w, SkAccum{acc, g.N}, splits, sm_count, err, st);
 }
 
@@ -552,8 +625,8 @@ cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void
 // sums into f = bf16(silu(g) * u) (grid barrier, no kernel in between).
 cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* w_gu,
                               const void* w_down, bf16* f, float* h, int ld_h, float* acc,
-                              size_t acc_bytes, unsigned* bar, int sm_count, int* err,
-                              cudaStream_t st) {
+                              size_t acc_bytes, unsigned* bar, const NormIn* norm, int sm_count,
+                              int* err, cudaStream_t st) {
     const int F = g_gu.N / 2;
     const GemmShape g_dn{g_gu.M, ld_h, F};
     const int splits = acc && (size_t)g_gu.M * g_gu.N * 4 <= acc_bytes
@@ -562,12 +635,21 @@ cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* 
     const int dn_splits = choose_splits(g_dn, sm_count, 16);
     cudaError_t e;
     if (splits == 1) {
+        if (norm) {
+            e = launch_rmsnorm(g_gu.M, g_gu.K, norm->h, nullptr, norm->w, norm->eps, (bf16*)x, st);
+            if (e != cudaSuccess) return e;
+        }
         e = dispatch_skinny(g_gu, x, w_gu, SkSwiGLU{EpiSwiGLU{f, F}}, 1, sm_count, err, st);
         if (e != cudaSuccess) return e;
         return dispatch_skinny(g_dn, f, w_down, SkResid{pr, dn_splits}, dn_splits, sm_count, err,
                                st);
     }
-    e = dispatch_skinny(g_gu, x, w_gu, SkAccum{acc, g_gu.N}, splits, sm_count, err, st);
+    if (norm)
+        e = dispatch_skinny(g_gu, x, w_gu, SkAccum{acc, g_gu.N}, splits, sm_count, err, st,
+                            ProRMSNorm{bar + 2, norm->h, norm->w, norm->eps, g_gu.M, g_gu.K,
+                                       (bf16*)x});
+    else
+        e = dispatch_skinny(g_gu, x, w_gu, SkAccum{acc, g_gu.N}, splits, sm_count, err, st);
     if (e != cudaSuccess) return e;
     return dispatch_skinny(g_dn, f, w_down, SkResid{pr, dn_splits}, dn_splits, sm_count, err, st,
                            ProSwiGLU{bar, acc, g_gu.M, F, f});

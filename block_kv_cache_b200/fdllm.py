@@ -40,7 +40,7 @@ class AttnDesc(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 
 class LMHeadDesc(ctypes.Structure):
@@ -108,9 +108,10 @@ def load() -> ctypes.CDLL:
     L.fdl_linear_residual.argtypes = [vp, i, i, i, vp, vp, vp, vp]
     L.fdl_linear_swiglu.argtypes = [vp, i, i, i, vp, vp, vp, vp]
     L.fdl_full_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp]
-    L.fdl_ffn.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
-    L.fdl_qkv_attention.argtypes = [vp, ctypes.POINTER(QKVDesc), vp, vp, vp, vp, vp, vp, vp, vp,
-                                    vp]
+    fl = ctypes.c_float
+    L.fdl_ffn.argtypes = [vp, i, i, i, vp, fl, vp, vp, vp, vp, vp, vp]
+    L.fdl_qkv_attention.argtypes = [vp, ctypes.POINTER(QKVDesc), vp, vp, fl, vp, vp, vp, vp, vp,
+                                    vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -334,17 +335,22 @@ class Context:
         return q_out
 
     def qkv_attention(self, x, w, rope, q_out, k_cache, v_cache, out, *, n_q_heads,
-                      rows_per_seq, pos0, bias=None, stream=None):
-        """qkv_rope_store of the block rows, then DualCache attention of the block
-        [pos0, pos0 + rows_per_seq) of every sequence over the caches -> out."""
+                      rows_per_seq, pos0, bias=None, h=None, norm_w=None, eps=1e-5,
+                      stream=None):
+        """[x = RMSNorm(h) * norm_w if norm_w is given], qkv_rope_store of the block
+        rows, then DualCache attention of the block [pos0, pos0 + rows_per_seq) of
+        every sequence over the caches -> out."""
         _need(x, "x", torch.bfloat16, 2)
         _need(w, "w", torch.bfloat16, 2)
+        if norm_w is not None:
+            _need(h, "h", torch.float32, 2)
         b, hkv, L, d = k_cache.shape
         d_ = QKVDesc(x.shape[0], x.shape[1], int(n_q_heads), hkv, d, b, L, int(rows_per_seq),
                      int(pos0), rope.shape[0])
-        _check(load().fdl_qkv_attention(self._h, ctypes.byref(d_), _ptr(x), _ptr(w), _ptr(bias),
-                                        _ptr(rope), _ptr(q_out), _ptr(k_cache), _ptr(v_cache),
-                                        _ptr(out), _stream(stream)))
+        _check(load().fdl_qkv_attention(self._h, ctypes.byref(d_), _ptr(h), _ptr(norm_w),
+                                        float(eps), _ptr(x), _ptr(w), _ptr(bias), _ptr(rope),
+                                        _ptr(q_out), _ptr(k_cache), _ptr(v_cache), _ptr(out),
+                                        _stream(stream)))
         return out
 
     def linear_residual(self, x, w, h, *, stream=None):
@@ -367,8 +373,9 @@ class Context:
                                         _ptr(out), _stream(stream)))
         return out
 
-    def ffn(self, x, w_gu, w_down, h, *, f=None, stream=None):
-        """h += (silu(x Wg^T) * (x Wu^T)) Wd^T; returns f, the SwiGLU output."""
+    def ffn(self, x, w_gu, w_down, h, *, f=None, norm_w=None, eps=1e-5, stream=None):
+        """[x = RMSNorm(h) * norm_w if norm_w is given], then
+        h += (silu(x Wg^T) * (x Wu^T)) Wd^T; returns f, the SwiGLU output."""
         _need(x, "x", torch.bfloat16, 2)
         _need(w_gu, "w_gu", torch.bfloat16, 2)
         _need(w_down, "w_down", torch.bfloat16, 2)
@@ -377,8 +384,8 @@ class Context:
         F = w_gu.shape[0] // 2
         if f is None:
             f = torch.empty((rows, F), dtype=torch.bfloat16, device=x.device)
-        _check(load().fdl_ffn(self._h, rows, hidden, F, _ptr(x), _ptr(w_gu), _ptr(w_down),
-                              _ptr(f), _ptr(h), _stream(stream)))
+        _check(load().fdl_ffn(self._h, rows, hidden, F, _ptr(norm_w), float(eps), _ptr(x),
+                              _ptr(w_gu), _ptr(w_down), _ptr(f), _ptr(h), _stream(stream)))
         return f
 
     def full_attention(self, q, k_cache, v_cache, *, out=None, scale=0.0, stream=None):

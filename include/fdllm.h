@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define FDL_ABI_VERSION 1
+#define FDL_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define FDL_API __attribute__((visibility("default")))
@@ -300,22 +300,29 @@ FDL_API int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* desc, const voi
                                const void* w, const float* bias, const float* rope,
                                void* q_out, void* k_cache, void* v_cache, void* stream);
 
-/* The block-slot projection of a cached DualCache step followed by the block's
- * attention: the result equals fdl_qkv_rope_store(desc, ...) and then
- * fdl_dualcache_attention over the caches with block_start = desc->pos0,
- * block_len = desc->rows_per_seq, scale 1/sqrt(128) and no LSE. Requires
- * rows == batch * rows_per_seq (the block rows of every sequence) and
- * rows_per_seq <= 128. out [batch, rows_per_seq, n_q_heads, 128] bf16 is
- * written; q_out, k_cache, v_cache as for fdl_qkv_rope_store. When the
- * attention grid fits on the device at once, the projection's epilogue
- * (bias, RoPE, q and block-slot store) is done by the CTAs of the attention
- * kernel between a grid-wide barrier and the attention, instead of by a
- * kernel of its own. Errors: as fdl_qkv_rope_store, plus FDL_EINVAL for the
- * row layout. */
-FDL_API int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* desc, const void* x,
-                              const void* w, const float* bias, const float* rope,
-                              void* q_out, void* k_cache, void* v_cache, void* out,
-                              void* stream);
+/* The attention half of a cached DualCache step for the block rows:
+ *   x = RMSNorm(h) * norm_w          (when norm_w != NULL; x is then written)
+ *   q, k, v = x w^T (+ bias), RoPE, k/v into the cache block slot
+ *   out = DualCache attention of the block over the whole cache
+ * The result equals fdl_rmsnorm (if norm_w), fdl_qkv_rope_store(desc, ...) and
+ * fdl_dualcache_attention with block_start = desc->pos0, block_len =
+ * desc->rows_per_seq, scale 1/sqrt(128), no LSE. Requires rows == batch *
+ * rows_per_seq (the block rows of every sequence), rows_per_seq <= 128.
+ *   h       [rows, hidden] f32 (read; only with norm_w); norm_w [hidden] f32;
+ *           eps > 0 the RMSNorm epsilon
+ *   x       [rows, hidden] bf16: written when norm_w is given, else the input
+ *   out     [batch, rows_per_seq, n_q_heads, 128] bf16 (written)
+ *   q_out, k_cache, v_cache, w, bias, rope as for fdl_qkv_rope_store.
+ * When the shapes allow (few rows, split-K projection, an attention grid that
+ * fits on the device at once) the RMSNorm runs in the projection's kernel and
+ * the projection's epilogue (bias, RoPE, q and block-slot store) in the
+ * attention kernel, each behind a grid-wide barrier, instead of in kernels
+ * of their own. Errors: as fdl_qkv_rope_store, plus FDL_EINVAL for the row
+ * layout or the norm arguments. */
+FDL_API int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* desc, const float* h,
+                              const float* norm_w, float eps, void* x, const void* w,
+                              const float* bias, const float* rope, void* q_out, void* k_cache,
+                              void* v_cache, void* out, void* stream);
 
 /* h[rows, out_features] += x w^T  (f32 residual stream; x bf16 [rows, in],
  * w bf16 [out, in]). in % 64 == 0, out % 64 == 0. Errors: FDL_EINVAL, FDL_ECUDA. */
@@ -329,19 +336,22 @@ FDL_API int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in
 FDL_API int fdl_linear_swiglu(fdl_ctx* ctx, int rows, int out_features, int in_features,
                               const void* x, const void* w_gu, void* out, void* stream);
 
-/* Feed-forward half of a layer with its residual (SwiGLU MLP):
+/* Feed-forward half of a layer with its residual (pre-norm SwiGLU MLP):
+ *   x  = RMSNorm(h) * norm_w           (when norm_w != NULL; x is then written)
  *   f  = silu(x Wg^T) * (x Wu^T)      bf16 [rows, ffn], written
  *   h += f Wd^T                        f32 [rows, hidden], updated
- * x bf16 [rows, hidden]; w_gu bf16 [2*ffn, hidden] interleaved as for
- * fdl_linear_swiglu; w_down bf16 [hidden, ffn]. hidden % 64 == 0,
- * ffn % 64 == 0. The result equals fdl_linear_swiglu followed by
- * fdl_linear_residual. For the few rows of a cached block step (rows <= 256,
- * hidden and ffn multiples of 128) the SwiGLU of the split-K gate/up sums is
- * applied by the CTAs of the down projection, between a grid-wide barrier
- * and the projection itself, instead of by a kernel of its own.
+ * x bf16 [rows, hidden] (the input when norm_w is NULL); norm_w [hidden] f32,
+ * eps > 0; w_gu bf16 [2*ffn, hidden] interleaved as for fdl_linear_swiglu;
+ * w_down bf16 [hidden, ffn]. hidden % 64 == 0, ffn % 64 == 0. The result
+ * equals fdl_rmsnorm (if norm_w), fdl_linear_swiglu and fdl_linear_residual.
+ * For the few rows of a cached block step (rows <= 256, hidden and ffn
+ * multiples of 128) the RMSNorm runs in the gate/up projection's kernel and
+ * the SwiGLU of the split-K gate/up sums in the down projection's kernel,
+ * each behind a grid-wide barrier, instead of in kernels of their own.
  * Errors: FDL_EINVAL, FDL_ECUDA. */
-FDL_API int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const void* x,
-                    const void* w_gu, const void* w_down, void* f, float* h, void* stream);
+FDL_API int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const float* norm_w, float eps,
+                    void* x, const void* w_gu, const void* w_down, void* f, float* h,
+                    void* stream);
 
 /* Full bidirectional attention of every position (the refresh forward after
  * a block completes): out[b, i, h, :] = softmax over all j of q_i . k_j.

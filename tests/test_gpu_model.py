@@ -99,91 +99,58 @@ def test_linear_swiglu(ctx, M, F, K):
     assert rel(out.float().cpu().numpy(), ref) <= BF16_TOL
 
 
-@pytest.mark.parametrize("M,D,F", [(32, 4096, 12288), (32, 512, 1024), (7, 256, 640),
-                                   (64, 1024, 4096), (300, 256, 192), (1, 128, 128)])
-def test_ffn_block(ctx, M, D, F):
-    """h += SwiGLU(x) Wd^T in one call; for few rows the SwiGLU of the split-K
-    sums runs in the down projection's kernel behind a grid barrier. Called
-    twice so that the context's scratch (zeroed sums, barrier words) is
-    checked to be reusable."""
-    g = synth.rng(M * 7 + F)
-    x = bf_vals(g.standard_normal((M, D)))
+@pytest.mark.parametrize("M,D,F,norm", [(32, 4096, 12288, True), (32, 4096, 12288, False),
+                                        (32, 512, 1024, True), (7, 256, 640, True),
+                                        (64, 1024, 4096, True), (300, 256, 192, True),
+                                        (1, 128, 128, False)])
+def test_ffn_block(ctx, M, D, F, norm):
+    """h += SwiGLU(RMSNorm(h) or x) Wd^T in one call; for few rows the norm runs
+    in the gate/up kernel and the SwiGLU of the split-K sums in the down
+    projection's kernel, each behind a grid barrier. Called twice so that
+    the context's scratch (zeroed sums, barrier words) is checked to be
+    reusable."""
+    g = synth.rng(M * 7 + F + norm)
     wg = bf_vals(g.standard_normal((F, D)) * 0.05)
     wu = bf_vals(g.standard_normal((F, D)) * 0.05)
     wd = bf_vals(g.standard_normal((D, F)) * 0.03)
     wgu = np.empty((2 * F, D), np.float32)
     wgu[0::2], wgu[1::2] = wg, wu
-    h0 = g.standard_normal((M, D)).astype(np.float32)
-    x64 = x.astype(np.float64)
-    f_ref = O.silu(x64 @ wg.T) * (x64 @ wu.T)
-    xg, wgug, wdg = bf(x), bf(wgu), bf(wd)
+    h0 = (g.standard_normal((M, D)) * 2).astype(np.float32)
+    wn = g.uniform(0.5, 1.5, D).astype(np.float32)
+    x_in = bf_vals(g.standard_normal((M, D)))
+    x_ref = O.rms_norm(h0, wn, 1e-5) if norm else x_in.astype(np.float64)
+    wgug, wdg = bf(wgu), bf(wd)
     for rep in range(2):
         h = f32(h0)
-        f = ctx.ffn(xg, wgug, wdg, h)
+        x = torch.empty((M, D), dtype=torch.bfloat16, device="cuda") if norm else bf(x_in)
+        f = ctx.ffn(x, wgug, wdg, h, norm_w=f32(wn) if norm else None, eps=1e-5)
+        if norm:
+            assert rel(x.float().cpu().numpy(), x_ref) <= BF16_TOL, rep
+        xg64 = x.float().cpu().numpy().astype(np.float64)   # the operand the GEMMs consumed
+        f_ref = O.silu(xg64 @ wg.T) * (xg64 @ wu.T)
         assert rel(f.float().cpu().numpy(), f_ref) <= BF16_TOL, rep
-        # the down projection consumes the bf16 f the call wrote
         ref = h0.astype(np.float64) + f.float().cpu().numpy().astype(np.float64) @ wd.astype(np.float64).T
         assert rel(h.cpu().numpy(), ref) <= 1e-4, rep
     ctx.device_status()
 
 
-@pytest.mark.parametrize("Hq,Hkv,bias,rows_per_seq,pos0,batch,L", [
-    (4, 4, False, 32, 64, 2, 128),     # block slot of 2 sequences
-    (4, 2, True, 128, 0, 2, 128),      # refresh: every position, GQA, Qwen-style bias
-    (7, 1, True, 32, 96, 1, 160),
+@pytest.mark.parametrize("batch,Hq,Hkv,bias,B,pos0,L,D,norm", [
+    (1, 32, 32, False, 32, 1024, 2048, 4096, True),   # LLaDA-8B layer: fused path
+    (1, 32, 32, False, 32, 1024, 2048, 4096, False),
+    (1, 8, 8, False, 32, 96, 256, 1024, True),        # fused, several splits per head
+    (2, 28, 4, True, 32, 512, 1024, 3584, True),      # GQA 7:1 with bias (Dream / Qwen2.5)
+    (2, 4, 2, True, 32, 64, 160, 256, True),          # no K split: separate calls
 ])
-def test_qkv_rope_store(ctx, Hq, Hkv, bias, rows_per_seq, pos0, batch, L):
-    g = synth.rng(Hq * 10 + pos0)
-    D, d = 256, 128
-    M = rows_per_seq * batch
-    N = (Hq + 2 * Hkv) * d
-    x = bf_vals(g.standard_normal((M, D)))
-    w = bf_vals(g.standard_normal((N, D)) * 0.06)
-    b = (g.standard_normal(N) * 0.1).astype(np.float32) if bias else None
-    k0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
-    v0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
-    from block_kv_cache_b200 import fdllm
-    rope = torch.from_numpy(fdllm.rope_table(10000.0, L, d)).cuda()
-    kc, vc = bf(k0), bf(v0)
-    q = torch.empty((M, Hq, d), dtype=torch.bfloat16, device="cuda")
-    ctx.qkv_rope_store(bf(x), bf(w), rope, q, kc, vc, n_q_heads=Hq, rows_per_seq=rows_per_seq,
-                       pos0=pos0, bias=None if b is None else f32(b))
-    y = x.astype(np.float64) @ w.astype(np.float64).T
-    if b is not None:
-        y = y + b
-    pos = pos0 + np.arange(M) % rows_per_seq
-    qr = O.apply_rope(y[:, :Hq * d].reshape(M, Hq, d), pos)
-    kr = O.apply_rope(y[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d), pos)
-    vr = y[:, (Hq + Hkv) * d:].reshape(M, Hkv, d)
-    assert rel(q.float().cpu().numpy(), qr) <= BF16_TOL
-    kg, vg = kc.float().cpu().numpy(), vc.float().cpu().numpy()
-    written = np.zeros((batch, L), bool)
-    for r in range(M):
-        sq, p = r // rows_per_seq, pos[r]
-        written[sq, p] = True
-        assert np.abs(kg[sq, :, p] - kr[r]).max() <= BF16_TOL * np.abs(kr).max()
-        assert np.abs(vg[sq, :, p] - vr[r]).max() <= BF16_TOL * np.abs(vr).max()
-    # rows outside the written positions untouched
-    for sq in range(batch):
-        keep = ~written[sq]
-        assert np.array_equal(kg[sq][:, keep], k0[sq][:, keep])
-        assert np.array_equal(vg[sq][:, keep], v0[sq][:, keep])
-
-
-@pytest.mark.parametrize("batch,Hq,Hkv,bias,B,pos0,L,D", [
-    (1, 32, 32, False, 32, 1024, 2048, 4096),   # LLaDA-8B layer: fused path
-    (1, 8, 8, False, 32, 96, 256, 1024),        # fused, several splits per head
-    (2, 28, 4, True, 32, 512, 1024, 3584),      # GQA 7:1 with bias (Dream / Qwen2.5 shape)
-    (2, 4, 2, True, 32, 64, 160, 256),          # no K split: separate calls
-])
-def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D):
-    """Block-slot projection + DualCache attention in one call equals the
-    oracle's projection, RoPE, cache store and attention over the cache."""
-    g = synth.rng(Hq * 3 + L + D)
+def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D, norm):
+    """Norm + block-slot projection + DualCache attention in one call equals
+    the oracle's norm, projection, RoPE, cache store and attention."""
+    g = synth.rng(Hq * 3 + L + D + norm)
     d = 128
     M = batch * B
     N = (Hq + 2 * Hkv) * d
-    x = bf_vals(g.standard_normal((M, D)))
+    h0 = (g.standard_normal((M, D)) * 2).astype(np.float32)
+    wn = g.uniform(0.5, 1.5, D).astype(np.float32)
+    x_in = bf_vals(g.standard_normal((M, D)))
     w = bf_vals(g.standard_normal((N, D)) * (1.0 / np.sqrt(D)))
     bvec = (g.standard_normal(N) * 0.1).astype(np.float32) if bias else None
     k0 = bf_vals(g.standard_normal((batch, Hkv, L, d)))
@@ -193,12 +160,18 @@ def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D):
     kc, vc = bf(k0), bf(v0)
     q = torch.empty((M, Hq, d), dtype=torch.bfloat16, device="cuda")
     out = torch.empty((batch, B, Hq, d), dtype=torch.bfloat16, device="cuda")
-    xg, wg = bf(x), bf(w)
+    wg = bf(w)
     bg = None if bvec is None else f32(bvec)
+    hg, wng = f32(h0), f32(wn)
     for rep in range(2):                       # scratch and barrier words are reusable
+        xg = torch.empty((M, D), dtype=torch.bfloat16, device="cuda") if norm else bf(x_in)
         ctx.qkv_attention(xg, wg, rope, q, kc, vc, out, n_q_heads=Hq, rows_per_seq=B,
-                          pos0=pos0, bias=bg)
+                          pos0=pos0, bias=bg, h=hg if norm else None,
+                          norm_w=wng if norm else None, eps=1e-5)
         ctx.device_status()
+        x = xg.float().cpu().numpy()            # the operand the projection consumed
+        if norm:
+            assert rel(x, O.rms_norm(h0, wn, 1e-5)) <= BF16_TOL
         y = x.astype(np.float64) @ w.astype(np.float64).T
         if bvec is not None:
             y = y + bvec
