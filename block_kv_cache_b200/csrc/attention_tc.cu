@@ -722,7 +722,7 @@ cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads,
                                        cudaStream_t st) {
     // query blocks of Bq rows: as many whole heads of a GQA group per 256 rows
     const int grp = n_q_heads / n_kv_heads;
-    int bq = grp == 1 ? 128 : grp == 2 ? 128 : grp <= 4 ? 64 : 32;
+    int bq = grp == 1 ? 256 : grp == 2 ? 128 : grp <= 4 ? 64 : 32;
     while (bq > 32 && seq_len % bq) bq /= 2;
     if (seq_len % bq) return cudaErrorInvalidValue;
     AttnShape s{batch * (seq_len / bq), n_q_heads, n_kv_heads, head_dim, seq_len, 0, bq, scale,

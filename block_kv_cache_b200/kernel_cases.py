@@ -87,6 +87,28 @@ def run_attention(a, ctx):
             "TFLOPs": flops / us / 1e6}
 
 
+def run_full(a, ctx):
+    """Full bidirectional attention of every position (the refresh forward):
+    q [b, L, Hq, d], caches [b, Hkv, L, d], `layers` distinct caches cycled."""
+    L = a.prefix + a.block + a.suffix
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    qs = [torch.randn(a.batch, L, a.heads, a.head_dim, generator=g, device="cuda").to(
+        torch.bfloat16) for _ in range(a.layers)]
+    ks = [torch.randn(a.batch, a.kv_heads, L, a.head_dim, generator=g, device="cuda").to(
+        torch.bfloat16) for _ in range(a.layers)]
+    vs = [torch.randn_like(k) for k in ks]
+    out = torch.empty_like(qs[0])
+    us = _timed(a, lambda i: ctx.full_attention(qs[i % a.layers], ks[i % a.layers],
+                                                vs[i % a.layers], out=out))
+    ctx.device_status()
+    flops = 4.0 * a.batch * a.heads * L * L * a.head_dim
+    nbytes = 2 * a.batch * a.kv_heads * L * a.head_dim * 2 + 2 * a.batch * L * a.heads * a.head_dim * 2
+    return {"op": "full_attention", "heads": a.heads, "kv_heads": a.kv_heads, "L": L,
+            "batch": a.batch, "graph": a.graph, "us": us, "GBps": nbytes / us / 1e3,
+            "TFLOPs": flops / us / 1e6}
+
+
 def run_linear(a, ctx):
     """One projection of the transformer at (rows, n, k); `layers` distinct weight
     matrices are cycled so the weight stream comes from HBM, not L2."""
@@ -140,7 +162,7 @@ def run_ffn(a, ctx):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["lmhead", "attention", "swiglu", "resid", "qkv", "ffn"])
+    p.add_argument("op", choices=["lmhead", "attention", "full", "swiglu", "resid", "qkv", "ffn"])
     p.add_argument("--n", type=int, default=24576)
     p.add_argument("--k", type=int, default=4096)
     p.add_argument("--rows", type=int, default=32)
@@ -166,6 +188,8 @@ def main():
         r = run_attention(a, ctx)
     elif a.op == "ffn":
         r = run_ffn(a, ctx)
+    elif a.op == "full":
+        r = run_full(a, ctx)
     else:
         r = run_linear(a, ctx)
     print(json.dumps(r), flush=True)
