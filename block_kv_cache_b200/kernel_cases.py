@@ -109,6 +109,37 @@ def run_full(a, ctx):
             "TFLOPs": flops / us / 1e6}
 
 
+def run_qkv_attention(a, ctx):
+    """The attention half of a cached step: RMSNorm + block-slot projection +
+    DualCache attention (`layers` distinct weights and caches cycled)."""
+    from block_kv_cache_b200 import fdllm as F
+    L = a.prefix + a.block + a.suffix
+    Hq, Hkv, d, D = a.heads, a.kv_heads, a.head_dim, a.hidden
+    N = (Hq + 2 * Hkv) * d
+    rows = a.batch * a.block
+    g = torch.Generator(device="cuda")
+    g.manual_seed(0)
+    ws = [(torch.randn(N, D, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+          for _ in range(a.layers)]
+    kc = [torch.randn(a.batch, Hkv, L, d, generator=g, device="cuda").to(torch.bfloat16)
+          for _ in range(a.layers)]
+    vc = [torch.randn_like(k) for k in kc]
+    h = torch.randn(rows, D, generator=g, device="cuda")
+    nw = torch.ones(D, device="cuda")
+    x = torch.empty((rows, D), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((rows, Hq, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((a.batch, a.block, Hq, d), dtype=torch.bfloat16, device="cuda")
+    rope = torch.from_numpy(F.rope_table(10000.0, L, d)).cuda()
+    us = _timed(a, lambda i: ctx.qkv_attention(x, ws[i % a.layers], rope, q, kc[i % a.layers],
+                                               vc[i % a.layers], out, n_q_heads=Hq,
+                                               rows_per_seq=a.block, pos0=a.prefix, h=h,
+                                               norm_w=nw))
+    ctx.device_status()
+    nbytes = N * D * 2 + 2 * a.batch * Hkv * L * d * 2 + rows * D * 6 + 2 * rows * Hq * d * 2
+    return {"op": "qkv_attention", "rows": rows, "hidden": D, "heads": Hq, "kv_heads": Hkv,
+            "L": L, "graph": a.graph, "us": us, "GBps": nbytes / us / 1e3}
+
+
 def run_linear(a, ctx):
     """One projection of the transformer at (rows, n, k); `layers` distinct weight
     matrices are cycled so the weight stream comes from HBM, not L2."""
@@ -150,10 +181,12 @@ def run_ffn(a, ctx):
            for _ in range(a.layers)]
     wd = [(torch.randn(a.k, a.n, generator=g, device="cuda") * 0.02).to(torch.bfloat16)
           for _ in range(a.layers)]
-    x = torch.randn(a.rows, a.k, generator=g, device="cuda").to(torch.bfloat16)
-    h = torch.zeros((a.rows, a.k), dtype=torch.float32, device="cuda")
+    x = torch.empty((a.rows, a.k), dtype=torch.bfloat16, device="cuda")
+    h = torch.randn(a.rows, a.k, generator=g, device="cuda")
+    nw = torch.ones(a.k, device="cuda")
     f = torch.empty((a.rows, a.n), dtype=torch.bfloat16, device="cuda")
-    us = _timed(a, lambda i: ctx.ffn(x, wgu[i % a.layers], wd[i % a.layers], h, f=f))
+    # as in a decoder layer: x = RMSNorm(h), h += down(SwiGLU(x))
+    us = _timed(a, lambda i: ctx.ffn(x, wgu[i % a.layers], wd[i % a.layers], h, f=f, norm_w=nw))
     ctx.device_status()
     nbytes = 3 * a.n * a.k * 2 + a.rows * a.k * 2 + 2 * a.rows * a.n * 2 + 2 * a.rows * a.k * 4
     return {"op": "ffn", "rows": a.rows, "hidden": a.k, "ffn": a.n, "graph": a.graph, "us": us,
@@ -162,7 +195,8 @@ def run_ffn(a, ctx):
 
 def main():
     p = argparse.ArgumentParser()
-    p.add_argument("op", choices=["lmhead", "attention", "full", "swiglu", "resid", "qkv", "ffn"])
+    p.add_argument("op", choices=["lmhead", "attention", "full", "qkvattn", "swiglu", "resid",
+                                  "qkv", "ffn"])
     p.add_argument("--n", type=int, default=24576)
     p.add_argument("--k", type=int, default=4096)
     p.add_argument("--rows", type=int, default=32)
@@ -190,6 +224,8 @@ def main():
         r = run_ffn(a, ctx)
     elif a.op == "full":
         r = run_full(a, ctx)
+    elif a.op == "qkvattn":
+        r = run_qkv_attention(a, ctx)
     else:
         r = run_linear(a, ctx)
     print(json.dumps(r), flush=True)
