@@ -135,6 +135,21 @@ def read_peaks():
 LAUNCHES = {"cached": 32 * 5 + 5, "refresh": 32 * 7 + 5}
 
 
+def combine_ranks(dist, world, ms, toks, device):
+    """Whole-job figures of a replicated run: the slowest rank's time and the
+    tokens of all ranks (every rank decodes its own sequences, so the work per
+    GPU is fixed as the rank count grows). Every rank makes the same two
+    collective calls."""
+    import torch
+    if world == 1:
+        return float(ms), float(toks)
+    t_ms = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    t_tok = torch.tensor([float(toks)], dtype=torch.float64, device=device)
+    dist.all_reduce(t_ms, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t_tok, op=dist.ReduceOp.SUM)
+    return float(t_ms.item()), float(t_tok.item())
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_gpu(args):
     import torch
@@ -198,24 +213,10 @@ def run_gpu(args):
     ms = ev0.elapsed_time(ev1)
     ctx.device_status()
 
-    t = torch.tensor([ms, float(toks)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        tm, tt = t[0:1].clone(), t[1:2].clone()
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tt, op=dist.ReduceOp.SUM)
-        ms_max, toks_all = float(tm), float(tt)
-    else:
-        ms_max, toks_all = ms, float(toks)
-
+    ms_max, toks_all = combine_ranks(dist, world, ms, toks, "cuda")
     e2e = run_e2e(torch, dec, prompt, args.e2e_steps)
-    te = torch.tensor([e2e["ms"], float(e2e["toks"])], dtype=torch.float64, device="cuda")
-    if world > 1:
-        a, b = te[0:1].clone(), te[1:2].clone()
-        dist.all_reduce(a, op=dist.ReduceOp.MAX)
-        dist.all_reduce(b, op=dist.ReduceOp.SUM)
-        e2e_val = float(b) / (float(a) / 1e3)
-    else:
-        e2e_val = e2e["toks"] / (e2e["ms"] / 1e3)
+    e2e_ms, e2e_toks = combine_ranks(dist, world, e2e["ms"], e2e["toks"], "cuda")
+    e2e_val = e2e_toks / (e2e_ms / 1e3)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -232,6 +233,10 @@ def run_gpu(args):
         ffn_bytes = 3 * F * D * 2 + 2 * M * D * 2 + 2 * M * F * 2 + 3 * M * D * 4
         sw_avg_ms = sw_ms / max(sw_n, 1)
         ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
+        # DRAM bytes read + written by the two kernels of one such call, from an
+        # ncu capture of the same kernels at this shape (kernel_cases ffn --rows
+        # 32 --n 12288 --k 4096): 205.08 + 3.51 + 104.40 + 1.77 MB
+        ffn_traffic = 205_079_808 + 3_514_624 + 104_400_896 + 1_767_424
         out = {
             "metric": METRIC, "value": toks_all / (ms_max / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -254,7 +259,9 @@ def run_gpu(args):
                                    "60% of the step's weight bytes",
                          "bytes_per_call": ffn_bytes,
                          "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                         "frac": (ach / peak) if ach else None, "traffic": None,
+                         "frac": (ach / peak) if ach else None, "traffic": ffn_traffic,
+                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
+                                           "the two kernels of one call",
                          "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)"
                          if peaks.get("hbm_gbs") else "fallback 6650 GB/s",
                          "avg_launch_us": sw_avg_ms * 1e3, "launches_timed": sw_n},
