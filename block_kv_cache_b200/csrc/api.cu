@@ -433,8 +433,8 @@ int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const
         e = fdl::launch_skinny_qkv_sums(gs, x, w, ctx->d_acc, splits, norm_w ? &ni : nullptr,
                                         ctx->d_sync + 6, ctx->sm_count, ctx->d_err, st);
         if (e == cudaSuccess)
-            e = fdl::launch_qkv_attention_bf16(as, ctx->d_acc, d->rows, p, ctx->d_sync + 4, out,
-                                               ctx->sm_count, ctx->d_err, st);
+            e = fdl::launch_qkv_attention_bf16(as, ctx->d_acc, p, out, ctx->sm_count, ctx->d_err,
+                                               st);
     } else {
         e = norm_w ? fdl::launch_rmsnorm(d->rows, d->hidden, h, nullptr, norm_w, eps,
                                          (fdl::bf16*)x, st)

@@ -74,7 +74,9 @@ namespace {
 
 template <int D, int MT>
 struct Att4 {
-    static constexpr int STAGES = MT == 1 ? 3 : 2;
+    // K/V ring depth: the ring turns over once per (HBM latency + one tile's
+    // S, softmax and PV chain), so the period of a tile is that over STAGES
+    static constexpr int STAGES = MT == 1 ? 5 : 2;
     static constexpr int THREADS = 32 * (4 * MT + 2);
     static constexpr int TMA_WARP = 4 * MT, MMA_WARP = 4 * MT + 1;
     static constexpr int DC = D / 64;
@@ -86,8 +88,8 @@ struct Att4 {
     static constexpr int OFF_K = OFF_Q + DC * Q_CHUNK;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
     static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;   // P[buffer][m]
-    static constexpr int OFF_RED = OFF_P + 2 * MT * P_TILE;  // 256 x (max, sum) floats
-    static constexpr int OFF_BAR = OFF_RED + 256 * 2 * 4;
+    static constexpr int OFF_RED = OFF_P + 2 * MT * P_TILE;  // 128 MT x (max, sum) floats
+    static constexpr int OFF_BAR = OFF_RED + 128 * MT * 2 * 4;
     static constexpr size_t TOTAL = 1024 + OFF_BAR + 256;
     // After the last MMA, [OFF_K, OFF_RED) holds this CTA's partial output
     // (R rows x D floats, float4 slots XOR-swizzled by row) for the cluster.
@@ -153,72 +155,148 @@ struct AttnArgs {
 // ---- prologues: work every CTA does after the preceding kernel -----------------
 struct AttNoPro {
     static constexpr bool kActive = false;
-    unsigned* bar = nullptr;
-    __device__ void work(int, int) const {}
 };
 
 // The epilogue of a split-K block-slot projection (bias, RoPE, q and the K/V
-// block slot written; the f32 sums zeroed again), shared by the CTAs of the
-// attention kernel that reads the result, followed by a grid barrier: no
-// kernel of its own. Item = one (token, head, dimension pair d / d + 64).
+// block slot), done by the attention CTAs that consume it, with no kernel of
+// its own and no wait on another CTA. Each CTA forms its own query tile in
+// shared memory straight from the f32 sums and writes the block-slot K/V rows
+// that fall in its own key range (only it reads them); the sums it read are
+// zeroed again (the q sums, which every split of a head reads, by split 0
+// once the cluster has merged). One query chunk per kv head (hc == grp) and
+// one query block per sequence.
 struct ProQKV {
     static constexpr bool kActive = true;
-    unsigned* bar;           // grid barrier words
     float* acc;              // [M, N] sums, N = (Hq + 2 Hkv) * 128
-    int M;
     EpiQKV p;
-    __device__ void work(int part, int nparts) const {
-        constexpr int D = 128, U = 8;
-        const int heads = p.n_q_heads + 2 * p.n_kv_heads, N = heads * D;
-        const int n = M * heads * 64, stride = nparts * blockDim.x;
-        for (int e0 = part * blockDim.x + threadIdx.x; e0 < n; e0 += U * stride) {
-            // every load of the batch first (sums, bias, rotation), then the math
-            float lo[U], hi[U], b0[U], b1[U];
-            float2 cs[U];
+};
+
+// Item = 8 consecutive dimensions d of one row and their rotation partners
+// d + 64 (RoPE over 128-dimensional heads). Loads of a batch first, then math.
+template <int QCHUNK>
+__device__ __forceinline__ void qkv_tile(const ProQKV& pro, const AttnArgs& a, uint8_t* sq,
+                                         int g, int bb, int k_begin, int k_end, bool write_q) {
+    constexpr int U = 2;
+    const EpiQKV& p = pro.p;
+    const int N = (p.n_q_heads + 2 * p.n_kv_heads) * 128;
+    const int nq = a.rows * 8;
+    const int kv0 = max(a.blk0, k_begin), kv1 = min(a.blk1, k_end);
+    const int n = nq + (kv1 > kv0 ? (kv1 - kv0) * 16 : 0);
+    for (int e0 = threadIdx.x; e0 < n; e0 += U * blockDim.x) {
+        float4 v[U][4], bs[U][4], cs[U][4];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int e = e0 + u * stride;
-                if (e < n) {
-                    const int t = e / (heads * 64), r = e - t * heads * 64;
-                    const int h = r >> 6, d = r & 63;
-                    const float* row = acc + (size_t)t * N + h * D + d;
-                    lo[u] = __ldcg(row);
-                    hi[u] = __ldcg(row + 64);
-                    b0[u] = p.bias ? __ldg(p.bias + h * D + d) : 0.f;
-                    b1[u] = p.bias ? __ldg(p.bias + h * D + d + 64) : 0.f;
-                    const int pos = p.pos0 + t % p.rows_per_seq;
-                    cs[u] = h < p.n_q_heads + p.n_kv_heads
-                                ? __ldg(p.rope + (size_t)pos * (D / 2) + d)
-                                : make_float2(1.f, 0.f);
-                }
+        for (int u = 0; u < U; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e >= n) continue;
+            int i, col, pc;
+            bool rot = true;
+            if (e < nq) {                        // q: packed row r = i * hc + j
+                const int r = e >> 3;
+                pc = e & 7;
+                i = r / a.hc;
+                col = (g * a.hc + r % a.hc) * 128;
+            } else {                             // k or v of a block-slot row
+                const int f = e - nq, kind = (f >> 3) & 1;
+                pc = f & 7;
+                i = kv0 + (f >> 4) - a.blk0;
+                col = (p.n_q_heads + kind * p.n_kv_heads + g) * 128;
+                rot = kind == 0;
             }
+            const float* src = pro.acc + (size_t)(bb * a.B + i) * N + col + pc * 8;
+            v[u][0] = __ldcg(reinterpret_cast<const float4*>(src));
+            v[u][1] = __ldcg(reinterpret_cast<const float4*>(src + 4));
+            v[u][2] = __ldcg(reinterpret_cast<const float4*>(src + 64));
+            v[u][3] = __ldcg(reinterpret_cast<const float4*>(src + 68));
+            if (p.bias) {
+                const float4* b4 = reinterpret_cast<const float4*>(p.bias + col + pc * 8);
+                bs[u][0] = __ldg(b4);
+                bs[u][1] = __ldg(b4 + 1);
+                bs[u][2] = __ldg(b4 + 16);
+                bs[u][3] = __ldg(b4 + 17);
+            } else {
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int e = e0 + u * stride;
-                if (e >= n) continue;
-                const int t = e / (heads * 64), r = e - t * heads * 64;
-                const int h = r >> 6, d = r & 63;
-                float* row = acc + (size_t)t * N + h * D + d;
-                __stcg(row, 0.f);
-                __stcg(row + 64, 0.f);
-                const float y0 = lo[u] + b0[u], y1 = hi[u] + b1[u];
-                const float r0 = y0 * cs[u].x - y1 * cs[u].y, r1 = y1 * cs[u].x + y0 * cs[u].y;
-                const int seq = t / p.rows_per_seq, pos = p.pos0 + t % p.rows_per_seq;
-                bf16* dst;
-                if (h < p.n_q_heads)
-                    dst = p.q + ((size_t)t * p.n_q_heads + h) * D;
-                else if (h < p.n_q_heads + p.n_kv_heads)
-                    dst = p.k_cache +
-                          (((size_t)seq * p.n_kv_heads + h - p.n_q_heads) * p.seq_len + pos) * D;
-                else
-                    dst = p.v_cache + (((size_t)seq * p.n_kv_heads + h - p.n_q_heads - p.n_kv_heads) *
-                                           p.seq_len + pos) * D;
-                dst[d] = __float2bfloat16_rn(r0);
-                dst[d + 64] = __float2bfloat16_rn(r1);
+                for (int x = 0; x < 4; ++x) bs[u][x] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            if (rot) {
+                const float4* c4 = reinterpret_cast<const float4*>(
+                    p.rope + (size_t)(p.pos0 + i) * 64 + pc * 8);
+#pragma unroll
+                for (int x = 0; x < 4; ++x) cs[u][x] = __ldg(c4 + x);
+            } else {
+#pragma unroll
+                for (int x = 0; x < 4; ++x) cs[u][x] = make_float4(1.f, 0.f, 1.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = e0 + u * blockDim.x;
+            if (e >= n) continue;
+            const float* lo = reinterpret_cast<const float*>(&v[u][0]);
+            const float* hi = reinterpret_cast<const float*>(&v[u][2]);
+            const float* blo = reinterpret_cast<const float*>(&bs[u][0]);
+            const float* bhi = reinterpret_cast<const float*>(&bs[u][2]);
+            const float* c = reinterpret_cast<const float*>(&cs[u][0]);
+            uint32_t o0[4], o1[4];
+#pragma unroll
+            for (int x = 0; x < 8; x += 2) {
+                float r0[2], r1[2];
+#pragma unroll
+                for (int y = 0; y < 2; ++y) {
+                    const float y0 = lo[x + y] + blo[x + y], y1 = hi[x + y] + bhi[x + y];
+                    const float co = c[2 * (x + y)], si = c[2 * (x + y) + 1];
+                    r0[y] = y0 * co - y1 * si;
+                    r1[y] = y1 * co + y0 * si;
+                }
+                o0[x >> 1] = pack_bf16(r0[0], r0[1]);
+                o1[x >> 1] = pack_bf16(r1[0], r1[1]);
+            }
+            const uint4 w0 = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+            const uint4 w1 = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+            if (e < nq) {
+                const int r = e >> 3, pc = e & 7;
+                uint8_t* dst = sq + r * 128 + ((pc ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4*>(dst) = w0;
+                *reinterpret_cast<uint4*>(dst + QCHUNK) = w1;
+                if (write_q) {
+                    const int i = r / a.hc;
+                    bf16* q = p.q + ((size_t)(bb * a.B + i) * p.n_q_heads + g * a.hc + r % a.hc) *
+                                        128 + pc * 8;
+                    *reinterpret_cast<uint4*>(q) = w0;
+                    *reinterpret_cast<uint4*>(q + 64) = w1;
+                }
+            } else {
+                const int f = e - nq, kind = (f >> 3) & 1, pc = f & 7, row = kv0 + (f >> 4);
+                bf16* dst = (kind ? p.v_cache : p.k_cache) +
+                            (((size_t)bb * p.n_kv_heads + g) * p.seq_len + row) * 128 + pc * 8;
+                *reinterpret_cast<uint4*>(dst) = w0;
+                *reinterpret_cast<uint4*>(dst + 64) = w1;
+                // only this thread reads these sums: zero them for the next call
+                float* src = pro.acc + (size_t)(bb * a.B + row - a.blk0) * N +
+                             (p.n_q_heads + kind * p.n_kv_heads + g) * 128 + pc * 8;
+                const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+                __stcg(reinterpret_cast<float4*>(src), z);
+                __stcg(reinterpret_cast<float4*>(src + 4), z);
+                __stcg(reinterpret_cast<float4*>(src + 64), z);
+                __stcg(reinterpret_cast<float4*>(src + 68), z);
             }
         }
     }
-};
+}
+
+// Zero the q sums of this CTA's query rows (after every split has read them).
+__device__ __forceinline__ void qkv_zero_q(const ProQKV& pro, const AttnArgs& a, int g, int bb) {
+    const int N = (pro.p.n_q_heads + 2 * pro.p.n_kv_heads) * 128;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = threadIdx.x; e < a.rows * 8; e += blockDim.x) {
+        const int r = e >> 3, pc = e & 7;
+        float* src = pro.acc + (size_t)(bb * a.B + r / a.hc) * N + (g * a.hc + r % a.hc) * 128 +
+                     pc * 8;
+        __stcg(reinterpret_cast<float4*>(src), z);
+        __stcg(reinterpret_cast<float4*>(src + 4), z);
+        __stcg(reinterpret_cast<float4*>(src + 64), z);
+        __stcg(reinterpret_cast<float4*>(src + 68), z);
+    }
+}
 
 template <int D, int MT, class Pro>
 __global__ void __launch_bounds__(Att4<D, MT>::THREADS, 1)
@@ -314,10 +392,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     pdl_wait();
     if constexpr (Pro::kActive) {
-        pro.work(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z),
-                 gridDim.x * gridDim.y * gridDim.z);
-        fence_proxy_async_global();                 // the TMA below reads what was written
-        grid_barrier(pro.bar, abort_flag, a.err);
+        static_assert(D == 128, "the q/k/v prologue rotates 128-dim heads");
+        qkv_tile<S::Q_CHUNK>(pro, a, smem + S::OFF_Q, g, bb, k_begin, k_end, split == 0);
+        fence_proxy_async();                        // the MMA reads the Q tile written here
+        fence_proxy_async_global();                 // the TMA reads the block-slot rows
+        __syncthreads();
     }
     pdl_trigger();
     bool ok = *abort_flag == 0;
@@ -325,10 +404,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (warp == S::TMA_WARP) {
         // ---------------------------------------------------------------- TMA
         if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            if constexpr (Pro::kActive) fence_proxy_async_global();
-            const int head0 = g * grp + chunk * a.hc;
-            if (ok) {
+            if constexpr (Pro::kActive) {
+                fence_proxy_async_global();
+                mbar_arrive(bar_q);                 // the Q tile is already in place
+            } else if (ok) {
+                const int head0 = g * grp + chunk * a.hc;
+                prefetch_tmap(&tmQ);
                 mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
                 for (int dc = 0; dc < S::DC; ++dc)
                     tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
@@ -541,21 +622,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         cluster_sync();
         const int rpc = (a.rows + a.n_splits - 1) / a.n_splits;      // rows per CTA
         const int r0 = split * rpc, r1 = min(a.rows, r0 + rpc);
-        const int items = (r1 > r0 ? r1 - r0 : 0) * (D / 4);
+        // item = 8 output columns of one row: two float4 slots per split
+        const int items = (r1 > r0 ? r1 - r0 : 0) * (D / 8);
         const uint32_t part_base = sb + S::OFF_K, red_base = sb + S::OFF_RED;
         for (int it = threadIdx.x; it < items; it += S::THREADS) {
-            const int pr = r0 + it / (D / 4), d4 = it % (D / 4);
+            const int pr = r0 + it / (D / 8), d8 = it % (D / 8);
             const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
             if (i >= a.B || hig >= grp) continue;
             float2 ml[ATT_MAX_SPLITS];
-            float4 v[ATT_MAX_SPLITS];
+            float4 v0[ATT_MAX_SPLITS], v1[ATT_MAX_SPLITS];
             const uint32_t off_ml = red_base + pr * 8;
-            const uint32_t off_o = part_base + (uint32_t)(pr * D + ((d4 ^ (pr & 7)) << 2)) * 4;
+            const uint32_t off_0 =
+                part_base + (uint32_t)(pr * D + (((2 * d8) ^ (pr & 7)) << 2)) * 4;
+            const uint32_t off_1 =
+                part_base + (uint32_t)(pr * D + (((2 * d8 + 1) ^ (pr & 7)) << 2)) * 4;
 #pragma unroll
             for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {    // issue every remote load first
                 if (cc < a.n_splits) {
                     ml[cc] = ld_cluster_f2(cluster_map(off_ml, cc));
-                    v[cc] = ld_cluster_f4(cluster_map(off_o, cc));
+                    v0[cc] = ld_cluster_f4(cluster_map(off_0, cc));
+                    v1[cc] = ld_cluster_f4(cluster_map(off_1, cc));
                 }
             }
             float M = -INFINITY;
@@ -563,27 +649,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc)
                 if (cc < a.n_splits) M = fmaxf(M, ml[cc].x);
             float Lsum = 0.f;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {
                 if (cc < a.n_splits && ml[cc].x != -INFINITY) {
                     const float w = ex2(ml[cc].x - M);
                     Lsum += ml[cc].y * w;
-                    acc.x += v[cc].x * w; acc.y += v[cc].y * w;
-                    acc.z += v[cc].z * w; acc.w += v[cc].w * w;
+                    acc[0] += v0[cc].x * w; acc[1] += v0[cc].y * w;
+                    acc[2] += v0[cc].z * w; acc[3] += v0[cc].w * w;
+                    acc[4] += v1[cc].x * w; acc[5] += v1[cc].y * w;
+                    acc[6] += v1[cc].z * w; acc[7] += v1[cc].w * w;
                 }
             }
             const float inv = 1.f / Lsum;
             const int head = g * grp + hig;
-            bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D + d4 * 4;
-            *reinterpret_cast<uint2*>(dst) =
-                make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
-            if (a.lse && d4 == 0)
+            bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D + d8 * 8;
+            *reinterpret_cast<uint4*>(dst) =
+                make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                           pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+            if (a.lse && d8 == 0)
                 a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
                     (M + log2f(Lsum)) * 0.69314718055994530942f;
         }
         cluster_sync();                    // no CTA leaves while others read its smem
     }
+    // every split of this head has read the q sums (the cluster barrier above,
+    // or, with one split, the barrier after the prologue)
+    if constexpr (Pro::kActive)
+        if (split == 0) qkv_zero_q(pro, a, g, bb);
     tc_fence_before();
     __syncthreads();
     if (warp == S::MMA_WARP) {
@@ -653,39 +746,10 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     if (D == 128)
         return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
                          : run_tc<128, 1>(p, tq, tk, tv, a, hb, hk, st, pro);
-    return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
-                     : run_tc<64, 1>(p, tq, tk, tv, a, hb, hk, st, pro);
-}
-
-// Largest number of clusters of the given size that fit on the device at once
-// (queried once per kernel and size).
-template <int D, int MT>
-int max_active_clusters(int size, int sm_count) {
-    static int cache[ATT_MAX_SPLITS + 1] = {0};
-    if (size < 1 || size > ATT_MAX_SPLITS) return 0;
-    if (cache[size] == 0) {
-        using S = Att4<D, MT>;
-        auto kfn = attn_tc_kernel<D, MT, ProQKV>;
-        int n = 0;
-        if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)S::TOTAL) == cudaSuccess) {
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(size * (sm_count / size));
-            cfg.blockDim = dim3(S::THREADS);
-            cfg.dynamicSmemBytes = S::TOTAL;
-            cudaLaunchAttribute at;
-            at.id = cudaLaunchAttributeClusterDimension;
-            at.val.clusterDim.x = size;
-            at.val.clusterDim.y = 1;
-            at.val.clusterDim.z = 1;
-            cfg.attrs = &at;
-            cfg.numAttrs = 1;
-            if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) n = 0;
-        }
-        cudaGetLastError();
-        cache[size] = n > 0 ? n : -1;
-    }
-    return cache[size] > 0 ? cache[size] : 0;
+    if constexpr (Pro::kActive) return cudaErrorInvalidValue;   // 128-dim heads only
+    else
+        return p.mt == 2 ? run_tc<64, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
+                         : run_tc<64, 1>(p, tq, tk, tv, a, hb, hk, st, pro);
 }
 
 }  // namespace
@@ -699,21 +763,14 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
 
 bool qkv_attention_fusable(const AttnShape& s, int sm_count) {
     if (s.head_dim != 128 || !s.bf16 || s.q_per_kv != 1) return false;
-    const AttnPlan p = attn_tc_plan(s, sm_count);
-    const int ctas = p.n_splits * s.n_kv_heads * p.n_chunks * s.batch;
-    if (ctas > sm_count) return false;               // one CTA per SM: all resident
-    if (p.n_splits == 1) return true;
-    const int clusters = ctas / p.n_splits;
-    const int fit = p.mt == 2 ? max_active_clusters<128, 2>(p.n_splits, sm_count)
-                              : max_active_clusters<128, 1>(p.n_splits, sm_count);
-    return clusters <= fit;
+    // each CTA forms the query tile of one whole GQA group
+    return attn_tc_plan(s, sm_count).n_chunks == 1;
 }
 
-cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, int rows, const EpiQKV& pq,
-                                      unsigned* bar, void* out, int sm_count, int* err,
-                                      cudaStream_t st) {
+cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQKV& pq, void* out,
+                                      int sm_count, int* err, cudaStream_t st) {
     return launch_attn(s, pq.q, pq.k_cache, pq.v_cache, out, nullptr, sm_count, err, st,
-                       ProQKV{bar, acc, rows, pq});
+                       ProQKV{acc, pq});
 }
 
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,

@@ -29,14 +29,14 @@ cudaError_t launch_attention_bf16(const AttnShape& s, const void* q, const void*
 
 // Block-slot projection fused with DualCache attention: the split-K sums of
 // the q/k/v projection (acc, rows x N f32, zero-kept) are finished (bias,
-// RoPE, q and the cache block slot written, zeros restored) by the CTAs of the
-// attention kernel before a grid barrier, then the attention runs. Only when
-// qkv_attention_fusable(s): every CTA of the attention grid fits on the device
-// at once (bf16, head_dim 128, one query block per sequence).
+// RoPE, zeros restored) by the CTAs of the attention kernel: each forms its
+// query tile in shared memory (and split 0 writes q) and writes the block-slot
+// K/V rows of its own key range, then the attention runs. Only when
+// qkv_attention_fusable(s): bf16, head_dim 128, one query block per sequence
+// and the whole GQA group of a kv head in one CTA.
 bool qkv_attention_fusable(const AttnShape& s, int sm_count);
-cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, int rows, const EpiQKV& pq,
-                                      unsigned* bar, void* out, int sm_count, int* err,
-                                      cudaStream_t st);
+cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQKV& pq, void* out,
+                                      int sm_count, int* err, cudaStream_t st);
 
 // Full bidirectional attention of every position of every sequence (the
 // refresh forward): q, out [b, L, Hq, d] bf16; caches [b, Hkv, L, d].

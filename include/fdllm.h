@@ -313,12 +313,13 @@ FDL_API int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* desc, const voi
  *   x       [rows, hidden] bf16: written when norm_w is given, else the input
  *   out     [batch, rows_per_seq, n_q_heads, 128] bf16 (written)
  *   q_out, k_cache, v_cache, w, bias, rope as for fdl_qkv_rope_store.
- * When the shapes allow (few rows, split-K projection, an attention grid that
- * fits on the device at once) the RMSNorm runs in the projection's kernel and
- * the projection's epilogue (bias, RoPE, q and block-slot store) in the
- * attention kernel, each behind a grid-wide barrier, instead of in kernels
- * of their own. Errors: as fdl_qkv_rope_store, plus FDL_EINVAL for the row
- * layout or the norm arguments. */
+ * When the shapes allow (few rows, split-K projection, a whole GQA group of
+ * query heads per attention CTA) the RMSNorm runs in the projection's kernel
+ * (behind a grid-wide barrier) and the projection's epilogue (bias, RoPE, q
+ * and block-slot store) in the attention kernel's CTAs, each forming its own
+ * query tile and block-slot rows, instead of in kernels of their own.
+ * Errors: as fdl_qkv_rope_store, plus FDL_EINVAL for the row layout or the
+ * norm arguments. */
 FDL_API int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* desc, const float* h,
                               const float* norm_w, float eps, void* x, const void* w,
                               const float* bias, const float* rope, void* q_out, void* k_cache,

@@ -140,6 +140,9 @@ def test_ffn_block(ctx, M, D, F, norm):
     (1, 8, 8, False, 32, 96, 256, 1024, True),        # fused, several splits per head
     (2, 28, 4, True, 32, 512, 1024, 3584, True),      # GQA 7:1 with bias (Dream / Qwen2.5)
     (2, 4, 2, True, 32, 64, 160, 256, True),          # no K split: separate calls
+    (1, 8, 8, False, 32, 48, 256, 1024, False),       # block slot across two splits
+    (1, 8, 4, True, 16, 192, 224, 1024, True),        # block in the ragged last tile
+    (1, 32, 2, False, 32, 64, 256, 1024, False),      # GQA 16:1, two query chunks: separate calls
 ])
 def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D, norm):
     """Norm + block-slot projection + DualCache attention in one call equals
