@@ -249,6 +249,8 @@ def run_gpu(args):
                        "steps_by_kind": kinds, "tokens_decoded": toks,
                        "host_ms_per_step": {k: (statistics.median(v) if v else None)
                                             for k, v in step_ms.items()},
+                       "host_ms_per_step_mean": {k: (statistics.fmean(v) if v else None)
+                                                 for k, v in step_ms.items()},
                        "weights_gb": round(w.nbytes() / 1e9, 2),
                        "graph_capture_s": round(capture_s, 2),
                        "l2": "no flush: 16 GB of weights (> 126 MB L2) are streamed every step"},

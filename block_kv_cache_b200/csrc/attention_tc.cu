@@ -74,9 +74,7 @@ namespace {
 
 template <int D, int MT>
 struct Att4 {
-    // K/V ring depth: the ring turns over once per (HBM latency + one tile's
-    // S, softmax and PV chain), so the period of a tile is that over STAGES
-    static constexpr int STAGES = MT == 1 ? 5 : 2;
+    static constexpr int STAGES = MT == 1 ? 3 : 2;
     static constexpr int THREADS = 32 * (4 * MT + 2);
     static constexpr int TMA_WARP = 4 * MT, MMA_WARP = 4 * MT + 1;
     static constexpr int DC = D / 64;
@@ -160,11 +158,13 @@ struct AttNoPro {
 // The epilogue of a split-K block-slot projection (bias, RoPE, q and the K/V
 // block slot), done by the attention CTAs that consume it, with no kernel of
 // its own and no wait on another CTA. Each CTA forms its own query tile in
-// shared memory straight from the f32 sums and writes the block-slot K/V rows
-// that fall in its own key range (only it reads them); the sums it read are
-// zeroed again (the q sums, which every split of a head reads, by split 0
-// once the cluster has merged). One query chunk per kv head (hc == grp) and
-// one query block per sequence.
+// shared memory straight from the f32 sums, then its first MMA can go; the
+// block-slot K/V rows that fall in its own key range (only it reads them) are
+// written by its idle softmax warps while the others run, and the tiles that
+// hold them come last in its tile order. The sums read are zeroed again (the
+// q sums, which every split of a head reads, by split 0 once the cluster has
+// merged). One query chunk per kv head (hc == grp), one query block per
+// sequence.
 struct ProQKV {
     static constexpr bool kActive = true;
     float* acc;              // [M, N] sums, N = (Hq + 2 Hkv) * 128
@@ -173,20 +173,20 @@ struct ProQKV {
 
 // Item = 8 consecutive dimensions d of one row and their rotation partners
 // d + 64 (RoPE over 128-dimensional heads). Loads of a batch first, then math.
+// Items [0, nq) are the query tile's, the rest block-slot K/V rows from kv0 on;
+// thread tid of nthreads takes every nthreads-th item.
 template <int QCHUNK>
-__device__ __forceinline__ void qkv_tile(const ProQKV& pro, const AttnArgs& a, uint8_t* sq,
-                                         int g, int bb, int k_begin, int k_end, bool write_q) {
+__device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, uint8_t* sq,
+                                          int g, int bb, int kv0, int nq, int n, int tid,
+                                          int nthreads, bool write_q) {
     constexpr int U = 2;
     const EpiQKV& p = pro.p;
     const int N = (p.n_q_heads + 2 * p.n_kv_heads) * 128;
-    const int nq = a.rows * 8;
-    const int kv0 = max(a.blk0, k_begin), kv1 = min(a.blk1, k_end);
-    const int n = nq + (kv1 > kv0 ? (kv1 - kv0) * 16 : 0);
-    for (int e0 = threadIdx.x; e0 < n; e0 += U * blockDim.x) {
+    for (int e0 = tid; e0 < n; e0 += U * nthreads) {
         float4 v[U][4], bs[U][4], cs[U][4];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int e = e0 + u * blockDim.x;
+            const int e = e0 + u * nthreads;
             if (e >= n) continue;
             int i, col, pc;
             bool rot = true;
@@ -229,7 +229,7 @@ __device__ __forceinline__ void qkv_tile(const ProQKV& pro, const AttnArgs& a, u
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int e = e0 + u * blockDim.x;
+            const int e = e0 + u * nthreads;
             if (e >= n) continue;
             const float* lo = reinterpret_cast<const float*>(&v[u][0]);
             const float* hi = reinterpret_cast<const float*>(&v[u][2]);
@@ -319,7 +319,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto s_free = [&](int b) { return smem_u32(bars + 3 + 3 * STAGES + b); };
     auto p_full = [&](int b) { return smem_u32(bars + 5 + 3 * STAGES + b); };
     auto o_done = [&](int b) { return smem_u32(bars + 7 + 3 * STAGES + b); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 3 * STAGES);
+    const uint32_t bar_kv = smem_u32(bars + 9 + 3 * STAGES);   // block-slot rows written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 3 * STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int split = blockIdx.x;                    // == rank in the cluster
@@ -334,6 +335,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // softmax warps with at least one real row (a warp covers 32 packed rows)
     const int live_warps = (a.rows + 31) / 32;
     const int live_threads = live_warps * 32;
+    // warps that write the block-slot K/V rows: the idle softmax warps, else all
+    const int kv_w0 = live_warps < 4 * MT ? live_warps : 0;
+    // Tile order: with the fused prologue the tiles holding block-slot rows of
+    // this split come last (a rotation; the online softmax is order-free).
+    int rot = 0;
+    if constexpr (Pro::kActive) {
+        if (a.blk0 < k_end && a.blk1 > k_begin)
+            rot = ((min(a.blk1, k_end) - 1 - k_begin) / KT + 1) % nt;
+    }
+    auto tile_of = [&](int t) { const int u = t + rot; return u >= nt ? u - nt : u; };
+    auto in_block = [&](int tile) {
+        const int k0 = k_begin + tile * KT;
+        return k0 < a.blk1 && k0 + KT > a.blk0;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -342,6 +357,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             mbar_init(v_full(s), 1);
             mbar_init(kv_empty(s), 1);
         }
+        mbar_init(bar_kv, (4 * MT - kv_w0) * 32);
         for (int b2 = 0; b2 < 2; ++b2) {
             mbar_init(s_full(b2), 1);
             mbar_init(s_free(b2), live_threads);
@@ -382,9 +398,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             for (int t = 0; t < nt && t < STAGES; ++t) {
-                const int k0 = k_begin + t * KT, k1 = k0 + KT;
-                if (k1 <= a.L && (k1 <= a.blk0 || k0 >= a.blk1)) {
-                    load_kv(t, t);
+                const int tile = tile_of(t);
+                if (k_begin + (tile + 1) * KT <= a.L && !in_block(tile)) {
+                    load_kv(tile, t);
                     early |= 1u << t;
                 }
             }
@@ -393,9 +409,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     pdl_wait();
     if constexpr (Pro::kActive) {
         static_assert(D == 128, "the q/k/v prologue rotates 128-dim heads");
-        qkv_tile<S::Q_CHUNK>(pro, a, smem + S::OFF_Q, g, bb, k_begin, k_end, split == 0);
+        qkv_items<S::Q_CHUNK>(pro, a, smem + S::OFF_Q, g, bb, 0, a.rows * 8, a.rows * 8,
+                              threadIdx.x, blockDim.x, split == 0);
         fence_proxy_async();                        // the MMA reads the Q tile written here
-        fence_proxy_async_global();                 // the TMA reads the block-slot rows
         __syncthreads();
     }
     pdl_trigger();
@@ -416,12 +432,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                 bb * a.B);
             }
             int t = 0;
+            bool kv_rows = !Pro::kActive;           // block-slot rows in place
             for (; ok && t < nt; ++t) {
-                const int st = t % STAGES;
+                const int st = t % STAGES, tile = tile_of(t);
                 if (t < STAGES && ((early >> t) & 1u)) continue;
+                if (!kv_rows && in_block(tile)) {
+                    if (!(ok = mbar_wait(bar_kv, 0, abort_flag, a.err))) break;
+                    fence_proxy_async_global();
+                    kv_rows = true;
+                }
                 if (!(ok = mbar_wait(kv_empty(st), ((t / STAGES) & 1) ^ 1, abort_flag, a.err)))
                     break;
-                load_kv(t, st);
+                load_kv(tile, st);
             }
             // tail: every stage handed out has been released again
             for (int u = t; ok && u < t + STAGES; ++u)
@@ -483,135 +505,152 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 }
             }
         }
-    } else if (warp < live_warps) {
-        // ------------------------------------------------------------ softmax
-        const int q = warp & 3;                          // TMEM lane quarter
-        const int m = warp >> 2;                         // 128-row tile
-        const int r = q * 32 + lane;                     // row within the tile
-        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        float m_run = -INFINITY, l_run = 0.f;            // running max (log2 units), sum
-        for (int t = 0; t < nt; ++t) {
-            const int b2 = t & 1;
-            if (!(ok = mbar_wait_warp(s_full(b2), (t >> 1) & 1, abort_flag, a.err))) break;
-            tc_fence_after();
-            float sr[KT];
-#pragma unroll
-            for (int j = 0; j < KT; j += 16)
-                tmem_ld16(tmem + lane_base + S::TMEM_S + (b2 * MT + m) * KT + j,
-                          reinterpret_cast<uint32_t*>(sr) + j);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(s_free(b2));
-
-            const int kbase = k_begin + t * KT;          // global key of sr[0]
-            if (kbase + KT > k_end) {                    // ragged last tile
-#pragma unroll
-                for (int j = 0; j < KT; ++j)
-                    if (kbase + j >= k_end) sr[j] = -INFINITY;
+    } else {
+        if constexpr (Pro::kActive) {
+            if (warp >= kv_w0) {
+                // the block-slot K/V rows of this split's key range
+                const int kv0 = max(a.blk0, k_begin), kv1 = min(a.blk1, k_end);
+                qkv_items<S::Q_CHUNK>(pro, a, smem + S::OFF_Q, g, bb, kv0, 0,
+                                      kv1 > kv0 ? (kv1 - kv0) * 16 : 0,
+                                      threadIdx.x - kv_w0 * 32, (4 * MT - kv_w0) * 32, false);
+                fence_proxy_async_global();         // the TMA reads these rows
+                mbar_arrive(bar_kv);
             }
-            float mx = sr[0];
-#pragma unroll
-            for (int j = 1; j < KT; ++j) mx = fmaxf(mx, sr[j]);
-            mx *= a.scale_log2;                          // scale > 0 commutes with max
-            float alpha = 1.f;
-            bool rescale = false;
-            if (mx > m_run + 8.f || m_run == -INFINITY) {
-                const float mn = fmaxf(m_run, mx);
-                if (mn != -INFINITY) {
-                    alpha = ex2(m_run - mn);             // 0 on the first update
-                    rescale = m_run != -INFINITY;
-                    m_run = mn;
-                }
-            }
-            const float nmr = m_run == -INFINITY ? 0.f : -m_run;
-            float l = 0.f;
-            uint32_t pk[KT / 2];
-#pragma unroll
-            for (int j = 0; j < KT; j += 2) {
-                const float p0 = ex2(fmaf(sr[j], a.scale_log2, nmr));
-                const float p1 = ex2(fmaf(sr[j + 1], a.scale_log2, nmr));
-                l += p0 + p1;
-                pk[j >> 1] = pack_bf16(p0, p1);
-            }
-            l_run = l_run * alpha + l;
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O holds P V up to tile t-1: wait for PV(t-1), then scale it
-                if (t > 0) {
-                    if (!(ok = mbar_wait_warp(o_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag,
-                                              a.err)))
-                        break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int d0 = 0; d0 < D; d0 += 16) {
-                        uint32_t o[16];
-                        const uint32_t ta = tmem + lane_base + S::TMEM_O + m * D + d0;
-                        tmem_ld16(ta, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 16; ++x)
-                            o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-                        tmem_st16(ta, o);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            // P buffer b2 is free once PV(t-2) is done
-            if (!(ok = mbar_wait_warp(o_done(b2), ((t >> 1) & 1) ^ 1, abort_flag, a.err))) break;
-            uint8_t* prow = smem + S::OFF_P + (b2 * MT + m) * S::P_TILE + r * 128;
-#pragma unroll
-            for (int piece = 0; piece < 8; ++piece)      // 8 keys per 16-byte piece
-                *reinterpret_cast<uint4*>(prow + ((piece ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * piece], pk[4 * piece + 1], pk[4 * piece + 2],
-                               pk[4 * piece + 3]);
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(p_full(b2));
         }
-        // ----------------------------------------------------------- epilogue
-        if (ok)
-            ok = mbar_wait_warp(o_done((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, a.err);
-        // the live softmax warps agree on running the epilogue; every wait
-        // above is bounded, so all of them get here
-        named_sync(1, live_threads);
-        ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
-        if (ok) {
-            tc_fence_after();
-            float o[D];
+        if (warp < live_warps) {
+            // ------------------------------------------------------------ softmax
+            const int q = warp & 3;                          // TMEM lane quarter
+            const int m = warp >> 2;                         // 128-row tile
+            const int r = q * 32 + lane;                     // row within the tile
+            const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+            float m_run = -INFINITY, l_run = 0.f;            // running max (log2 units), sum
+            for (int t = 0; t < nt; ++t) {
+                const int b2 = t & 1;
+                if (!(ok = mbar_wait_warp(s_full(b2), (t >> 1) & 1, abort_flag, a.err))) break;
+                tc_fence_after();
+                float sr[KT];
 #pragma unroll
-            for (int d0 = 0; d0 < D; d0 += 16)
-                tmem_ld16(tmem + lane_base + S::TMEM_O + m * D + d0,
-                          reinterpret_cast<uint32_t*>(o) + d0);
-            tmem_wait_ld();
-            const int pr = m * 128 + r;                  // packed row
-            const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
-            const bool row_ok = pr < a.rows;
-            const bool valid = row_ok && i < a.B && hig < grp;
-            if (a.n_splits == 1) {
-                if (valid) {
-                    const int head = g * grp + hig;
-                    const float inv = 1.f / l_run;
-                    bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D;
+                for (int j = 0; j < KT; j += 16)
+                    tmem_ld16(tmem + lane_base + S::TMEM_S + (b2 * MT + m) * KT + j,
+                              reinterpret_cast<uint32_t*>(sr) + j);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(s_free(b2));
+
+                const int kbase = k_begin + tile_of(t) * KT; // global key of sr[0]
+                if (kbase + KT > k_end) {                    // ragged last tile
 #pragma unroll
-                    for (int d = 0; d < D; d += 8)
-                        *reinterpret_cast<uint4*>(dst + d) = make_uint4(
-                            pack_bf16(o[d] * inv, o[d + 1] * inv),
-                            pack_bf16(o[d + 2] * inv, o[d + 3] * inv),
-                            pack_bf16(o[d + 4] * inv, o[d + 5] * inv),
-                            pack_bf16(o[d + 6] * inv, o[d + 7] * inv));
-                    if (a.lse)
-                        a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
-                            (m_run + log2f(l_run)) * 0.69314718055994530942f;
+                    for (int j = 0; j < KT; ++j)
+                        if (kbase + j >= k_end) sr[j] = -INFINITY;
                 }
-            } else if (row_ok) {
-                // publish this CTA's partial for the cluster merge
-                float* part = reinterpret_cast<float*>(smem + S::OFF_K) + (size_t)pr * D;
+                float m8[8];                                 // 8 independent max chains
 #pragma unroll
-                for (int d4 = 0; d4 < D / 4; ++d4)
-                    *reinterpret_cast<float4*>(part + ((d4 ^ (pr & 7)) << 2)) =
-                        make_float4(o[4 * d4], o[4 * d4 + 1], o[4 * d4 + 2], o[4 * d4 + 3]);
-                float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
-                red[2 * pr] = m_run;
-                red[2 * pr + 1] = l_run;
+                for (int j = 0; j < 8; ++j) m8[j] = sr[j];
+#pragma unroll
+                for (int j = 8; j < KT; ++j) m8[j & 7] = fmaxf(m8[j & 7], sr[j]);
+                float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                mx *= a.scale_log2;                          // scale > 0 commutes with max
+                float alpha = 1.f;
+                bool rescale = false;
+                if (mx > m_run + 8.f || m_run == -INFINITY) {
+                    const float mn = fmaxf(m_run, mx);
+                    if (mn != -INFINITY) {
+                        alpha = ex2(m_run - mn);             // 0 on the first update
+                        rescale = m_run != -INFINITY;
+                        m_run = mn;
+                    }
+                }
+                const float nmr = m_run == -INFINITY ? 0.f : -m_run;
+                float l = 0.f;
+                uint32_t pk[KT / 2];
+#pragma unroll
+                for (int j = 0; j < KT; j += 2) {
+                    const float p0 = ex2(fmaf(sr[j], a.scale_log2, nmr));
+                    const float p1 = ex2(fmaf(sr[j + 1], a.scale_log2, nmr));
+                    l += p0 + p1;
+                    pk[j >> 1] = pack_bf16(p0, p1);
+                }
+                l_run = l_run * alpha + l;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O holds P V up to tile t-1: wait for PV(t-1), then scale it
+                    if (t > 0) {
+                        if (!(ok = mbar_wait_warp(o_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag,
+                                                  a.err)))
+                            break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int d0 = 0; d0 < D; d0 += 16) {
+                            uint32_t o[16];
+                            const uint32_t ta = tmem + lane_base + S::TMEM_O + m * D + d0;
+                            tmem_ld16(ta, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 16; ++x)
+                                o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                            tmem_st16(ta, o);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // P buffer b2 is free once PV(t-2) is done
+                if (!(ok = mbar_wait_warp(o_done(b2), ((t >> 1) & 1) ^ 1, abort_flag, a.err))) break;
+                uint8_t* prow = smem + S::OFF_P + (b2 * MT + m) * S::P_TILE + r * 128;
+#pragma unroll
+                for (int piece = 0; piece < 8; ++piece)      // 8 keys per 16-byte piece
+                    *reinterpret_cast<uint4*>(prow + ((piece ^ (r & 7)) << 4)) =
+                        make_uint4(pk[4 * piece], pk[4 * piece + 1], pk[4 * piece + 2],
+                                   pk[4 * piece + 3]);
+                fence_proxy_async();
+                tc_fence_before();
+                mbar_arrive(p_full(b2));
+            }
+            // ----------------------------------------------------------- epilogue
+            if (ok)
+                ok = mbar_wait_warp(o_done((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, a.err);
+            // the live softmax warps agree on running the epilogue; every wait
+            // above is bounded, so all of them get here
+            named_sync(1, live_threads);
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
+            if (ok) {
+                tc_fence_after();
+                float o[D];
+#pragma unroll
+                for (int d0 = 0; d0 < D; d0 += 16)
+                    tmem_ld16(tmem + lane_base + S::TMEM_O + m * D + d0,
+                              reinterpret_cast<uint32_t*>(o) + d0);
+                tmem_wait_ld();
+                const int pr = m * 128 + r;                  // packed row
+                const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
+                const bool row_ok = pr < a.rows;
+                const bool valid = row_ok && i < a.B && hig < grp;
+                if (a.n_splits == 1) {
+                    if (valid) {
+                        const int head = g * grp + hig;
+                        const float inv = 1.f / l_run;
+                        bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D;
+#pragma unroll
+                        for (int d = 0; d < D; d += 8)
+                            *reinterpret_cast<uint4*>(dst + d) = make_uint4(
+                                pack_bf16(o[d] * inv, o[d + 1] * inv),
+                                pack_bf16(o[d + 2] * inv, o[d + 3] * inv),
+                                pack_bf16(o[d + 4] * inv, o[d + 5] * inv),
+                                pack_bf16(o[d + 6] * inv, o[d + 7] * inv));
+                        if (a.lse)
+                            a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
+                                (m_run + log2f(l_run)) * 0.69314718055994530942f;
+                    }
+                } else if (row_ok) {
+                    // publish this CTA's partial for the cluster merge
+                    float* part = reinterpret_cast<float*>(smem + S::OFF_K) + (size_t)pr * D;
+#pragma unroll
+                    for (int d4 = 0; d4 < D / 4; ++d4)
+                        *reinterpret_cast<float4*>(part + ((d4 ^ (pr & 7)) << 2)) =
+                            make_float4(o[4 * d4], o[4 * d4 + 1], o[4 * d4 + 2], o[4 * d4 + 3]);
+                    float* red = reinterpret_cast<float*>(smem + S::OFF_RED);
+                    red[2 * pr] = m_run;
+                    red[2 * pr + 1] = l_run;
+                }
             }
         }
     }
