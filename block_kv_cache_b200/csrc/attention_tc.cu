@@ -421,7 +421,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         // ---------------------------------------------------------------- TMA
         if (lane == 0) {
             if constexpr (Pro::kActive) {
-                fence_proxy_async_global();
                 mbar_arrive(bar_q);                 // the Q tile is already in place
             } else if (ok) {
                 const int head0 = g * grp + chunk * a.hc;

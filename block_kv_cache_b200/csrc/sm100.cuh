@@ -98,39 +98,56 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
 
 // Barrier over every CTA of the grid. Only for grids whose CTAs are all
 // resident at once (persistent grids of at most one CTA per SM, launched when
-// nothing else can hold an SM indefinitely). bar[0] counts arrivals and bar[1]
-// is the generation; both start at zero and are left consistent for the next
-// use (the last CTA to arrive resets the count before it releases the
-// others). Bounded: a CTA that waits longer than the timeout raises *abort,
-// records DEV_TIMEOUT and returns false; afterwards the two words are no
-// longer consistent, so the caller's context has to be recreated.
+// nothing else can hold an SM indefinitely). The two words at bar hold one
+// 64-bit arrival counter (8-byte aligned, zero at first use) that only grows:
+// one barrier adds exactly kBarrierQuantum to it whatever the grid size (CTA 0
+// adds the quantum less the other CTAs' ones), so a CTA that arrives at count
+// c leaves once the count reaches the next multiple of the quantum above c.
+// One release add and acquire polls: no reset, no second word, no full
+// fences. Bounded: a CTA that waits longer than the timeout raises *abort,
+// records DEV_TIMEOUT and returns false; afterwards the counter is no longer
+// at a multiple of the quantum, so the caller's context has to be recreated.
+constexpr unsigned long long kBarrierQuantum = 1ull << 20;   // > any grid size
+
+__device__ __forceinline__ unsigned long long atom_add_release_gpu(unsigned long long* p,
+                                                                   unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.release.gpu.global.add.u64 %0, [%1], %2;"
+                 : "=l"(old)
+                 : "l"(p), "l"(v)
+                 : "memory");
+    return old;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ bool grid_barrier(unsigned* bar, volatile int* abort, int* err) {
-    __syncthreads();
+    __syncthreads();                                 // the CTA's writes precede the release
     if (threadIdx.x == 0) {
-        volatile unsigned* gen = bar + 1;
-        const unsigned g = *gen;                     // before arriving
-        __threadfence();
-        if (atomicAdd(bar, 1u) == gridDim.x * gridDim.y * gridDim.z - 1) {
-            atomicExch(bar, 0u);
-            __threadfence();
-            atomicAdd(bar + 1, 1u);
-        } else {
-            uint32_t n = 0;
-            uint64_t t0 = 0;
-            while (*gen == g) {
-                if ((++n & 63u) == 0) {
-                    const uint64_t now = globaltimer();
-                    if (t0 == 0) {
-                        t0 = now;
-                    } else if (now - t0 > kWaitTimeoutNs) {
-                        *abort = 1;
-                        record_error(err, DEV_TIMEOUT);
-                        break;
-                    }
+        unsigned long long* cnt = reinterpret_cast<unsigned long long*>(bar);
+        const unsigned long long nb = (unsigned long long)gridDim.x * gridDim.y * gridDim.z;
+        const bool first = (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
+        const unsigned long long old =
+            atom_add_release_gpu(cnt, first ? kBarrierQuantum - (nb - 1) : 1ull);
+        const unsigned long long target = (old / kBarrierQuantum + 1) * kBarrierQuantum;
+        uint32_t n = 0;
+        uint64_t t0 = 0;
+        while (ld_acquire_gpu(cnt) < target) {
+            if ((++n & 63u) == 0) {
+                const uint64_t now = globaltimer();
+                if (t0 == 0) {
+                    t0 = now;
+                } else if (now - t0 > kWaitTimeoutNs) {
+                    *abort = 1;
+                    record_error(err, DEV_TIMEOUT);
+                    break;
                 }
             }
         }
-        __threadfence();
     }
     __syncthreads();
     return *abort == 0;
