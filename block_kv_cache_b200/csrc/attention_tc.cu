@@ -24,9 +24,13 @@
 //       the log2 domain (scale*log2 e folded into one FFMA); P(t) as bf16 into
 //       one of two shared-memory buffers; O rescaled in TMEM only when the
 //       running max grows by more than 8 (a factor 2^8)
-//   TMA warp (1 thread): Q once, then K and V tiles
+//   TMA warp (1 thread): Q once, then K and V tiles; a K stage is released
+//       as soon as S(t) is done, a V stage once PV(t) is, so the next K tile
+//       does not wait for the softmax
 //   MMA warp (1 thread): TMEM owner; tcgen05.mma S(t) = Q K(t)^T into one of
-//       two S buffers, then O += P(t) V(t) with V as an MN-major operand
+//       two S buffers and O += P(u) V(u) with V as an MN-major operand, each
+//       issued as soon as its operands are there (non-blocking barrier polls),
+//       so a PV never queues behind the wait for the next K tile
 //
 // Roofline: HBM. Algorithmic bytes per call = K and V once (2*b*Hkv*L*d*2)
 // + q and out (2*b*B*Hq*d*2).
@@ -314,13 +318,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t bar_q = smem_u32(bars + 0);
     auto k_full = [&](int s) { return smem_u32(bars + 1 + s); };
     auto v_full = [&](int s) { return smem_u32(bars + 1 + STAGES + s); };
-    auto kv_empty = [&](int s) { return smem_u32(bars + 1 + 2 * STAGES + s); };
-    auto s_full = [&](int b) { return smem_u32(bars + 1 + 3 * STAGES + b); };
-    auto s_free = [&](int b) { return smem_u32(bars + 3 + 3 * STAGES + b); };
-    auto p_full = [&](int b) { return smem_u32(bars + 5 + 3 * STAGES + b); };
-    auto o_done = [&](int b) { return smem_u32(bars + 7 + 3 * STAGES + b); };
-    const uint32_t bar_kv = smem_u32(bars + 9 + 3 * STAGES);   // block-slot rows written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 3 * STAGES);
+    // K and V stages are released separately: K once S(t) is done, V once PV(t) is
+    auto k_empty = [&](int s) { return smem_u32(bars + 1 + 2 * STAGES + s); };
+    auto v_empty = [&](int s) { return smem_u32(bars + 1 + 3 * STAGES + s); };
+    auto s_full = [&](int b) { return smem_u32(bars + 1 + 4 * STAGES + b); };
+    auto s_free = [&](int b) { return smem_u32(bars + 3 + 4 * STAGES + b); };
+    auto p_full = [&](int b) { return smem_u32(bars + 5 + 4 * STAGES + b); };
+    auto o_done = [&](int b) { return smem_u32(bars + 7 + 4 * STAGES + b); };
+    const uint32_t bar_kv = smem_u32(bars + 9 + 4 * STAGES);   // block-slot rows written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 4 * STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int split = blockIdx.x;                    // == rank in the cluster
@@ -355,7 +361,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(k_full(s), 1);
             mbar_init(v_full(s), 1);
-            mbar_init(kv_empty(s), 1);
+            mbar_init(k_empty(s), 1);
+            mbar_init(v_empty(s), 1);
         }
         mbar_init(bar_kv, (4 * MT - kv_w0) * 32);
         for (int b2 = 0; b2 < 2; ++b2) {
@@ -374,14 +381,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t tmem = *tmem_slot;
     const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
     const uint64_t kv_policy = l2_evict_first();
-    auto load_kv = [&](int t, int st) {
-        // one copy per tile and operand: all D columns as DC sub-tiles
+    // one copy per tile and operand: all D columns as DC sub-tiles
+    auto load_k = [&](int t, int st) {
         mbar_arrive_expect_tx(k_full(st), S::KV_TILE);
         if (a.q_per_kv == 1)   // one query block: every K/V byte is read once
             tma_load_3d_hint(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0,
                              krow0 + t * KT, 0, kv_policy);
         else
             tma_load_3d(sb + S::OFF_K + st * S::KV_TILE, &tmK, k_full(st), 0, krow0 + t * KT, 0);
+    };
+    auto load_v = [&](int t, int st) {
         mbar_arrive_expect_tx(v_full(st), S::KV_TILE);
         if (a.q_per_kv == 1)
             tma_load_3d_hint(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0,
@@ -400,7 +409,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             for (int t = 0; t < nt && t < STAGES; ++t) {
                 const int tile = tile_of(t);
                 if (k_begin + (tile + 1) * KT <= a.L && !in_block(tile)) {
-                    load_kv(tile, t);
+                    load_k(tile, t);
+                    load_v(tile, t);
                     early |= 1u << t;
                 }
             }
@@ -420,9 +430,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (warp == S::TMA_WARP) {
         // ---------------------------------------------------------------- TMA
         if (lane == 0) {
+            bool q_issued = false;
             if constexpr (Pro::kActive) {
                 mbar_arrive(bar_q);                 // the Q tile is already in place
             } else if (ok) {
+                q_issued = true;
                 const int head0 = g * grp + chunk * a.hc;
                 prefetch_tmap(&tmQ);
                 mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
@@ -430,31 +442,71 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                     tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,
                                 bb * a.B);
             }
-            int t = 0;
+            // K and V tiles are requested as their stages come free, in tile
+            // order each; whichever can go first does (non-blocking polls)
+            int nk = 0, nv = 0;
             bool kv_rows = !Pro::kActive;           // block-slot rows in place
-            for (; ok && t < nt; ++t) {
-                const int st = t % STAGES, tile = tile_of(t);
-                if (t < STAGES && ((early >> t) & 1u)) continue;
-                if (!kv_rows && in_block(tile)) {
-                    if (!(ok = mbar_wait(bar_kv, 0, abort_flag, a.err))) break;
-                    fence_proxy_async_global();
-                    kv_rows = true;
+            PollBudget pb;
+            while (ok && (nk < nt || nv < nt)) {
+                bool moved = false;
+                if (nk < nt) {
+                    const int st = nk % STAGES, tile = tile_of(nk);
+                    if (nk < STAGES && ((early >> nk) & 1u)) {
+                        ++nk;
+                        moved = true;
+                    } else {
+                        if (!kv_rows && in_block(tile) && mbar_test(bar_kv, 0)) {
+                            fence_proxy_async_global();
+                            kv_rows = true;
+                        }
+                        if ((kv_rows || !in_block(tile)) &&
+                            mbar_test(k_empty(st), ((nk / STAGES) & 1) ^ 1)) {
+                            load_k(tile, st);
+                            ++nk;
+                            moved = true;
+                        }
+                    }
                 }
-                if (!(ok = mbar_wait(kv_empty(st), ((t / STAGES) & 1) ^ 1, abort_flag, a.err)))
-                    break;
-                load_kv(tile, st);
+                if (nv < nk) {
+                    const int st = nv % STAGES, tile = tile_of(nv);
+                    if (nv < STAGES && ((early >> nv) & 1u)) {
+                        ++nv;
+                        moved = true;
+                    } else if (mbar_test(v_empty(st), ((nv / STAGES) & 1) ^ 1)) {
+                        load_v(tile, st);
+                        ++nv;
+                        moved = true;
+                    }
+                }
+                if (moved) {
+                    pb.reset();
+                } else {
+                    __nanosleep(32);                // leave issue slots to the softmax warps
+                    ok = pb.idle(abort_flag, a.err);
+                }
             }
             // tail: every stage handed out has been released again
-            for (int u = t; ok && u < t + STAGES; ++u)
-                ok = mbar_wait(kv_empty(u % STAGES), ((u / STAGES) & 1) ^ 1, abort_flag, a.err);
-            if (!ok && early) {
-                // gave up: the tiles requested early must land before the CTA exits
+            for (int u = nt; ok && u < nt + STAGES; ++u) {
+                ok = mbar_wait(k_empty(u % STAGES), ((u / STAGES) & 1) ^ 1, abort_flag, a.err);
+                if (ok)
+                    ok = mbar_wait(v_empty(u % STAGES), ((u / STAGES) & 1) ^ 1, abort_flag,
+                                   a.err);
+            }
+            if (!ok) {
+                // gave up: every copy requested into this CTA's shared memory must
+                // land before the CTA exits (the last STAGES of each operand)
                 volatile int no_abort = 0;
-                for (int u = 0; u < STAGES; ++u)
-                    if ((early >> u) & 1u) {
-                        mbar_wait(k_full(u), 0, &no_abort, a.err);
+                for (int u = (nk > STAGES ? nk - STAGES : 0); u < nk; ++u)
+                    mbar_wait(k_full(u % STAGES), (u / STAGES) & 1, &no_abort, a.err);
+                for (int u = (nv > STAGES ? nv - STAGES : 0); u < nv; ++u)
+                    mbar_wait(v_full(u % STAGES), (u / STAGES) & 1, &no_abort, a.err);
+                for (int u = nv; u < STAGES && u < nt; ++u)   // early V not yet counted
+                    if ((early >> u) & 1u)
                         mbar_wait(v_full(u), 0, &no_abort, a.err);
-                    }
+                for (int u = nk; u < STAGES && u < nt; ++u)
+                    if ((early >> u) & 1u)
+                        mbar_wait(k_full(u), 0, &no_abort, a.err);
+                if (q_issued) mbar_wait(bar_q, 0, &no_abort, a.err);
             }
         }
     } else if (warp == S::MMA_WARP) {
@@ -463,44 +515,62 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, KT);
             constexpr uint32_t idesc_o = umma_idesc_bf16_f32(128, D, true);
             ok = mbar_wait(bar_q, 0, abort_flag, a.err);
-            for (int t = 0; ok && t <= nt; ++t) {
-                if (t < nt) {
-                    const int st = t % STAGES, b2 = t & 1;
-                    if (!(ok = mbar_wait(k_full(st), (t / STAGES) & 1, abort_flag, a.err))) break;
-                    if (!(ok = mbar_wait(s_free(b2), ((t >> 1) & 1) ^ 1, abort_flag, a.err)))
-                        break;
-                    tc_fence_after();
+            // S(t) = Q K(t)^T and O += P(u) V(u), each issued as soon as its
+            // operands are there: a PV never queues behind the next tile's K
+            int ns = 0, npv = 0;
+            PollBudget pb;
+            while (ok && npv < nt) {
+                bool moved = false;
+                if (npv < ns) {
+                    const int u = npv, su = u % STAGES, pbuf = u & 1;
+                    if (mbar_test(p_full(pbuf), (u >> 1) & 1) &&
+                        mbar_test(v_full(su), (u / STAGES) & 1)) {
+                        tc_fence_after();
 #pragma unroll
-                    for (int m = 0; m < MT; ++m)
+                        for (int m = 0; m < MT; ++m)
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t qa = sb + S::OFF_Q + (kk >> 2) * S::Q_CHUNK +
-                                                m * 16384 + (kk & 3) * 32;
-                            const uint32_t ka = sb + S::OFF_K + st * S::KV_TILE +
-                                                (kk >> 2) * S::KV_CHUNK + (kk & 3) * 32;
-                            umma_bf16(tmem + S::TMEM_S + (b2 * MT + m) * KT, umma_desc_sw128(qa),
-                                      umma_desc_sw128(ka), idesc_s, kk > 0);
-                        }
-                    umma_commit(s_full(b2));
+                            for (int ks = 0; ks < KT / 16; ++ks) {
+                                const uint32_t pa = sb + S::OFF_P + (pbuf * MT + m) * S::P_TILE +
+                                                    (ks & 3) * 32;
+                                const uint32_t va = sb + S::OFF_V + su * S::KV_TILE + ks * 2048;
+                                umma_bf16(tmem + S::TMEM_O + m * D, umma_desc_sw128(pa),
+                                          umma_desc_sw128_mn(va, S::KV_CHUNK), idesc_o,
+                                          (u > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        umma_commit(o_done(pbuf));
+                        umma_commit(v_empty(su));
+                        ++npv;
+                        moved = true;
+                    }
                 }
-                if (t > 0) {
-                    const int u = t - 1, su = u % STAGES, pb = u & 1;
-                    if (!(ok = mbar_wait(p_full(pb), (u >> 1) & 1, abort_flag, a.err))) break;
-                    if (!(ok = mbar_wait(v_full(su), (u / STAGES) & 1, abort_flag, a.err))) break;
-                    tc_fence_after();
+                if (ns < nt) {
+                    const int t = ns, st = t % STAGES, b2 = t & 1;
+                    if (mbar_test(k_full(st), (t / STAGES) & 1) &&
+                        mbar_test(s_free(b2), ((t >> 1) & 1) ^ 1)) {
+                        tc_fence_after();
 #pragma unroll
-                    for (int m = 0; m < MT; ++m)
+                        for (int m = 0; m < MT; ++m)
 #pragma unroll
-                        for (int ks = 0; ks < KT / 16; ++ks) {
-                            const uint32_t pa = sb + S::OFF_P + (pb * MT + m) * S::P_TILE +
-                                                (ks & 3) * 32;
-                            const uint32_t va = sb + S::OFF_V + su * S::KV_TILE + ks * 2048;
-                            umma_bf16(tmem + S::TMEM_O + m * D, umma_desc_sw128(pa),
-                                      umma_desc_sw128_mn(va, S::KV_CHUNK), idesc_o,
-                                      (u > 0 || ks > 0) ? 1u : 0u);
-                        }
-                    umma_commit(o_done(pb));
-                    umma_commit(kv_empty(su));
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t qa = sb + S::OFF_Q + (kk >> 2) * S::Q_CHUNK +
+                                                    m * 16384 + (kk & 3) * 32;
+                                const uint32_t ka = sb + S::OFF_K + st * S::KV_TILE +
+                                                    (kk >> 2) * S::KV_CHUNK + (kk & 3) * 32;
+                                umma_bf16(tmem + S::TMEM_S + (b2 * MT + m) * KT,
+                                          umma_desc_sw128(qa), umma_desc_sw128(ka), idesc_s,
+                                          kk > 0);
+                            }
+                        umma_commit(s_full(b2));
+                        umma_commit(k_empty(st));
+                        ++ns;
+                        moved = true;
+                    }
+                }
+                if (moved) {
+                    pb.reset();
+                } else {
+                    __nanosleep(32);                // leave issue slots to the softmax warps
+                    ok = pb.idle(abort_flag, a.err);
                 }
             }
         }

@@ -51,6 +51,42 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Non-blocking: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Poll budget of a producer loop that waits on several barriers at once:
+// returns false (after raising *abort and recording DEV_TIMEOUT) once it has
+// found nothing to do for longer than the timeout, or when another thread has
+// given up. Call reset() whenever the loop made progress.
+struct PollBudget {
+    uint32_t n = 0;
+    uint64_t t0 = 0;
+    __device__ __forceinline__ void reset() { n = 0; t0 = 0; }
+    __device__ __forceinline__ bool idle(volatile int* abort, int* err) {
+        if ((++n & 63u) != 0) return true;
+        if (*abort) return false;
+        const uint64_t now = globaltimer();
+        if (t0 == 0) {
+            t0 = now;
+        } else if (now - t0 > kWaitTimeoutNs) {
+            *abort = 1;
+            record_error(err, DEV_TIMEOUT);
+            return false;
+        }
+        return true;
+    }
+};
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
