@@ -399,14 +399,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             tma_load_3d(sb + S::OFF_V + st * S::KV_TILE, &tmV, v_full(st), 0, krow0 + t * KT, 0);
     };
     // With a prologue, the preceding kernel is this call's own projection,
-    // which writes no cache row: whole tiles outside the block slot can be
-    // requested before it ends (ring stages are fresh, so no empty wait).
+    // which writes no cache row: the first tile, when it lies outside the block
+    // slot, can be requested before that kernel ends (its ring stage is fresh,
+    // so no empty wait). One tile only: a larger burst delays the loads of the
+    // prologue that follows (measured).
     uint32_t early = 0;
     if constexpr (Pro::kActive) {
         if (warp == S::TMA_WARP && lane == 0) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            for (int t = 0; t < nt && t < STAGES; ++t) {
+            for (int t = 0; t < nt && t < 1; ++t) {
                 const int tile = tile_of(t);
                 if (k_begin + (tile + 1) * KT <= a.L && !in_block(tile)) {
                     load_k(tile, t);

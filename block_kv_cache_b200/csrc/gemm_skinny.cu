@@ -247,13 +247,16 @@ struct ProRMSNorm {
         const bool in_regs = n4 <= RV * (int)blockDim.x;
         for (int r = part; r < M; r += nparts) {
             const float4* x = reinterpret_cast<const float4*>(h + (size_t)r * D);
-            float4 v[RV];
+            const float4* w4 = reinterpret_cast<const float4*>(w);
+            float4 v[RV], gw[RV];
             float ss = 0.f;
             if (in_regs) {                           // one pass: the row stays in registers
+                // the row and the norm weights in one round of loads
 #pragma unroll
                 for (int k = 0; k < RV; ++k) {
                     const int j = threadIdx.x + k * blockDim.x;
                     v[k] = j < n4 ? __ldcg(x + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    gw[k] = j < n4 ? __ldg(w4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
 #pragma unroll
                 for (int k = 0; k < RV; ++k)
@@ -271,14 +274,13 @@ struct ProRMSNorm {
 #pragma unroll
             for (int k = 0; k < SK_THREADS / 32; ++k) tot += red[k];
             const float inv = rsqrtf(tot / (float)D + eps);
-            const float4* w4 = reinterpret_cast<const float4*>(w);
             __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + (size_t)r * D);
             if (in_regs) {
 #pragma unroll
                 for (int k = 0; k < RV; ++k) {
                     const int j = threadIdx.x + k * blockDim.x;
                     if (j < n4) {
-                        const float4 g = __ldg(w4 + j);
+                        const float4 g = gw[k];
                         o2[2 * j] = __floats2bfloat162_rn(v[k].x * inv * g.x, v[k].y * inv * g.y);
                         o2[2 * j + 1] =
                             __floats2bfloat162_rn(v[k].z * inv * g.z, v[k].w * inv * g.w);
