@@ -235,8 +235,8 @@ def run_gpu(args):
         ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
         # DRAM bytes read + written by the two kernels of one such call, from an
         # ncu capture of the same kernels at this shape (kernel_cases ffn --rows
-        # 32 --n 12288 --k 4096): 205.08 + 3.51 + 104.40 + 1.77 MB
-        ffn_traffic = 205_079_808 + 3_514_624 + 104_400_896 + 1_767_424
+        # 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
+        ffn_traffic = 205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
         out = {
             "metric": METRIC, "value": toks_all / (ms_max / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
