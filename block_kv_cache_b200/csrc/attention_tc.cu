@@ -92,7 +92,12 @@ struct Att4 {
     static constexpr int OFF_P = OFF_V + STAGES * KV_TILE;   // P[buffer][m]
     static constexpr int OFF_RED = OFF_P + 2 * MT * P_TILE;  // 128 MT x (max, sum) floats
     static constexpr int OFF_BAR = OFF_RED + 128 * MT * 2 * 4;
-    static constexpr size_t TOTAL = 1024 + OFF_BAR + 256;
+    // Receive buffer of the pushed split merge (single-tile shapes): partial
+    // rows of every split for the rows this CTA owns, (D + 4) floats each.
+    static constexpr int OFF_RCV = OFF_BAR + 256;
+    static constexpr int RCV_BYTES = MT == 1 ? 65536 : 0;
+    static constexpr int RCV_ROW = (D + 4) * 4;
+    static constexpr size_t TOTAL = 1024 + OFF_RCV + RCV_BYTES;
     // After the last MMA, [OFF_K, OFF_RED) holds this CTA's partial output
     // (R rows x D floats, float4 slots XOR-swizzled by row) for the cluster.
     static_assert(128 * MT * D * 4 <= OFF_RED - OFF_K, "partial buffer");
@@ -150,6 +155,7 @@ struct AttnArgs {
     float* lse;         // optional
     int B, Hq, Hkv, L, hc, n_chunks, rows, tiles, tps, n_splits, q_per_kv;
     int blk0, blk1;     // block slot [blk0, blk1) of every sequence
+    int push;           // splits push their partial rows to the owner's buffer
     float scale_log2;
     int* err;
 };
@@ -326,7 +332,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     auto p_full = [&](int b) { return smem_u32(bars + 5 + 4 * STAGES + b); };
     auto o_done = [&](int b) { return smem_u32(bars + 7 + 4 * STAGES + b); };
     const uint32_t bar_kv = smem_u32(bars + 9 + 4 * STAGES);   // block-slot rows written
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 4 * STAGES);
+    const uint32_t bar_rcv = smem_u32(bars + 10 + 4 * STAGES);  // pushed partials landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11 + 4 * STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int split = blockIdx.x;                    // == rank in the cluster
@@ -355,9 +362,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int k0 = k_begin + tile * KT;
         return k0 < a.blk1 && k0 + KT > a.blk0;
     };
+    // split merge: split c owns packed rows [c * rpc, c * rpc + own)
+    const int rpc = (a.rows + a.n_splits - 1) / a.n_splits;
+    const int own = max(0, min(rpc, a.rows - split * rpc));
+    const bool push = a.push != 0 && a.n_splits > 1 &&
+                      a.n_splits * rpc * S::RCV_ROW <= S::RCV_BYTES;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
+        mbar_init(bar_rcv, 1);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(k_full(s), 1);
             mbar_init(v_full(s), 1);
@@ -373,11 +386,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         *abort_flag = 0;
         fence_barrier_init();
+        // every split pushes D + 2 floats for each row this CTA owns
+        if (push) mbar_arrive_expect_tx(bar_rcv, (uint32_t)(a.n_splits * own * (D * 4 + 8)));
     }
     if (warp == S::MMA_WARP) tmem_alloc(smem_u32(tmem_slot), S::TMEM_ALLOC);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the receive barriers of the cluster are initialised once every thread
+    // has arrived here; the matching wait comes just before the first push
+    if (push) cluster_arrive();
+    bool rcv_ready = !push;
     const uint32_t tmem = *tmem_slot;
     const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
     const uint64_t kv_policy = l2_evict_first();
@@ -683,6 +702,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             // above is bounded, so all of them get here
             named_sync(1, live_threads);
             ok = __all_sync(0xffffffffu, ok && *abort_flag == 0);
+            if (push) {                     // the owners' receive barriers exist
+                cluster_wait();
+                rcv_ready = true;
+            }
             if (ok) {
                 tc_fence_after();
                 float o[D];
@@ -711,6 +734,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                             a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
                                 (m_run + log2f(l_run)) * 0.69314718055994530942f;
                     }
+                } else if (row_ok && push) {
+                    // push this row's partial into the owner's receive buffer
+                    const int oc = pr / rpc, j = pr - oc * rpc;
+                    const uint32_t dst = cluster_map(
+                        sb + S::OFF_RCV + (uint32_t)((split * rpc + j) * S::RCV_ROW), oc);
+                    const uint32_t rbar = cluster_map(bar_rcv, oc);
+#pragma unroll
+                    for (int d4 = 0; d4 < D / 4; ++d4)
+                        st_async_f4(dst + d4 * 16,
+                                    make_float4(o[4 * d4], o[4 * d4 + 1], o[4 * d4 + 2],
+                                                o[4 * d4 + 3]),
+                                    rbar);
+                    st_async_f2(dst + D * 4, make_float2(m_run, l_run), rbar);
                 } else if (row_ok) {
                     // publish this CTA's partial for the cluster merge
                     float* part = reinterpret_cast<float*>(smem + S::OFF_K) + (size_t)pr * D;
@@ -726,11 +762,61 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
     }
 
-    if (a.n_splits > 1) {
+    if (push) {
+        // -------------------------------------- merge of the pushed split partials
+        if (!rcv_ready) cluster_wait();
+        // every split's rows have landed (bounded; on the give-up path still wait
+        // for what is in flight, so that no push lands after this CTA has left)
+        volatile int no_abort = 0;
+        const bool got = own == 0 || mbar_wait(bar_rcv, 0, &no_abort, a.err);
+        const int items = got && *abort_flag == 0 ? own * (D / 8) : 0;
+        for (int it = threadIdx.x; it < items; it += S::THREADS) {
+            const int j = it / (D / 8), d8 = it % (D / 8);
+            const int pr = split * rpc + j;
+            const int i = pr / a.hc, hig = chunk * a.hc + pr % a.hc;
+            if (i >= a.B || hig >= grp) continue;
+            float2 ml[ATT_MAX_SPLITS];
+            float4 v0[ATT_MAX_SPLITS], v1[ATT_MAX_SPLITS];
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {
+                if (cc < a.n_splits) {
+                    const uint8_t* row = smem + S::OFF_RCV + (cc * rpc + j) * S::RCV_ROW;
+                    ml[cc] = *reinterpret_cast<const float2*>(row + D * 4);
+                    v0[cc] = *reinterpret_cast<const float4*>(row + d8 * 32);
+                    v1[cc] = *reinterpret_cast<const float4*>(row + d8 * 32 + 16);
+                }
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc)
+                if (cc < a.n_splits) M = fmaxf(M, ml[cc].x);
+            float Lsum = 0.f;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int cc = 0; cc < ATT_MAX_SPLITS; ++cc) {
+                if (cc < a.n_splits && ml[cc].x != -INFINITY) {
+                    const float w = ex2(ml[cc].x - M);
+                    Lsum += ml[cc].y * w;
+                    acc[0] += v0[cc].x * w; acc[1] += v0[cc].y * w;
+                    acc[2] += v0[cc].z * w; acc[3] += v0[cc].w * w;
+                    acc[4] += v1[cc].x * w; acc[5] += v1[cc].y * w;
+                    acc[6] += v1[cc].z * w; acc[7] += v1[cc].w * w;
+                }
+            }
+            const float inv = 1.f / Lsum;
+            const int head = g * grp + hig;
+            bf16* dst = a.out + (((size_t)bb * a.B + i) * a.Hq + head) * D + d8 * 8;
+            *reinterpret_cast<uint4*>(dst) =
+                make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                           pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+            if (a.lse && d8 == 0)
+                a.lse[((size_t)bb * a.Hq + head) * a.B + i] =
+                    (M + log2f(Lsum)) * 0.69314718055994530942f;
+        }
+    } else if (a.n_splits > 1) {
         // ------------------------------------------------ cluster merge of splits
         // every thread of every CTA of the cluster takes part in both barriers
         cluster_sync();
-        const int rpc = (a.rows + a.n_splits - 1) / a.n_splits;      // rows per CTA
         const int r0 = split * rpc, r1 = min(a.rows, r0 + rpc);
         // item = 8 output columns of one row: two float4 slots per split
         const int items = (r1 > r0 ? r1 - r0 : 0) * (D / 8);
@@ -783,8 +869,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         cluster_sync();                    // no CTA leaves while others read its smem
     }
-    // every split of this head has read the q sums (the cluster barrier above,
-    // or, with one split, the barrier after the prologue)
+    // every split of this head has read the q sums (split 0 has received every
+    // split's partial, or passed the cluster barrier above, or, with one split,
+    // the barrier after the prologue)
     if constexpr (Pro::kActive)
         if (split == 0) qkv_zero_q(pro, a, g, bb);
     tc_fence_before();
@@ -850,6 +937,12 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     a.q_per_kv = s.q_per_kv;
     a.blk0 = s.block_start;
     a.blk1 = s.block_start + s.block_len;
+    {
+        // pushed merge when every split's rows for one owner fit its buffer
+        const int rpc = (p.rows + p.n_splits - 1) / p.n_splits;
+        const int need = p.n_splits * rpc * (D + 4) * 4;
+        a.push = p.mt == 1 && p.n_splits > 1 && need <= Att4<128, 1>::RCV_BYTES ? 1 : 0;
+    }
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
     const int hb = s.batch, hk = s.n_kv_heads;
