@@ -39,10 +39,25 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-CFG = dict(layers=32, hidden=4096, heads=32, kv_heads=32, head_dim=128, ffn=12288,
-           vocab=126464, mask_id=126336, batch=1, prompt=1024, gen=1024, block=32, tau=0.9)
-WORKLOAD = ("LLaDA-8B-shaped random-init model, bf16, batch 1, prompt 1024 + gen 1024, "
-            "block 32, DualCache, tau 0.9: Fast-dLLM block decoding steps")
+CONFIGS = {
+    # the headline workload: LLaDA-8B-shaped, batch 1
+    "llada": dict(layers=32, hidden=4096, heads=32, kv_heads=32, head_dim=128, ffn=12288,
+                  vocab=126464, mask_id=126336, batch=1, prompt=1024, gen=1024, block=32,
+                  tau=0.9, qkv_bias=False,
+                  workload="LLaDA-8B-shaped random-init model, bf16, batch 1, prompt 1024 + "
+                           "gen 1024, block 32, DualCache, tau 0.9: Fast-dLLM block decoding "
+                           "steps"),
+    # Dream-7B-shaped (Qwen2.5-7B layout: GQA 28/4, q/k/v bias), batch 32; the mask
+    # id is not given for it: vocab - 1
+    "dream": dict(layers=28, hidden=3584, heads=28, kv_heads=4, head_dim=128, ffn=18944,
+                  vocab=152064, mask_id=152063, batch=32, prompt=512, gen=512, block=32,
+                  tau=0.9, qkv_bias=True,
+                  workload="Dream-7B-shaped random-init model, bf16, batch 32, prompt 512 + "
+                           "gen 512, block 32, DualCache, tau 0.9: Fast-dLLM block decoding "
+                           "steps"),
+}
+CFG = dict(CONFIGS["llada"])
+WORKLOAD = CFG["workload"]
 METRIC = "generated tokens/s per B200"
 
 
@@ -56,6 +71,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile-steps", action="store_true",
                    help="also print the per-call time of a cached step and of a refresh")
+    p.add_argument("--config", choices=sorted(CONFIGS), default="llada",
+                   help="workload: the LLaDA-8B-shaped batch-1 decode (default) or the "
+                        "Dream-7B-shaped batch-32 decode")
     return p.parse_args()
 
 
@@ -63,7 +81,7 @@ def shape():
     from block_kv_cache_b200.model import ModelShape
     c = CFG
     return ModelShape(c["vocab"], c["hidden"], c["layers"], c["heads"], c["kv_heads"], c["ffn"],
-                      c["mask_id"], c["head_dim"])
+                      c["mask_id"], c["head_dim"], qkv_bias=c["qkv_bias"])
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -128,11 +146,6 @@ def read_peaks():
         return {}
 
 
-# kernels per step: embed, final norm, LM head (2), unmask, and per layer
-#   cached:  QKV GEMM (norm inside), attention (QKV epilogue inside), O GEMM,
-#            gate/up GEMM (norm inside), down GEMM (SwiGLU inside)
-#   refresh: norm, QKV GEMM, full attention, O GEMM, norm, gate/up GEMM, down GEMM
-LAUNCHES = {"cached": 32 * 5 + 5, "refresh": 32 * 7 + 5}
 
 
 def combine_ranks(dist, world, ms, toks, device):
@@ -178,6 +191,9 @@ def run_gpu(args):
     t0 = time.perf_counter()
     dec.capture_all(c["prompt"], c["gen"], c["tau"], time_ffn=True)
     capture_s = time.perf_counter() - t0
+    # kernels each step graph launches (kernel nodes of the captured graphs)
+    for key in list(dec.graphs):
+        dec.kernel_launches(*key)
 
     dec.begin(prompt, c["tau"])
     for _ in range(max(args.warmup, 3)):
@@ -191,7 +207,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    toks, kinds = 0, {"refresh": 0, "cached": 0}
+    toks, kinds, launches = 0, {"refresh": 0, "cached": 0}, 0
     sw_ms, sw_n = 0.0, 0
     step_ms = {"refresh": [], "cached": []}
     with ClockSampler(local) as clk:
@@ -200,6 +216,7 @@ def run_gpu(args):
             h0 = time.perf_counter()
             toks += dec.step()
             step_ms[dec.last_kind].append((time.perf_counter() - h0) * 1e3)
+            launches += dec.kernel_launches(*dec._last_key)
             kinds[dec.last_kind] += 1
             if dec.last_kind == "cached":
                 for a, b in dec.last_timers():
@@ -231,12 +248,27 @@ def run_gpu(args):
         # rows read for the norm and read + written by the down projection, x and
         # f each written and read back
         ffn_bytes = 3 * F * D * 2 + 2 * M * D * 2 + 2 * M * F * 2 + 3 * M * D * 4
+        ffn_flops = 6.0 * M * D * F
         sw_avg_ms = sw_ms / max(sw_n, 1)
-        ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
+        if M <= 256:
+            # few rows: the call streams its weights (HBM-bound)
+            ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
+            bound, unit, kpeak, src = "hbm", "GB/s", peak, (
+                "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks.get("hbm_gbs")
+                else "fallback 6650 GB/s")
+        else:
+            # a batch of blocks: the call is two dense GEMMs (tensor-bound), timed
+            # inside a long step, so against the sustained bf16 peak
+            ach = ffn_flops / (sw_avg_ms / 1e3) / 1e12 if sw_n else None
+            kpeak = peaks.get("bf16_tflops_sustained") or 1400.0
+            bound, unit, src = "tensor", "TFLOP/s", (
+                "MEASURED_PEAKS.json bf16_tflops_sustained (measured)"
+                if peaks.get("bf16_tflops_sustained") else "fallback 1400 TFLOP/s sustained")
         # DRAM bytes read + written by the two kernels of one such call, from an
-        # ncu capture of the same kernels at this shape (kernel_cases ffn --rows
-        # 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
-        ffn_traffic = 205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
+        # ncu capture of the same kernels at the LLaDA-8B shape (kernel_cases ffn
+        # --rows 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
+        ffn_traffic = (205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
+                       if (M, D, F) == (32, 4096, 12288) else None)
         out = {
             "metric": METRIC, "value": toks_all / (ms_max / 1e3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -253,19 +285,20 @@ def run_gpu(args):
                                                  for k, v in step_ms.items()},
                        "weights_gb": round(w.nbytes() / 1e9, 2),
                        "graph_capture_s": round(capture_s, 2),
-                       "l2": "no flush: 16 GB of weights (> 126 MB L2) are streamed every step"},
-            "gpu_launches": sum(LAUNCHES[k] * n for k, n in kinds.items()),
-            "roofline": {"kernel": "ffn call of a cached step (M=32): gate/up GEMM 24576x4096 "
-                                   "whose CTAs apply the RMSNorm first, with split-K sums, then "
-                                   "the down GEMM 4096x12288 whose CTAs apply the SwiGLU first; "
-                                   "60% of the step's weight bytes",
-                         "bytes_per_call": ffn_bytes,
-                         "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                         "frac": (ach / peak) if ach else None, "traffic": ffn_traffic,
+                       "l2": f"no flush: {w.nbytes() / 1e9:.0f} GB of weights (> 126 MB L2) "
+                             f"are streamed every step"},
+            "gpu_launches": launches,
+            "roofline": {"kernel": f"ffn call of layer 0 of a cached step (M={M}): RMSNorm, "
+                                   f"gate/up GEMM {2 * F}x{D}, SwiGLU, down GEMM {D}x{F} "
+                                   f"(with M <= 256 the RMSNorm and the SwiGLU run in the "
+                                   f"GEMM kernels' prologues)",
+                         "bytes_per_call": ffn_bytes, "flops_per_call": ffn_flops,
+                         "bound": bound, "achieved": ach, "peak": kpeak, "unit": unit,
+                         "frac": (ach / kpeak) if ach else None, "traffic": ffn_traffic,
                          "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                           "the two kernels of one call",
-                         "peak_source": "MEASURED_PEAKS.json hbm_gbs (measured)"
-                         if peaks.get("hbm_gbs") else "fallback 6650 GB/s",
+                                           "the two kernels of one call" if ffn_traffic
+                         else "no capture at this shape",
+                         "peak_source": src,
                          "avg_launch_us": sw_avg_ms * 1e3, "launches_timed": sw_n},
             "e2e": {"value": e2e_val, "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
@@ -311,9 +344,11 @@ def run_e2e(torch, dec, prompt, steps):
 # ----------------------------------------------------------------------------- CPU oracle
 class OracleSample:
     """A bounded sample of one decode step computed by the CPU oracle (float64
-    NumPy): one transformer layer of a cached block step (32 block rows over a
-    2048-row cache) and the full LM-head confidence of the block; a whole step
-    is extrapolated as 32 x layer + LM head."""
+    NumPy): one transformer layer of a cached block step of one sequence (its
+    block rows over its cache) and the full LM-head confidence of the block; a
+    sequence's step is extrapolated as layers x layer + LM head. The rows of a
+    batch are independent, so the batch's tokens per second equal one
+    sequence's (batch tokens per step, batch times the work)."""
 
     def __init__(self, seed=0):
         from oracle import fastdllm as O
@@ -321,13 +356,13 @@ class OracleSample:
         self.O = O
         c = CFG
         P = synth.model_params(vocab=8, hidden=c["hidden"], n_layers=1, n_q_heads=c["heads"],
-                               head_dim=c["head_dim"], ffn=c["ffn"], seed=seed, w_std=0.02,
-                               dtype="bf16")
+                               n_kv_heads=c["kv_heads"], head_dim=c["head_dim"], ffn=c["ffn"],
+                               seed=seed, w_std=0.02, dtype="bf16", qkv_bias=c["qkv_bias"])
         self.P = P
         g = synth.rng(seed + 1)
         L = c["prompt"] + c["gen"]
-        self.k = g.standard_normal((c["heads"], L, c["head_dim"]))
-        self.v = g.standard_normal((c["heads"], L, c["head_dim"]))
+        self.k = g.standard_normal((c["kv_heads"], L, c["head_dim"]))
+        self.v = g.standard_normal((c["kv_heads"], L, c["head_dim"]))
         self.h = g.standard_normal((c["block"], c["hidden"]))
         self.lm = synth.lmhead_case(rows=c["block"], hidden=c["hidden"], vocab=c["vocab"],
                                     seed=seed, w_seed=0, mask_id=c["mask_id"])
@@ -369,9 +404,10 @@ def cpu_baseline(budget_s=20.0):
     step_s = statistics.median(e[0] for e in est)
     return {"value": 1.0 / step_s, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
             "host_cpus": os.cpu_count(),
-            "sample": f"{n} samples of one layer of a cached block step (32 rows over a "
-                      f"2048-row cache) + the full LM head, float64 NumPy; step time "
-                      f"extrapolated as 32 x layer ({statistics.median(e[1] for e in est):.3f} s)"
+            "sample": f"{n} samples of one layer of a cached block step of one sequence "
+                      f"({CFG['block']} rows over a {CFG['prompt'] + CFG['gen']}-row cache) + "
+                      f"the full LM head, float64 NumPy; step time extrapolated as "
+                      f"{CFG['layers']} x layer ({statistics.median(e[1] for e in est):.3f} s)"
                       f" + LM head ({statistics.median(e[2] for e in est):.3f} s), 1 token "
                       f"per step as on the GPU"}
 
@@ -399,16 +435,21 @@ def run_reference(args):
                       "layers": CFG["layers"], "parallelism": "cpu oracle"},
            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": _threads(),
                             "kind": "oracle", "host_cpus": os.cpu_count(),
-                            "sample": f"each step: one layer of a cached block step + the full "
-                                      f"LM head, extrapolated to 32 layers ({wall:.1f} s of "
-                                      f"CPU time for {args.steps} steps)"},
+                            "sample": f"each step: one layer of a cached block step of one "
+                                      f"sequence + the full LM head, extrapolated to "
+                                      f"{CFG['layers']} layers ({wall:.1f} s of CPU time for "
+                                      f"{args.steps} steps)"},
            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
 def main():
+    global WORKLOAD
     args = parse()
+    CFG.clear()
+    CFG.update(CONFIGS[args.config])
+    WORKLOAD = CFG["workload"]
     if args.impl == "reference":
         run_reference(args)
     else:

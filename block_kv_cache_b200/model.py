@@ -21,6 +21,7 @@ epilogue finds both halves of a feature in one tile.
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 
 import numpy as np
@@ -42,6 +43,29 @@ class ModelShape:
     rope_theta: float = 10000.0
     rms_eps: float = 1e-5
     qkv_bias: bool = False
+
+
+def graph_kernel_count(g: "torch.cuda.CUDAGraph") -> int:
+    """Kernel nodes of a captured CUDA graph (kept with keep_graph=True): the
+    kernels one replay launches, read through the CUDA driver API."""
+    cu = ctypes.CDLL("libcuda.so.1")
+    cu.cuGraphGetNodes.argtypes = [ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.POINTER(ctypes.c_size_t)]
+    cu.cuGraphNodeGetType.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int)]
+    h = ctypes.c_void_p(g.raw_cuda_graph())
+    n = ctypes.c_size_t(0)
+    if cu.cuGraphGetNodes(h, None, ctypes.byref(n)) != 0:
+        raise RuntimeError("cuGraphGetNodes failed")
+    nodes = (ctypes.c_void_p * n.value)()
+    if cu.cuGraphGetNodes(h, nodes, ctypes.byref(n)) != 0:
+        raise RuntimeError("cuGraphGetNodes failed")
+    kind = ctypes.c_int(-1)
+    count = 0
+    for nd in nodes:
+        if cu.cuGraphNodeGetType(ctypes.c_void_p(nd), ctypes.byref(kind)) != 0:
+            raise RuntimeError("cuGraphNodeGetType failed")
+        count += kind.value == 0                  # CU_GRAPH_NODE_TYPE_KERNEL
+    return count
 
 
 def _bf16(a, dev):
@@ -153,6 +177,7 @@ class BlockDecoder:
         self.masked = torch.empty((batch, seq_len), dtype=torch.uint8, device=dev)
         self.graphs = {}
         self.graph_timers = {}          # graph key -> [(event, event)] around the FFN calls
+        self._launches = {}             # graph key -> kernels per replay
         self._timers = None
         # rows of block k of every sequence in the flattened [b * L] token rows
         nblk = (seq_len + block - 1) // block
@@ -280,14 +305,22 @@ class BlockDecoder:
         time_ffn, timing events bracket layer 0's FFN call."""
         key = (kind, s, float(tau))
         if key not in self.graphs:
-            g = torch.cuda.CUDAGraph()
+            g = torch.cuda.CUDAGraph(keep_graph=True)   # the graph stays readable
             self._timers = [] if time_ffn else None
             with torch.cuda.graph(g):
                 self._step_calls(kind, s, tau)
+            g.instantiate()
             self.graph_timers[key] = self._timers or []
             self._timers = None
             self.graphs[key] = g
         return self.graphs[key]
+
+    def kernel_launches(self, kind, s, tau):
+        """Kernels one replay of the step graph (kind, s, tau) launches."""
+        key = (kind, s, float(tau))
+        if key not in self._launches:
+            self._launches[key] = graph_kernel_count(self.capture(kind, s, tau))
+        return self._launches[key]
 
     def last_timers(self):
         """Event pairs of the graph replayed by the last step()."""

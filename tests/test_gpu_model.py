@@ -291,3 +291,55 @@ def test_tau_one_single_layer_gpu_equals_sequential(ctx):
             continue                                   # near tie: either choice is correct
         gpu_pick = int(np.argmax(np.where(cand, conf, -1.0)))
         assert gpu_pick == top
+
+
+def test_dream_shape_full_decode(ctx):
+    """The Dream-7B-shaped configuration at full size: random-init 28 layers,
+    hidden 3584, GQA 28/4 with q/k/v bias, FFN 18944, vocab 152064, bf16,
+    batch 32, prompt 512 + gen 512, block 32, tau 0.9. The whole decode:
+    every step's unmask decisions bit-exact against the oracle given the GPU's
+    confidences; each sequence with masked positions in the block decodes at
+    least one per step; nothing outside the block changes; everything is
+    decoded at the end and the prompt is untouched. Then the LM-head
+    confidences of sampled rows of the last step against the oracle on the
+    GPU's own final hidden states (within 1e-5)."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights, ModelShape
+    sh = ModelShape(152064, 3584, 28, 28, 4, 18944, 152063, 128, qkv_bias=True)
+    w = DeviceWeights.random(sh, seed=77)
+    b, Lp, gen, B, tau = 32, 512, 512, 32, 0.9
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B)
+    prompt = synth.prompt_ids(3, b, Lp, sh.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
+    ctx.device_status()
+    xf = x.cpu().numpy()
+    assert steps == len(rec) and gen // B <= steps <= gen
+    total = np.zeros(b, np.int64)
+    for n, (kind, s, xb, mb, conf, tok) in enumerate(rec):
+        conf, tok = conf.reshape(b, B), tok.reshape(b, B)
+        xa, ma, _, nd = O.threshold_unmask(xb, mb, conf, tok, s, B, tau)
+        x_next = rec[n + 1][2] if n + 1 < len(rec) else xf
+        assert np.array_equal(xa, x_next), n
+        if n + 1 < len(rec):
+            assert np.array_equal(ma, rec[n + 1][3]), n
+        assert not np.any(ma.astype(bool) & ~mb.astype(bool)), n   # never re-masked
+        had = mb[:, s:s + B].any(axis=1)
+        dec_now = (mb[:, s:s + B].astype(bool) & ~ma[:, s:s + B].astype(bool)).sum(axis=1)
+        assert np.all(dec_now[had] >= 1), n                         # progress every step
+        total += dec_now
+        out = np.ones(Lp + gen, bool)
+        out[s:s + B] = False
+        assert np.array_equal(x_next[:, out], xb[:, out]), n
+    assert np.all(total == gen)                                     # everything decoded
+    assert np.array_equal(xf[:, :Lp], np.asarray(prompt))
+    assert xf.min() >= 0 and xf.max() < sh.vocab
+    # LM head of the last step on the GPU's final hidden states
+    rows = np.array([0, 31, 517, 1023])
+    h = dec.xn[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    lm = w.lm_head.float().cpu().numpy()
+    r = O.lmhead_confidence(h, lm)
+    conf_g = dec.conf.cpu().numpy().reshape(-1)[rows]
+    tok_g = dec.tok.cpu().numpy().reshape(-1)[rows]
+    assert np.abs(conf_g - r.conf).max() <= 1e-5
+    sure = r.gap > 1e-3
+    assert np.array_equal(tok_g[sure], r.tok[sure])
