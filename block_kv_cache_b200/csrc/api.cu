@@ -11,6 +11,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <vector>
+
 struct fdl_ctx {
     int device;
     int sm_count;
@@ -549,6 +551,267 @@ int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
                                                     out, ctx->sm_count, ctx->d_err,
                                                     (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "full_attention launch");
+}
+
+}  // extern "C"
+
+// ---- the whole decode ------------------------------------------------------------
+struct fdl_model {
+    fdl_model_desc d;
+    const void* embed;
+    const float* final_norm;
+    const void* lm_head;
+    std::vector<fdl_layer_weights> layers;
+};
+
+namespace {
+
+__global__ void fill_i32_kernel(int32_t* __restrict__ p, size_t n, int32_t v) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+         i += (size_t)gridDim.x * blockDim.x)
+        p[i] = v;
+}
+
+// rows of block k of every sequence in the flattened [b * L] token rows:
+// maps[k][i * B + j] = i * L + k * B + j (clamped to the last row)
+__global__ void block_rows_kernel(int32_t* __restrict__ maps, int b, int L, int B, int nblk) {
+    const size_t n = (size_t)nblk * b * B;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const int k = (int)(e / ((size_t)b * B)), r = (int)(e % ((size_t)b * B));
+        const int i = r / B, j = r % B;
+        const long v = (long)i * L + (long)k * B + j;
+        maps[e] = (int32_t)(v < (long)b * L ? v : (long)b * L - 1);
+    }
+}
+
+// Byte offsets of the generate workspace (256-byte aligned pieces).
+struct GenLayout {
+    size_t kc, vc, h_full, x_full, q_full, o_full, f_full, h_blk, x_blk, q_blk, o_blk, f_blk,
+        xn, conf, tok, masked, counts, maps, rope, lm_ws, total;
+    size_t kv_layer;    // bytes of one layer's K (or V) cache
+    size_t lm_bytes;
+};
+
+GenLayout gen_layout(const fdl_model_desc& d, int b, int L, int B, size_t lm_bytes) {
+    GenLayout g{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return at;
+    };
+    const size_t D = d.hidden, F = d.ffn, hd = 128, Hq = d.n_q_heads, Hkv = d.n_kv_heads;
+    const size_t rf = (size_t)b * L, rb = (size_t)b * B;
+    const int nblk = (L + B - 1) / B;
+    g.kv_layer = (size_t)b * Hkv * L * hd * 2;
+    g.kc = take(g.kv_layer * d.n_layers);
+    g.vc = take(g.kv_layer * d.n_layers);
+    g.h_full = take(rf * D * 4);
+    g.x_full = take(rf * D * 2);
+    g.q_full = take(rf * Hq * hd * 2);
+    g.o_full = take(rf * Hq * hd * 2);
+    g.f_full = take(rf * F * 2);
+    g.h_blk = take(rb * D * 4);
+    g.x_blk = take(rb * D * 2);
+    g.q_blk = take(rb * Hq * hd * 2);
+    g.o_blk = take(rb * Hq * hd * 2);
+    g.f_blk = take(rb * F * 2);
+    g.xn = take(rb * D * 2);
+    g.conf = take(rb * 4);
+    g.tok = take(rb * 4);
+    g.masked = take(rf);
+    g.counts = take((size_t)2 * b * 4);
+    g.maps = take((size_t)nblk * rb * 4);
+    g.rope = take((size_t)L * hd * 4);
+    g.lm_bytes = lm_bytes;
+    g.lm_ws = take(lm_bytes);
+    g.total = off;
+    return g;
+}
+
+bool model_desc_ok(const fdl_model_desc* d) {
+    return d && d->vocab >= 2 && d->hidden >= 128 && d->hidden % 128 == 0 && d->n_layers >= 1 &&
+           d->n_kv_heads >= 1 && d->n_q_heads >= d->n_kv_heads &&
+           d->n_q_heads % d->n_kv_heads == 0 && d->head_dim == 128 && d->ffn >= 64 &&
+           d->ffn % 64 == 0 && d->mask_id >= 0 && d->mask_id < d->vocab && d->rope_theta > 0.f &&
+           d->rms_eps > 0.f;
+}
+
+size_t lm_ws_bytes(fdl_ctx* ctx, const fdl_model_desc& d, int rows) {
+    const fdl_lmhead_desc ld{rows, d.hidden, d.vocab, FDL_BF16};
+    const size_t n = fdl_lmhead_workspace_bytes(ctx, &ld);
+    return n > 16 ? n : 16;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fdl_model_create(const fdl_model_desc* desc, const fdl_model_weights* w, fdl_model** out) {
+    if (!out) return fail(FDL_EINVAL, "model_create: out is NULL");
+    *out = nullptr;
+    if (!model_desc_ok(desc))
+        return fail(FDL_EINVAL, "model_create: bad description (hidden a multiple of 128, "
+                    "head_dim 128, Hq a multiple of Hkv, ffn a multiple of 64, 0 <= mask_id < "
+                    "vocab, rope_theta and rms_eps > 0)");
+    if (!w || !w->embed || !w->final_norm || !w->lm_head || !w->layers)
+        return fail(FDL_EINVAL, "model_create: NULL weight pointer");
+    if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->lm_head))
+        return fail(FDL_EINVAL, "model_create: weights must be 16-byte aligned");
+    fdl_model* m = new fdl_model;
+    m->d = *desc;
+    m->embed = w->embed;
+    m->final_norm = w->final_norm;
+    m->lm_head = w->lm_head;
+    m->layers.assign(w->layers, w->layers + desc->n_layers);
+    for (int l = 0; l < desc->n_layers; ++l) {
+        const fdl_layer_weights& L = m->layers[l];
+        if (!L.attn_norm || !L.w_qkv || !L.wo || !L.ffn_norm || !L.w_gu || !L.w_down ||
+            !aligned16(L.attn_norm) || !aligned16(L.w_qkv) || !aligned16(L.wo) ||
+            !aligned16(L.ffn_norm) || !aligned16(L.w_gu) || !aligned16(L.w_down) ||
+            (L.bias && !aligned16(L.bias))) {
+            delete m;
+            return fail(FDL_EINVAL, "model_create: layer %d: NULL or unaligned weight", l);
+        }
+    }
+    *out = m;
+    return FDL_OK;
+}
+
+int fdl_model_destroy(fdl_model* model) {
+    delete model;
+    return FDL_OK;
+}
+
+size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* m, int batch, int seq_len,
+                                    int block) {
+    if (!ctx || !m || batch < 1 || seq_len < 1 || block < 1 || block > 128) return 0;
+    return gen_layout(m->d, batch, seq_len, block, lm_ws_bytes(ctx, m->d, batch * block)).total;
+}
+
+int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b, int P, int gen,
+                 int B, float tau, int32_t* x, int* steps_out, void* ws, size_t ws_bytes,
+                 void* stream) {
+    if (!ctx || !m) return fail(FDL_EINVAL, "generate: ctx or model is NULL");
+    if (!prompt || !x || !steps_out) return fail(FDL_EINVAL, "generate: NULL buffer");
+    if (b < 1 || B < 1 || B > 128 || P < 0 || gen < B || P % B || gen % B)
+        return fail(FDL_EINVAL, "generate: need batch >= 1, 1 <= block <= 128, prompt_len and "
+                    "gen_len (>= block) multiples of block");
+    if (!(tau >= 0.f && tau <= 1.f)) return fail(FDL_EINVAL, "generate: tau must be in [0, 1]");
+    const fdl_model_desc& d = m->d;
+    const int L = P + gen, D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads;
+    const int hd = 128, rf = b * L, rb = b * B;
+    const GenLayout g = gen_layout(d, b, L, B, lm_ws_bytes(ctx, d, rb));
+    if (!ws || ws_bytes < g.total)
+        return fail(FDL_EWORKSPACE, "generate: workspace of %zu bytes needed", g.total);
+    if (((uintptr_t)ws & 255u) != 0) return fail(FDL_EINVAL, "generate: ws must be 256-byte aligned");
+    DeviceGuard guard(ctx->device);
+    cudaStream_t st = (cudaStream_t)stream;
+    char* base = static_cast<char*>(ws);
+    auto at = [&](size_t off) { return static_cast<void*>(base + off); };
+    char* kc = base + g.kc;
+    char* vc = base + g.vc;
+    float* h_full = (float*)at(g.h_full);
+    float* h_blk = (float*)at(g.h_blk);
+    float* conf = (float*)at(g.conf);
+    int32_t* tok = (int32_t*)at(g.tok);
+    uint8_t* masked = (uint8_t*)at(g.masked);
+    int32_t* remaining = (int32_t*)at(g.counts);
+    int32_t* n_decoded = remaining + b;
+    int32_t* maps = (int32_t*)at(g.maps);
+    float* rope = (float*)at(g.rope);
+    const int nblk = (L + B - 1) / B;
+
+    // state: x = prompts then mask ids, masked = the generated positions
+    cudaError_t e = cudaSuccess;
+    fill_i32_kernel<<<148, 256, 0, st>>>(x, (size_t)rf, d.mask_id);
+    if (e == cudaSuccess && P > 0)
+        e = cudaMemcpy2DAsync(x, (size_t)L * 4, prompt, (size_t)P * 4, (size_t)P * 4, b,
+                              cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(masked, 0, (size_t)rf, st);
+    if (e == cudaSuccess)
+        e = cudaMemset2DAsync(masked + P, (size_t)L, 1, (size_t)gen, b, st);
+    block_rows_kernel<<<64, 256, 0, st>>>(maps, b, L, B, nblk);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    {
+        std::vector<float> host_rope((size_t)L * hd);
+        int rc = fdl_rope_table((double)d.rope_theta, L, hd, host_rope.data());
+        if (rc) return rc;
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(rope, host_rope.data(), host_rope.size() * 4,
+                                cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);   // host_rope goes out of scope
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "generate: set-up");
+
+    const fdl_lmhead_desc lmd{rb, D, d.vocab, FDL_BF16};
+    auto layers = [&](float* h, void* xb, void* q, void* o, void* f, int rows, bool full,
+                      int s) -> int {
+        int rc = FDL_OK;
+        for (int li = 0; li < d.n_layers && rc == FDL_OK; ++li) {
+            const fdl_layer_weights& W = m->layers[li];
+            void* kl = kc + g.kv_layer * li;
+            void* vl = vc + g.kv_layer * li;
+            if (full) {
+                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, L, 0, L};
+                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, 0, 1, FDL_BF16, 0.f};
+                rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
+                if (!rc) rc = fdl_qkv_rope_store(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl, vl,
+                                                 stream);
+                if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
+            } else {
+                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, B, s, L};
+                rc = fdl_qkv_attention(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv, W.bias,
+                                       rope, q, kl, vl, o, stream);
+            }
+            if (!rc) rc = fdl_linear_residual(ctx, rows, D, Hq * hd, o, W.wo, h, stream);
+            if (!rc) rc = fdl_ffn(ctx, rows, D, F, W.ffn_norm, d.rms_eps, xb, W.w_gu, W.w_down, f,
+                                  h, stream);
+        }
+        return rc;
+    };
+
+    std::vector<int32_t> host_rem(b);
+    int steps = 0;
+    for (int blk = 0; blk < gen / B; ++blk) {
+        const int s = P + blk * B;
+        const int32_t* row_map = maps + (size_t)(s / B) * rb;
+        for (bool refresh = true;; refresh = false) {
+            int rc;
+            if (refresh) {
+                // full forward over every position: all K/V caches rewritten
+                rc = fdl_embed(ctx, rf, D, x, nullptr, m->embed, h_full, stream);
+                if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full),
+                                     at(g.f_full), rf, true, 0);
+                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, row_map, m->final_norm, d.rms_eps,
+                                          at(g.xn), stream);
+            } else {
+                // cached step: only the block's rows
+                rc = fdl_embed(ctx, rb, D, x, row_map, m->embed, h_blk, stream);
+                if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), rb,
+                                     false, s);
+                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_blk, nullptr, m->final_norm, d.rms_eps,
+                                          at(g.xn), stream);
+            }
+            if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head, nullptr, nullptr,
+                                                conf, tok, at(g.lm_ws), g.lm_bytes, stream);
+            const fdl_unmask_desc ud{b, L, s, B, tau};
+            if (!rc) rc = fdl_threshold_unmask(ctx, &ud, conf, tok, x, masked, remaining, n_decoded,
+                                               stream);
+            if (rc) return rc;
+            ++steps;
+            e = cudaMemcpyAsync(host_rem.data(), remaining, (size_t)b * 4, cudaMemcpyDeviceToHost,
+                                st);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) return cuda_fail(e, "generate: counters");
+            int rem = 0;
+            for (int i = 0; i < b; ++i) rem = host_rem[i] > rem ? host_rem[i] : rem;
+            if (rem == 0) break;
+        }
+    }
+    *steps_out = steps;
+    return FDL_OK;
 }
 
 }  // extern "C"

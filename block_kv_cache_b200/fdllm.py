@@ -29,7 +29,8 @@ EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
            "fdl_lmhead_confidence", "fdl_threshold_unmask",
            "fdl_lmhead_confidence_noalloc", "fdl_rope_table", "fdl_rmsnorm", "fdl_embed",
            "fdl_qkv_rope_store", "fdl_linear_residual", "fdl_linear_swiglu",
-           "fdl_full_attention", "fdl_ffn", "fdl_qkv_attention")
+           "fdl_full_attention", "fdl_ffn", "fdl_qkv_attention", "fdl_model_create",
+           "fdl_model_destroy", "fdl_generate_workspace_bytes", "fdl_generate")
 
 
 class AttnDesc(ctypes.Structure):
@@ -40,7 +41,7 @@ class AttnDesc(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 
 
 class LMHeadDesc(ctypes.Structure):
@@ -60,6 +61,25 @@ class QKVDesc(ctypes.Structure):
                 ("batch", ctypes.c_int), ("seq_len", ctypes.c_int),
                 ("rows_per_seq", ctypes.c_int), ("pos0", ctypes.c_int),
                 ("max_pos", ctypes.c_int)]
+
+
+class ModelDesc(ctypes.Structure):
+    _fields_ = [("vocab", ctypes.c_int), ("hidden", ctypes.c_int), ("n_layers", ctypes.c_int),
+                ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("ffn", ctypes.c_int), ("mask_id", ctypes.c_int),
+                ("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("attn_norm", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("wo", ctypes.c_void_p),
+                ("ffn_norm", ctypes.c_void_p), ("w_gu", ctypes.c_void_p),
+                ("w_down", ctypes.c_void_p)]
+
+
+class ModelWeights(ctypes.Structure):
+    _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+                ("lm_head", ctypes.c_void_p), ("layers", ctypes.POINTER(LayerWeights))]
 
 
 class FdlError(RuntimeError):
@@ -112,6 +132,12 @@ def load() -> ctypes.CDLL:
     L.fdl_ffn.argtypes = [vp, i, i, i, vp, fl, vp, vp, vp, vp, vp, vp]
     L.fdl_qkv_attention.argtypes = [vp, ctypes.POINTER(QKVDesc), vp, vp, fl, vp, vp, vp, vp, vp,
                                     vp, vp, vp, vp]
+    L.fdl_model_create.argtypes = [ctypes.POINTER(ModelDesc), ctypes.POINTER(ModelWeights),
+                                   ctypes.POINTER(vp)]
+    L.fdl_model_destroy.argtypes = [vp]
+    L.fdl_generate_workspace_bytes.argtypes = [vp, vp, i, i, i]
+    L.fdl_generate_workspace_bytes.restype = sz
+    L.fdl_generate.argtypes = [vp, vp, vp, i, i, i, i, fl, vp, ctypes.POINTER(i), vp, sz, vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -159,6 +185,41 @@ def rope_table(theta: float, max_pos: int, head_dim: int):
     _check(load().fdl_rope_table(float(theta), int(max_pos), int(head_dim),
                                  ctypes.c_void_p(out.ctypes.data)))
     return out
+
+
+class Model:
+    """A model recorded in the library (fdl_model_create): the description and
+    the device pointers of the weights, which the caller keeps alive.
+    `layers` holds per layer the tensors attn_norm, w_qkv, bias (or None), wo,
+    ffn_norm, w_gu, wd."""
+
+    def __init__(self, *, vocab, hidden, n_q_heads, n_kv_heads, ffn, mask_id, embed,
+                 final_norm, lm_head, layers, head_dim=128, rope_theta=10000.0, rms_eps=1e-5):
+        L = load()
+        self._keep = (embed, final_norm, lm_head, layers)
+        self.desc = ModelDesc(vocab, hidden, len(layers), n_q_heads, n_kv_heads, head_dim, ffn,
+                              mask_id, rope_theta, rms_eps)
+        arr = (LayerWeights * len(layers))()
+        for k, Lw in enumerate(layers):
+            arr[k] = LayerWeights(Lw["attn_norm"].data_ptr(), Lw["w_qkv"].data_ptr(),
+                                  Lw["bias"].data_ptr() if Lw.get("bias") is not None else None,
+                                  Lw["wo"].data_ptr(), Lw["ffn_norm"].data_ptr(),
+                                  Lw["w_gu"].data_ptr(), Lw["wd"].data_ptr())
+        w = ModelWeights(embed.data_ptr(), final_norm.data_ptr(), lm_head.data_ptr(), arr)
+        h = ctypes.c_void_p()
+        _check(L.fdl_model_create(ctypes.byref(self.desc), ctypes.byref(w), ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            load().fdl_model_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 class Context:
@@ -352,6 +413,23 @@ class Context:
                                         _ptr(q_out), _ptr(k_cache), _ptr(v_cache), _ptr(out),
                                         _stream(stream)))
         return out
+
+    def generate(self, model: Model, prompt, gen_len, *, block=32, tau=0.9, stream=None):
+        """The whole DualCache decode in the library (fdl_generate): prompt
+        [b, P] int32 CUDA tensor. Returns (x [b, P + gen_len] int32, steps)."""
+        _need(prompt, "prompt", torch.int32, 2)
+        b, P = prompt.shape
+        L = load()
+        n = L.fdl_generate_workspace_bytes(self._h, model._h, b, P + gen_len, int(block))
+        if n == 0:
+            raise ValueError("generate: bad shape")
+        ws = torch.empty(n, dtype=torch.uint8, device=prompt.device)
+        x = torch.empty((b, P + gen_len), dtype=torch.int32, device=prompt.device)
+        steps = ctypes.c_int(0)
+        _check(L.fdl_generate(self._h, model._h, _ptr(prompt), b, P, int(gen_len), int(block),
+                              float(tau), _ptr(x), ctypes.byref(steps), _ptr(ws), n,
+                              _stream(stream)))
+        return x, steps.value
 
     def linear_residual(self, x, w, h, *, stream=None):
         """h += x w^T (h f32)."""

@@ -131,6 +131,16 @@ class DeviceWeights:
         return DeviceWeights(shape, layers, embed, torch.ones(D, device=device),
                              rnd(shape.vocab, D))
 
+    def native(self) -> "fdllm.Model":
+        """These weights recorded in the library, for Context.generate (the
+        whole decode loop in native code)."""
+        sh = self.shape
+        return fdllm.Model(vocab=sh.vocab, hidden=sh.hidden, n_q_heads=sh.n_q_heads,
+                           n_kv_heads=sh.n_kv_heads, ffn=sh.ffn, mask_id=sh.mask_id,
+                           embed=self.embed, final_norm=self.final_norm, lm_head=self.lm_head,
+                           layers=self.layers, head_dim=sh.head_dim, rope_theta=sh.rope_theta,
+                           rms_eps=sh.rms_eps)
+
     def nbytes(self) -> int:
         n = self.embed.numel() * 2 + self.lm_head.numel() * 2
         for L in self.layers:

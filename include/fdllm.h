@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define FDL_ABI_VERSION 2
+#define FDL_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define FDL_API __attribute__((visibility("default")))
@@ -362,6 +362,87 @@ FDL_API int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const float* no
 FDL_API int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
                                const void* k_cache, const void* v_cache, void* out,
                                void* stream);
+
+/* ---- the whole decode: DualCache block decoding with the threshold rule ----
+ * Fast-dLLM (README "Key techniques" 1 and 2; aibase news "Innovations" 1
+ * and 2): the generated part is split into blocks of `block` positions,
+ * decoded left to right. A block starts with a full bidirectional forward
+ * over all positions (it rewrites every layer's K/V cache, and its logits
+ * serve the block's first step); then cached steps recompute only the
+ * block's rows, attending over [prefix | block | suffix] of the cache, until
+ * no position of the block is masked. Each step unmasks the masked positions
+ * of the block whose confidence exceeds tau, or the single most confident
+ * one (lowest position on ties), as fdl_threshold_unmask. The model is a
+ * pre-norm bidirectional transformer: x = RMSNorm(h); q/k/v (+ bias), RoPE;
+ * attention; h += o W_o^T; x = RMSNorm(h); h += (silu(x W_g^T) * (x W_u^T))
+ * W_d^T; final RMSNorm; LM head. */
+typedef struct {
+    int vocab;        /* V >= 2 */
+    int hidden;       /* D, multiple of 128 */
+    int n_layers;     /* >= 1 */
+    int n_q_heads;    /* Hq, multiple of n_kv_heads */
+    int n_kv_heads;   /* Hkv >= 1 */
+    int head_dim;     /* 128 */
+    int ffn;          /* F, multiple of 64 */
+    int mask_id;      /* token id of a masked position, in [0, V) */
+    float rope_theta; /* > 0 */
+    float rms_eps;    /* > 0 */
+} fdl_model_desc;
+
+/* Device pointers of one layer, owned by the caller; every matrix K-major. */
+typedef struct {
+    const float* attn_norm;  /* f32 [D] */
+    const void* w_qkv;       /* bf16 [(Hq + 2 Hkv) * 128, D]: q rows, then k, then v */
+    const float* bias;       /* f32 [(Hq + 2 Hkv) * 128] or NULL */
+    const void* wo;          /* bf16 [D, Hq * 128] */
+    const float* ffn_norm;   /* f32 [D] */
+    const void* w_gu;        /* bf16 [2F, D], gate and up rows interleaved (2f, 2f + 1) */
+    const void* w_down;      /* bf16 [D, F] */
+} fdl_layer_weights;
+
+typedef struct {
+    const void* embed;                /* bf16 [V, D] */
+    const float* final_norm;          /* f32 [D] */
+    const void* lm_head;              /* bf16 [V, D] */
+    const fdl_layer_weights* layers;  /* host array of n_layers (copied by create) */
+} fdl_model_weights;
+
+typedef struct fdl_model fdl_model;   /* the description and the weight pointers */
+
+/* Record a model: copies the description and the pointers (host memory
+ * only; the weights stay the caller's and must outlive the model). Checks
+ * shapes, alignment (16 bytes) and non-NULL pointers. *out is NULL on failure.
+ * Errors: FDL_EINVAL. */
+FDL_API int fdl_model_create(const fdl_model_desc* desc, const fdl_model_weights* weights,
+                             fdl_model** out);
+FDL_API int fdl_model_destroy(fdl_model* model);
+
+/* Device workspace of fdl_generate for `batch` sequences of length seq_len
+ * in blocks of `block` positions: every layer's K/V cache (2 * layers * batch
+ * * Hkv * seq_len * 128 bf16), the activations of a full forward and of a
+ * block step, the LM-head scratch, the mask state and the rotary table. 0 on
+ * bad arguments. */
+FDL_API size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* model, int batch,
+                                            int seq_len, int block);
+
+/* Decode gen_len positions after the prompts of `batch` sequences.
+ *   prompt  [batch, prompt_len] int32 device (token ids)
+ *   out_x   [batch, prompt_len + gen_len] int32 device (written: the prompts,
+ *           then the decoded tokens)
+ *   block   positions per block, 1..128; prompt_len and gen_len multiples of it
+ *   tau     threshold in [0, 1]
+ *   *steps_out (host) the decode steps taken (refresh steps included)
+ *   ws      device workspace of fdl_generate_workspace_bytes bytes
+ * Every step reads `batch` 4-byte counters back to the host to decide
+ * between the next cached step and the next block; the call returns when the
+ * decode is complete (the stream is synchronised). The kernels and their
+ * order are those of the per-call functions above (fdl_embed, fdl_rmsnorm,
+ * fdl_qkv_rope_store, fdl_full_attention, fdl_qkv_attention,
+ * fdl_linear_residual, fdl_ffn, fdl_lmhead_confidence, fdl_threshold_unmask).
+ * Errors: FDL_EINVAL, FDL_EWORKSPACE, FDL_ECUDA, or those of the calls. */
+FDL_API int fdl_generate(fdl_ctx* ctx, const fdl_model* model, const int32_t* prompt, int batch,
+                         int prompt_len, int gen_len, int block, float tau, int32_t* out_x,
+                         int* steps_out, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -268,6 +268,50 @@ def test_decode_matches_oracle_step_by_step(ctx, seed, tau, hq, hkv, bias):
     _replay_check(P, rec, xf, B, tau)
 
 
+@pytest.mark.parametrize("seed,tau,hq,hkv,bias", [(0, 0.9, 2, 2, False), (1, 0.5, 4, 2, True),
+                                                  (2, 1.0, 2, 1, False)])
+def test_native_generate_equals_the_python_decoder(ctx, seed, tau, hq, hkv, bias):
+    """fdl_generate (the decode loop in the library) takes the same steps and
+    decodes the same tokens as the Python decoder above, whose trajectory the
+    oracle replays (same kernels in the same order; at these shapes no
+    projection splits K, so both runs are bit-identical)."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(seed, hq=hq, hkv=hkv, bias=bias)
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B = 2, 64, 64, 32
+    prompt = synth.prompt_ids(seed, b, Lp, P.mask_id)
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B)
+    x_py, steps_py = dec.generate(prompt, gen, tau=tau)
+    x_nat, steps_nat = ctx.generate(w.native(), torch.from_numpy(prompt).cuda(), gen, block=B,
+                                    tau=tau)
+    ctx.device_status()
+    assert steps_nat == steps_py
+    assert np.array_equal(x_nat.cpu().numpy(), x_py.cpu().numpy())
+
+
+def test_native_generate_fused_shapes(ctx):
+    """fdl_generate on shapes that take the fused split-K calls (hidden 1024,
+    GQA 8/2 with bias): the prompt is kept, every position is decoded, tau = 1
+    decodes exactly one position per step, and bad arguments are rejected."""
+    from block_kv_cache_b200 import fdllm
+    from block_kv_cache_b200.model import DeviceWeights, ModelShape
+    sh = ModelShape(4096, 1024, 2, 8, 2, 1024, 4095, 128, qkv_bias=True)
+    w = DeviceWeights.random(sh, seed=5)
+    b, Lp, gen, B = 3, 96, 64, 32
+    prompt = torch.from_numpy(synth.prompt_ids(9, b, Lp, sh.mask_id)).cuda()
+    m = w.native()
+    x, steps = ctx.generate(m, prompt, gen, block=B, tau=1.0)
+    ctx.device_status()
+    assert steps == gen                                         # one position per step
+    xh = x.cpu().numpy()
+    assert np.array_equal(xh[:, :Lp], prompt.cpu().numpy())
+    assert xh.min() >= 0 and xh.max() < sh.vocab
+    with pytest.raises(fdllm.FdlError):
+        ctx.generate(m, prompt, 48, block=B)                    # gen not a multiple of block
+    with pytest.raises(fdllm.FdlError):
+        ctx.generate(m, prompt[:, :Lp - 8].contiguous(), gen, block=B)   # prompt not either
+
+
 def test_tau_one_single_layer_gpu_equals_sequential(ctx):
     """tau = 1 and one layer: the GPU's DualCache decode equals sequential
     greedy decoding of the oracle wherever the oracle's choices are not
