@@ -10,15 +10,20 @@
 // head chunk) and a contiguous range ("split") of 64-key tiles streamed
 // through a TMA ring, so every K/V byte is read from HBM once. The splits of
 // one (sequence, kv head, chunk) form a thread-block cluster and merge their
-// partial softmaxes through distributed shared memory; the cluster writes the
-// final bf16 output and LSE, with no second pass over memory.
+// partial softmaxes on chip: with one 128-row tile each split pushes its
+// partial rows into the receive buffer of the CTA that owns them (st.async,
+// counted in bytes on the owner's mbarrier); otherwise the owners pull them
+// through distributed shared memory between two cluster barriers. The owners
+// write the final bf16 output and LSE, with no second pass over memory.
 //
 // The 128 TMEM lanes are the MMA's M dimension: R <= 128 packed rows use one
 // 128-row tile, R in (128, 256] two, each with its own softmax warpgroup. A
 // softmax warp reads only its own 32-lane quarter of TMEM; warps whose rows
 // are all padding sit out. (With one block of 32 queries per head, one warp
-// per tile does the softmax: 64 exponentials per tile per thread, less than
-// the time a 64-key tile takes to arrive at this SM's share of HBM bandwidth.)
+// per tile does the softmax: 64 exponentials and bf16 packs per thread, about
+// 1240 of the ~1550 cycles a 64-key tile takes on this B200 at L = 2048;
+// replicating the query rows into all four lane quarters, each warp taking a
+// quarter of the keys, measured slower.)
 //
 //   softmax warps (4 per 128-row tile): thread = TMEM lane; online softmax in
 //       the log2 domain (scale*log2 e folded into one FFMA); P(t) as bf16 into
