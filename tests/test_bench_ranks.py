@@ -53,3 +53,24 @@ def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.combine_ranks(None, 1, 12.5, 7, "cpu") == (12.5, 7.0)
+
+
+def test_bench_configs_are_complete_and_switchable():
+    """Both workloads carry every field the decoder and the bench read, and
+    the model shape follows the selected one."""
+    import bench
+    keys = {"layers", "hidden", "heads", "kv_heads", "head_dim", "ffn", "vocab", "mask_id",
+            "batch", "prompt", "gen", "block", "tau", "qkv_bias", "workload"}
+    for name, c in bench.CONFIGS.items():
+        assert keys <= set(c), name
+        assert c["heads"] % c["kv_heads"] == 0 and 0 <= c["mask_id"] < c["vocab"]
+        assert c["prompt"] % c["block"] == 0 and c["gen"] % c["block"] == 0
+    saved = dict(bench.CFG)
+    try:
+        bench.CFG.clear()
+        bench.CFG.update(bench.CONFIGS["dream"])
+        sh = bench.shape()
+        assert (sh.n_layers, sh.hidden, sh.n_kv_heads, sh.qkv_bias) == (28, 3584, 4, True)
+    finally:
+        bench.CFG.clear()
+        bench.CFG.update(saved)
