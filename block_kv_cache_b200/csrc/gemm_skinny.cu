@@ -176,8 +176,6 @@ struct SkAccum {
 // ---- prologues: work every CTA does after the preceding kernel, before the GEMM --
 struct NoPro {
     static constexpr bool kActive = false;
-    unsigned* bar = nullptr;
-    __device__ void work(int, int) const {}
 };
 
 // The SwiGLU of a split-K gate/up projection, done by the CTAs of the GEMM that
