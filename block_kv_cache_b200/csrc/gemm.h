@@ -64,7 +64,7 @@ struct NormIn {
 // epilogue is then up to the caller: launch_qkv_attention_bf16).
 int skinny_qkv_splits(const GemmShape& g, size_t acc_bytes, int sm_count);
 // With norm, the projection's CTAs first write x = RMSNorm(h) (grid barrier
-// on the two words at bar).
+// on the 64-bit counter at bar).
 cudaError_t launch_skinny_qkv_sums(const GemmShape& g, const void* x, const void* w, float* acc,
                                    int splits, const NormIn* norm, unsigned* bar, int sm_count,
                                    int* err, cudaStream_t st);
