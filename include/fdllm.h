@@ -18,7 +18,9 @@
  *    frees them; scratch memory is passed in by the caller (`ws`), sized by
  *    the matching *_workspace_bytes query.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). Every compute
- *    call is asynchronous on that stream: it returns after enqueueing.
+ *    call is asynchronous on that stream: it returns after enqueueing. The
+ *    exception is fdl_generate, whose decode loop reads a few counters back
+ *    after every step and returns when the decode is complete.
  *  - Return value: FDL_OK (0) or a negative fdl_status. Argument errors are
  *    detected on the host before anything is enqueued, so nothing runs on an
  *    error return. fdl_last_error() gives a message for the calling thread's
@@ -66,7 +68,7 @@ typedef struct fdl_ctx fdl_ctx;   /* opaque: device id, device error word, launc
 FDL_API int fdl_abi_version(void);
 
 /* Create a context on CUDA device `device`. Allocates, once, here (the only
- * allocations the library makes): the 4-byte device error word, a 32 MiB
+ * device allocations the library makes): the 4-byte device error word, a 32 MiB
  * zero-filled f32 accumulator used by the few-token projections to add
  * split-K partial sums (every kernel that adds into it leaves it zeroed), and
  * 256 zeroed bytes for the grid-wide barriers of fused kernels. After a call
@@ -77,7 +79,7 @@ FDL_API int fdl_abi_version(void);
  * is compute capability 10.0 (B200). *out is set to NULL on failure. */
 FDL_API int fdl_create(fdl_ctx** out, int device);
 
-/* Free the context and its error word. NULL is accepted. */
+/* Free the context and its device buffers. NULL is accepted. */
 FDL_API int fdl_destroy(fdl_ctx* ctx);
 
 /* Message for the calling thread's last non-OK return ("" if none). The
