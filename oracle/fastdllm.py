@@ -292,14 +292,21 @@ def _layer_rest(P, Lw, h, o):
     return h + (silu(g) * u) @ _f64(Lw["wd"]).T
 
 
-def full_forward(P, ids):
+def _embed_rows(P, ids):
+    """f64 embedding rows of `ids` (the rows are picked before widening: the
+    values are the same, the table is not copied)."""
+    return _f64(np.asarray(P.embed)[np.asarray(ids)])
+
+
+def full_hidden(P, ids):
     """No-cache forward of one sequence ids [L]: every position attends to
     every position ([news], "Challenges": without a cache all attention
     states are recomputed at every step).
-    Returns logits [L, V] and per-layer (k, v) as [Hkv, L, d]."""
+    Returns the final-norm hidden rows [L, D] and per-layer (k, v) as
+    [Hkv, L, d]."""
     L = len(ids)
     pos = np.arange(L)
-    h = _f64(P.embed)[np.asarray(ids)]
+    h = _embed_rows(P, ids)
     kv = []
     for Lw in P.layers:
         hn = rms_norm(h, Lw["attn_norm"], P.rms_eps)
@@ -308,20 +315,26 @@ def full_forward(P, ids):
         kv.append((kt.copy(), vt.copy()))
         o, _ = attention(q, kt, vt)
         h = _layer_rest(P, Lw, h, o)
-    hf = rms_norm(h, P.final_norm, P.rms_eps)
-    return hf @ _f64(P.lm_head).T, kv
+    return rms_norm(h, P.final_norm, P.rms_eps), kv
 
 
-def block_forward(P, blk_ids, block_start, caches):
+def full_forward(P, ids):
+    """full_hidden followed by the LM head: logits [L, V] and the per-layer
+    (k, v)."""
+    hf, kv = full_hidden(P, ids)
+    return lm_logits(hf, P.lm_head), kv
+
+
+def block_hidden(P, blk_ids, block_start, caches):
     """DualCache step of one sequence: only the block's tokens go through the
     layers; at each layer their fresh K/V overwrite the cache's block slot and
     the block attends over the whole cache ([news], Innovations 1: prefix and
     suffix K/V are reused from the cache; [readme], Key techniques 1).
     caches: list of (k, v) [Hkv, L, d] per layer, updated in place.
-    Returns logits [B, V] for the block's rows."""
+    Returns the final-norm hidden rows [B, D] of the block."""
     B = len(blk_ids)
     pos = np.arange(block_start, block_start + B)
-    h = _f64(P.embed)[np.asarray(blk_ids)]
+    h = _embed_rows(P, blk_ids)
     for Lw, (kc, vc) in zip(P.layers, caches):
         hn = rms_norm(h, Lw["attn_norm"], P.rms_eps)
         q, k, v = _layer_qkv(P, Lw, hn, pos)
@@ -329,8 +342,43 @@ def block_forward(P, blk_ids, block_start, caches):
         vc[:, block_start:block_start + B, :] = np.transpose(v, (1, 0, 2))
         o, _ = attention(q, kc, vc)
         h = _layer_rest(P, Lw, h, o)
-    hf = rms_norm(h, P.final_norm, P.rms_eps)
-    return hf @ _f64(P.lm_head).T
+    return rms_norm(h, P.final_norm, P.rms_eps)
+
+
+def block_forward(P, blk_ids, block_start, caches):
+    """block_hidden followed by the LM head: logits [B, V] of the block rows."""
+    return lm_logits(block_hidden(P, blk_ids, block_start, caches), P.lm_head)
+
+
+def prefix_hidden(P, tail_ids, start, caches):
+    """PrefixCache step of one sequence (the cache without the DualCache
+    extension: [readme], usage flags --use_cache without
+    --if_cache_position; [news], Innovations 1 describes DualCache as the
+    version that also caches the suffix). Only the prefix [0, start) is
+    taken from the cache: every position from the block start to the end
+    (the block and the masked suffix, tail_ids [L - start]) goes through the
+    layers, its fresh K/V overwrite cache rows [start, L), and those rows
+    attend over the whole cache [cached prefix | fresh block and suffix].
+    caches: list of (k, v) [Hkv, L, d] per layer, updated in place.
+    Returns the final-norm hidden rows [L - start, D]; the block's are the
+    first B of them."""
+    n = len(tail_ids)
+    pos = np.arange(start, start + n)
+    h = _embed_rows(P, tail_ids)
+    for Lw, (kc, vc) in zip(P.layers, caches):
+        assert kc.shape[1] == start + n
+        hn = rms_norm(h, Lw["attn_norm"], P.rms_eps)
+        q, k, v = _layer_qkv(P, Lw, hn, pos)
+        kc[:, start:, :] = np.transpose(k, (1, 0, 2))
+        vc[:, start:, :] = np.transpose(v, (1, 0, 2))
+        o, _ = attention(q, kc, vc)
+        h = _layer_rest(P, Lw, h, o)
+    return rms_norm(h, P.final_norm, P.rms_eps)
+
+
+def prefix_forward(P, tail_ids, start, caches):
+    """prefix_hidden followed by the LM head: logits [L - start, V]."""
+    return lm_logits(prefix_hidden(P, tail_ids, start, caches), P.lm_head)
 
 
 # ---------------------------------------------------------------------------
@@ -358,9 +406,9 @@ def _step_select(x, masked, logits_blk, s, B, tau):
 
 
 def generate_dualcache(P, prompt, gen_len, block=32, tau=0.9,
-                       refresh_every_step=False) -> DecodeTrace:
-    """Fast-dLLM block decoding of one sequence with DualCache and the
-    confidence-aware threshold rule.
+                       refresh_every_step=False, cache="dual") -> DecodeTrace:
+    """Fast-dLLM block decoding of one sequence with a block-wise K/V cache
+    and the confidence-aware threshold rule.
 
     The generated region (gen_len mask tokens after the prompt) is split into
     blocks of `block` positions, decoded left to right ([news], Innovations 1;
@@ -369,8 +417,12 @@ def generate_dualcache(P, prompt, gen_len, block=32, tau=0.9,
     first step; then cached block steps run until the block has no masked
     position; after the block completes the next block's refresh rewrites all
     K/V ([reviews], review 4 question 2). No refresh follows the last block.
+    cache="dual": a cached step recomputes only the block and reuses the
+    cached prefix and masked-suffix K/V (DualCache, block_forward);
+    cache="prefix": it recomputes the block and the suffix and reuses the
+    cached prefix only (prefix_forward).
     With refresh_every_step the cache is rebuilt before every step."""
-    assert gen_len % block == 0
+    assert gen_len % block == 0 and cache in ("dual", "prefix")
     Lp = len(prompt)
     x = np.concatenate([np.asarray(prompt), np.full(gen_len, P.mask_id)]).astype(np.int64)
     masked = np.zeros(len(x), np.int8)
@@ -389,14 +441,21 @@ def generate_dualcache(P, prompt, gen_len, block=32, tau=0.9,
                 logits, kv = full_forward(P, x)
                 tr.refreshes += 1
                 lg = logits[s:s + block]
-            else:
+            elif cache == "dual":
                 lg = block_forward(P, x[s:s + block], s, caches)
+            else:
+                lg = prefix_forward(P, x[s:], s, caches)[:block]
             dec = _step_select(x, masked, lg, s, block, tau)
             assert len(dec) >= 1
             tr.steps += 1
             tr.per_step.append((blk, dec))
     tr.x = x
     return tr
+
+
+def generate_prefixcache(P, prompt, gen_len, block=32, tau=0.9) -> DecodeTrace:
+    """Block decoding with the PrefixCache: generate_dualcache(cache="prefix")."""
+    return generate_dualcache(P, prompt, gen_len, block, tau, cache="prefix")
 
 
 def generate_nocache(P, prompt, gen_len, block=32, tau=0.9) -> DecodeTrace:

@@ -381,3 +381,65 @@ def test_parallel_decode_progress_and_blocks_left_to_right():
     assert all(v <= 8 for v in per_blk.values())
     assert tr.refreshes == 4
     assert tr.steps < 32          # some steps decoded more than one token
+
+
+# ---------------------------------------------------------------- PrefixCache
+def test_prefix_step_equals_full_forward_when_cache_current():
+    """With the cache holding the K/V of the current sequence, the PrefixCache
+    step (block and suffix recomputed over the cached prefix) reproduces the
+    full bidirectional forward on every row from the block start on, for any
+    depth, and leaves the cache as the full forward computed it."""
+    for n_layers, kvh, bias in [(1, 4, False), (3, 2, True)]:
+        P = synth.model_params(vocab=64, hidden=32, n_layers=n_layers, n_q_heads=4,
+                               n_kv_heads=kvh, head_dim=8, ffn=48, seed=20 + n_layers,
+                               qkv_bias=bias)
+        x = synth.rng(13).integers(0, 63, 40)
+        x[20:] = P.mask_id
+        x[27] = 9
+        logits, kv = O.full_forward(P, x)
+        caches = [(k.copy(), v.copy()) for k, v in kv]
+        lp = O.prefix_forward(P, x[16:], 16, caches)
+        assert lp.shape == (24, 64)
+        np.testing.assert_allclose(lp, logits[16:], rtol=1e-10, atol=1e-10)
+        for (k, v), (kc, vc) in zip(kv, caches):
+            np.testing.assert_allclose(kc, k, atol=1e-12)
+            np.testing.assert_allclose(vc, v, atol=1e-12)
+
+
+def test_prefix_step_reads_only_the_prefix_cache():
+    """The PrefixCache step attends over the cached prefix (perturbing a
+    prefix row changes the block's logits) and recomputes everything from the
+    block start on (perturbing a cached block or suffix row changes nothing),
+    unlike the DualCache step, which reads the cached suffix."""
+    P = _tiny_model(2, 4)
+    x = synth.rng(14).integers(0, 63, 40)
+    x[16:] = P.mask_id
+    _, kv = O.full_forward(P, x)
+    fresh = lambda: [(k.copy(), v.copy()) for k, v in kv]
+    base = O.prefix_forward(P, x[16:], 16, fresh())
+    c1 = fresh()
+    c1[0][0][:, 5, :] += 1.0                       # prefix row
+    assert np.abs(O.prefix_forward(P, x[16:], 16, c1) - base).max() > 1e-6
+    c2 = fresh()
+    c2[1][1][:, 30, :] += 5.0                      # suffix row: recomputed
+    c2[0][0][:, 18, :] -= 3.0                      # block row: recomputed
+    np.testing.assert_allclose(O.prefix_forward(P, x[16:], 16, c2), base, atol=1e-12)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_prefix_cache_single_layer_equals_no_cache(seed):
+    """One layer: the cached prefix K/V depend only on the prefix tokens and
+    positions, which do not change inside a block, so PrefixCache decoding
+    equals decoding without a cache, step for step, for any threshold; at
+    tau = 1 both equal the sequential greedy decode."""
+    P = _tiny_model(1, 30 + seed)
+    prompt = synth.prompt_ids(40 + seed, 1, 12, P.mask_id)[0]
+    for tau in (1.0, 0.5, 0.05):
+        a = O.generate_prefixcache(P, prompt, 24, block=8, tau=tau)
+        n = O.generate_nocache(P, prompt, 24, block=8, tau=tau)
+        assert [d for _, d in a.per_step] == [d for _, d in n.per_step]
+        np.testing.assert_array_equal(a.x, n.x)
+        assert a.refreshes == 3
+        if tau == 1.0:
+            s = O.generate_sequential(P, prompt, 24, block=8)
+            np.testing.assert_array_equal(a.x, s.x)
