@@ -5,23 +5,34 @@ on B200.
 Workload: bidirectional transformer of the LLaDA-8B shape (32 layers, hidden
 4096, 32 heads x 128, SwiGLU FFN 12288, RMSNorm, RoPE, vocab 126464), bf16,
 batch 1, prompt 1024 uniform random ids, gen 1024, block 32, DualCache,
-threshold 0.9. One step = one decoding step of the whole hot path:
-  * the first step of every block is a refresh: a full forward over all 2048
-    positions rewriting every layer's K/V cache, then the block's logits;
+threshold 0.9. One bench step = one whole block of the decode, the unit in
+which the method's work repeats:
+  * the block's first decode step is the refresh: a full forward over all
+    2048 positions rewriting every layer's K/V cache, then the block's logits;
   * the others are cached DualCache steps: only the block's 32 rows go
     through the 32 layers (projection + RoPE + cache-slot write, attention
-    over [prefix | block | masked suffix], O proj, SwiGLU FFN);
-  each step ends with the fused LM-head confidence reduction and the
+    over [prefix | block | masked suffix], O proj, SwiGLU FFN), until no
+    position of the block is masked;
+  every decode step ends with the fused LM-head confidence reduction and the
   threshold select/scatter; the host reads back 8 bytes (remaining and
   decoded counts) to decide refresh vs cached for the next step.
-Each (step kind, block) is a CUDA graph captured before timing. Weights are
-seeded random draws on the device (16 GB, larger than L2, streamed every
-step), so no L2 flush is needed. With random weights no confidence reaches
-0.9, so every step decodes one token (the fallback rule) and tokens/s equals
-steps/s.
+The timed steps start at the first block of a fresh decode (a decode that
+reaches its end starts again). Each (step kind, block) is a CUDA graph
+captured before timing. Weights are seeded random draws on the device (16 GB,
+larger than L2, streamed every step), so no L2 flush is needed. With random
+weights no confidence reaches 0.9, so every decode step decodes one position
+(the fallback rule); --planted-bias adds a logit bias per position so that
+the threshold rule fires. --cache prefix|none selects the PrefixCache or no
+cache instead of DualCache (the README's table columns).
+
+The line also carries `kernels`: the DualCache attention on the LLaDA-8B
+attention layer (L = 768) and the LM head + unmask at 32 and 1024 rows, each
+timed alone, and the fused attention call and full attention as timed inside
+the decode; `e2e` is one whole decode through the library's decode loop
+(fdl_generate) from a host prompt to a host copy of the sequence.
 
 Prints one JSON line on rank 0. `--impl reference` times the CPU oracle on
-the same workload instead (bounded sample per step, extrapolated).
+the same workload instead (bounded sample per block, extrapolated).
 """
 from __future__ import annotations
 
@@ -64,10 +75,21 @@ METRIC = "generated tokens/s per B200"
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=64)
-    p.add_argument("--warmup", type=int, default=4)
+    p.add_argument("--steps", type=int, default=32,
+                   help="timed steps; a step is one whole block (its refresh, then its "
+                        "cached steps)")
+    p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--e2e-steps", type=int, default=40)
+    p.add_argument("--cache", choices=["dual", "prefix", "none"], default="dual",
+                   help="K/V reuse after a block's first step (default: DualCache)")
+    p.add_argument("--planted-bias", action="store_true",
+                   help="a planted logit bias per generated position, so that the "
+                        "threshold rule decodes several positions per step")
+    p.add_argument("--block", type=int, default=None, help="block size (default 32)")
+    p.add_argument("--gen", type=int, default=None, help="generated length (default 1024)")
+    p.add_argument("--tau", type=float, default=None, help="threshold (default 0.9)")
+    p.add_argument("--no-kernels", dest="kernels", action="store_false",
+                   help="skip the per-kernel roofline cases")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile-steps", action="store_true",
                    help="also print the per-call time of a cached step and of a refresh")
@@ -164,6 +186,115 @@ def combine_ranks(dist, world, ms, toks, device):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def _peak(peaks, key, fallback):
+    v = peaks.get(key)
+    return (v, f"MEASURED_PEAKS.json {key} (measured)") if v else (fallback,
+                                                                   f"fallback {fallback}")
+
+
+def _graph_time_us(torch, calls, reps):
+    """Mean µs per call of `calls` (a list of callables) captured once in a CUDA
+    graph and replayed `reps` times, timed with CUDA events on the current
+    stream after one untimed replay."""
+    for c in calls[:2]:
+        c()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c in calls:
+            c()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * len(calls))
+    del g
+    return us
+
+
+def kernel_rooflines(torch, ctx, w, peaks):
+    """The two kernels the method's targets name, each timed alone (CUDA events
+    around graph replays), as fractions of the measured peaks:
+      * DualCache block attention on the LLaDA-8B attention layer (32 heads x
+        128, prompt 512 + gen 256, block 32 at position 512): 32 distinct layer
+        caches (403 MB, > L2) cycled; algorithmic bytes = K and V once + q + out;
+      * the LM head fused with the confidence reduction, followed by the
+        threshold unmask of the block, at 32 rows (batch 1: HBM-bound, the
+        weight stream) and 1024 rows (batch 32: tensor-bound), on the model's
+        126464 x 4096 head."""
+    from block_kv_cache_b200 import fdllm
+    hbm, hbm_src = _peak(peaks, "hbm_gbs", 6650.0)
+    tf, tf_src = _peak(peaks, "bf16_tflops", 1590.0)
+    out = {}
+    dev = "cuda"
+    g = torch.Generator(device=dev)
+    g.manual_seed(2024)
+    # ---- C2: DualCache attention, LLaDA-8B layer, L = 768
+    H, d, P, B, S, layers = 32, 128, 512, 32, 224, 32
+    L = P + B + S
+    qs = [torch.randn(1, B, H, d, generator=g, device=dev).to(torch.bfloat16)
+          for _ in range(layers)]
+    ks = [torch.randn(1, H, L, d, generator=g, device=dev).to(torch.bfloat16)
+          for _ in range(layers)]
+    vs = [torch.randn(1, H, L, d, generator=g, device=dev).to(torch.bfloat16)
+          for _ in range(layers)]
+    o = torch.empty_like(qs[0])
+    ws = ctx.workspace(ctx.attention_workspace_bytes(ctx.attn_desc(qs[0], ks[0], P)))
+    calls = [(lambda i=i: ctx.dualcache_attention(qs[i], ks[i], vs[i], P, out=o, ws=ws))
+             for i in range(layers)]
+    us = _graph_time_us(torch, calls, reps=20)
+    nbytes = 2 * H * L * d * 2 + 2 * B * H * d * 2
+    ach = nbytes / us / 1e3
+    out["dualcache_attention"] = {
+        "case": "LLaDA-8B attention layer: 32 heads x 128 (MHA), L = 768 (prompt 512 + gen 256), "
+                "block 32 at 512, bf16; 32 distinct layer caches cycled",
+        "bytes_per_call": nbytes, "us_per_call": us, "bound": "hbm", "achieved": ach,
+        "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "peak_source": hbm_src}
+    del qs, ks, vs, o, calls
+    # ---- LM head + threshold unmask, 32 and 1024 rows of the 126464 x 4096 head
+    V, D = w.lm_head.shape
+    for b in (1, 32):
+        M = 32 * b
+        h = torch.randn(M, D, generator=g, device=dev).to(torch.bfloat16)
+        conf = torch.empty(M, dtype=torch.float32, device=dev)
+        tok = torch.empty(M, dtype=torch.int32, device=dev)
+        lws = torch.empty(max(ctx.lmhead_workspace_bytes(
+            fdllm.LMHeadDesc(M, D, V, fdllm.FDL_BF16)), 16), dtype=torch.uint8, device=dev)
+        x = torch.zeros((b, 2048), dtype=torch.int32, device=dev)
+        msk = torch.zeros((b, 2048), dtype=torch.uint8, device=dev)
+        msk[:, 1024:] = 1
+        rem = torch.empty(b, dtype=torch.int32, device=dev)
+
+        def unit():
+            ctx.lmhead_confidence(h, w.lm_head, conf=conf, tok=tok, ws=lws)
+            ctx.threshold_unmask(conf.view(b, 32), tok.view(b, 32), x, msk, 1024, 0.9,
+                                 remaining=rem)
+        us = _graph_time_us(torch, [unit] * 8, reps=5)
+        nbytes = V * D * 2 + M * D * 2 + M * 16
+        flops = 2.0 * M * D * V
+        key = f"lmhead_unmask_m{M}"
+        if M <= 256:
+            ach = nbytes / us / 1e3
+            out[key] = {"case": f"LM head {V} x {D} + confidence reduction + threshold unmask, "
+                                f"{M} rows (batch {b} x block 32), bf16",
+                        "bytes_per_call": nbytes, "flops_per_call": flops, "us_per_call": us,
+                        "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                        "frac": ach / hbm, "peak_source": hbm_src}
+        else:
+            ach = flops / us / 1e6
+            out[key] = {"case": f"LM head {V} x {D} + confidence reduction + threshold unmask, "
+                                f"{M} rows (batch {b} x block 32), bf16",
+                        "bytes_per_call": nbytes, "flops_per_call": flops, "us_per_call": us,
+                        "bound": "tensor", "achieved": ach, "peak": tf, "unit": "TFLOP/s",
+                        "frac": ach / tf, "peak_source": tf_src + " (burst: timed alone)"}
+    ctx.device_status()
+    return out
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -186,42 +317,49 @@ def run_gpu(args):
     ctx = fdllm.Context(local)
     w = DeviceWeights.random(shape(), seed=1234)
     L = c["prompt"] + c["gen"]
-    dec = BlockDecoder(ctx, w, c["batch"], L, c["block"])
-    prompt = synth.prompt_ids(7 + rank, c["batch"], c["prompt"], c["mask_id"])
+    bias = planted_bias(torch, c, rank) if args.planted_bias else (None, None)
+    dec = BlockDecoder(ctx, w, c["batch"], L, c["block"], cache=args.cache, bias_tok=bias[0],
+                       bias_val=bias[1])
+    prompt = torch.from_numpy(synth.prompt_ids(7 + rank, c["batch"], c["prompt"],
+                                               c["mask_id"])).cuda()
     t0 = time.perf_counter()
-    dec.capture_all(c["prompt"], c["gen"], c["tau"], time_ffn=True)
+    dec.capture_all(c["prompt"], c["gen"], c["tau"], time_calls=True)
     capture_s = time.perf_counter() - t0
     # kernels each step graph launches (kernel nodes of the captured graphs)
     for key in list(dec.graphs):
         dec.kernel_launches(*key)
+    nblk = c["gen"] // c["block"]
 
+    # warm-up: W whole blocks
     dec.begin(prompt, c["tau"])
     for _ in range(max(args.warmup, 3)):
-        dec.step()
+        dec.block()
         if dec.done:
             dec.begin(prompt, c["tau"])
     ctx.device_status()
 
+    # timed: K whole blocks from the first block of a fresh decode (a block =
+    # its refresh forward, then cached steps until it is decoded); a decode
+    # that reaches its end starts again
+    dec.begin(prompt, c["tau"])
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    toks, kinds, launches = 0, {"refresh": 0, "cached": 0}, 0
-    sw_ms, sw_n = 0.0, 0
-    step_ms = {"refresh": [], "cached": []}
+    toks, kinds, launches = 0, {}, 0
+    step_ms = {}
+    replayed = []
+    dec.call_us.clear()
     with ClockSampler(local) as clk:
         ev0.record()
         for _ in range(args.steps):
-            h0 = time.perf_counter()
-            toks += dec.step()
-            step_ms[dec.last_kind].append((time.perf_counter() - h0) * 1e3)
-            launches += dec.kernel_launches(*dec._last_key)
-            kinds[dec.last_kind] += 1
-            if dec.last_kind == "cached":
-                for a, b in dec.last_timers():
-                    sw_ms += a.elapsed_time(b)
-                    sw_n += 1
+            n, steps = dec.block()
+            toks += n
+            for kind, s, ms in steps:
+                kinds[kind] = kinds.get(kind, 0) + 1
+                step_ms.setdefault(kind, []).append(ms)
+                replayed.append((kind, s))
             if dec.done:
                 dec.begin(prompt, c["tau"])
         ev1.record()
@@ -229,86 +367,27 @@ def run_gpu(args):
     barrier()
     ms = ev0.elapsed_time(ev1)
     ctx.device_status()
+    # kernels launched in the timed region: the kernel nodes of every step
+    # graph replayed (counted from the captured graphs)
+    launches = sum(dec.kernel_launches(k, s, c["tau"]) for k, s in replayed)
 
     ms_max, toks_all = combine_ranks(dist, world, ms, toks, "cuda")
-    e2e = run_e2e(torch, dec, prompt, args.e2e_steps)
+    e2e = run_e2e(torch, ctx, w, c, args, rank)
     e2e_ms, e2e_toks = combine_ranks(dist, world, e2e["ms"], e2e["toks"], "cuda")
     e2e_val = e2e_toks / (e2e_ms / 1e3)
+    kernels = kernel_rooflines(torch, ctx, w, read_peaks()) if rank == 0 and args.kernels else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(budget_s=20.0)
 
     if rank == 0:
-        peaks = read_peaks()
-        peak = peaks.get("hbm_gbs") or 6650.0
-        M = c["batch"] * c["block"]
-        D, F = c["hidden"], c["ffn"]
-        # algorithmic bytes of one FFN call: both weights once, the f32 residual
-        # rows read for the norm and read + written by the down projection, x and
-        # f each written and read back
-        ffn_bytes = 3 * F * D * 2 + 2 * M * D * 2 + 2 * M * F * 2 + 3 * M * D * 4
-        ffn_flops = 6.0 * M * D * F
-        sw_avg_ms = sw_ms / max(sw_n, 1)
-        if M <= 256:
-            # few rows: the call streams its weights (HBM-bound)
-            ach = ffn_bytes / (sw_avg_ms / 1e3) / 1e9 if sw_n else None
-            bound, unit, kpeak, src = "hbm", "GB/s", peak, (
-                "MEASURED_PEAKS.json hbm_gbs (measured)" if peaks.get("hbm_gbs")
-                else "fallback 6650 GB/s")
-        else:
-            # a batch of blocks: the call is two dense GEMMs (tensor-bound), timed
-            # inside a long step, so against the sustained bf16 peak
-            ach = ffn_flops / (sw_avg_ms / 1e3) / 1e12 if sw_n else None
-            kpeak = peaks.get("bf16_tflops_sustained") or 1400.0
-            bound, unit, src = "tensor", "TFLOP/s", (
-                "MEASURED_PEAKS.json bf16_tflops_sustained (measured)"
-                if peaks.get("bf16_tflops_sustained") else "fallback 1400 TFLOP/s sustained")
-        # DRAM bytes read + written by the two kernels of one such call, from an
-        # ncu capture of the same kernels at the LLaDA-8B shape (kernel_cases ffn
-        # --rows 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
-        ffn_traffic = (205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
-                       if (M, D, F) == (32, 4096, 12288) else None)
-        out = {
-            "metric": METRIC, "value": toks_all / (ms_max / 1e3), "unit": "tokens/s",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random init)",
-            "config": {"workload": WORKLOAD, "batch": c["batch"], "prompt": c["prompt"],
-                       "gen": c["gen"], "block": c["block"], "tau": c["tau"],
-                       "layers": c["layers"], "hidden": c["hidden"], "vocab": c["vocab"],
-                       "parallelism": f"replicas x{world}",
-                       "steps_by_kind": kinds, "tokens_decoded": toks,
-                       "host_ms_per_step": {k: (statistics.median(v) if v else None)
-                                            for k, v in step_ms.items()},
-                       "host_ms_per_step_mean": {k: (statistics.fmean(v) if v else None)
-                                                 for k, v in step_ms.items()},
-                       "weights_gb": round(w.nbytes() / 1e9, 2),
-                       "graph_capture_s": round(capture_s, 2),
-                       "l2": f"no flush: {w.nbytes() / 1e9:.0f} GB of weights (> 126 MB L2) "
-                             f"are streamed every step"},
-            "gpu_launches": launches,
-            "roofline": {"kernel": f"ffn call of layer 0 of a cached step (M={M}): RMSNorm, "
-                                   f"gate/up GEMM {2 * F}x{D}, SwiGLU, down GEMM {D}x{F} "
-                                   f"(with M <= 256 the RMSNorm and the SwiGLU run in the "
-                                   f"GEMM kernels' prologues)",
-                         "bytes_per_call": ffn_bytes, "flops_per_call": ffn_flops,
-                         "bound": bound, "achieved": ach, "peak": kpeak, "unit": unit,
-                         "frac": (ach / kpeak) if ach else None, "traffic": ffn_traffic,
-                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of "
-                                           "the two kernels of one call" if ffn_traffic
-                         else "no capture at this shape",
-                         "peak_source": src,
-                         "avg_launch_us": sw_avg_ms * 1e3, "launches_timed": sw_n},
-            "e2e": {"value": e2e_val, "unit": "tokens/s",
-                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-            "clocks": clk.summary(),
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(out), flush=True)
+        print(json.dumps(result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max,
+                                     capture_s, e2e, e2e_val, kernels, clk, cpu, launches)),
+              flush=True)
     if args.profile_steps and rank == 0:
-        s0 = c["prompt"] + dec.blk * c["block"] if not dec.done else c["prompt"]
-        prof = {k: dec.profile_step(k, s0, c["tau"]) for k in ("cached", "refresh")}
+        s0 = c["prompt"]
+        prof = {k: dec.profile_step(k, s0, c["tau"]) for k in ("refresh", dec.cached_kind())}
         print(json.dumps({"profile_us_per_step": prof}), flush=True)
     dec.graphs.clear()
     ctx.close()
@@ -316,39 +395,166 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def run_e2e(torch, dec, prompt, steps):
-    """The decode through the public API from a pinned host prompt to a host
-    copy of the sequence: prompt upload, `steps` steps (each reads its 8-byte
-    counters back), final sequence download."""
-    c = CFG
-    hp = torch.from_numpy(np.ascontiguousarray(prompt, dtype=np.int32)).pin_memory()
-    hx = torch.empty((c["batch"], c["prompt"] + c["gen"]), dtype=torch.int32).pin_memory()
+def planted_bias(torch, c, rank):
+    """A planted logit bias per generated position (token drawn != mask id, value
+    ~ U(0, 16)): with random weights no confidence reaches tau, and this makes
+    the threshold rule fire, as a trained model's confident positions would."""
+    from block_kv_cache_b200 import synth
+    g = synth.rng(4242 + rank)
+    bt = g.integers(0, c["mask_id"], (c["batch"], c["gen"])).astype(np.int32)
+    bv = g.uniform(0.0, 16.0, (c["batch"], c["gen"])).astype(np.float32)
+    return torch.from_numpy(bt).cuda(), torch.from_numpy(bv).cuda()
+
+
+def result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max, capture_s, e2e,
+                e2e_val, kernels, clk, cpu, launches):
+    peaks = read_peaks()
+    M = c["batch"] * c["block"]
+    D, F = c["hidden"], c["ffn"]
+    # algorithmic bytes of one FFN call: both weights once, the f32 residual
+    # rows read for the norm and read + written by the down projection, x and
+    # f each written and read back
+    ffn_bytes = 3 * F * D * 2 + 2 * M * D * 2 + 2 * M * F * 2 + 3 * M * D * 4
+    ffn_flops = 6.0 * M * D * F
+    cached = dec.cached_kind()
+    ffn_us = dec.call_us.get((cached, "ffn"), [])
+    att_us = dec.call_us.get((cached, "qkv_attention"), [])
+    full_us = dec.call_us.get(("refresh", "full_attention"), [])
+    ffn_avg = statistics.fmean(ffn_us) if ffn_us else None
+    roof = None
+    if ffn_avg and cached == "cached":
+        if M <= 256:
+            # few rows: the call streams its weights (HBM-bound)
+            kpeak, src = _peak(peaks, "hbm_gbs", 6650.0)
+            ach, bound, unit = ffn_bytes / ffn_avg / 1e3, "hbm", "GB/s"
+        else:
+            # a batch of blocks: two dense GEMMs (tensor-bound) timed inside a
+            # long step, so against the sustained bf16 peak
+            kpeak, src = _peak(peaks, "bf16_tflops_sustained", 1400.0)
+            ach, bound, unit = ffn_flops / ffn_avg / 1e6, "tensor", "TFLOP/s"
+        # DRAM bytes read + written by the two kernels of one such call, from an
+        # ncu capture of the same kernels at the LLaDA-8B shape (kernel_cases ffn
+        # --rows 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
+        traffic = (205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
+                   if (M, D, F) == (32, 4096, 12288) else None)
+        roof = {"kernel": f"ffn call of layer 0 of a cached step (M={M}): RMSNorm, gate/up GEMM "
+                          f"{2 * F}x{D}, SwiGLU, down GEMM {D}x{F} (with M <= 256 the RMSNorm "
+                          f"and the SwiGLU run in the GEMM kernels' prologues)",
+                "bytes_per_call": ffn_bytes, "flops_per_call": ffn_flops, "bound": bound,
+                "achieved": ach, "peak": kpeak, "unit": unit, "frac": ach / kpeak,
+                "traffic": traffic,
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the two "
+                                  "kernels of one call" if traffic else "no capture at this shape",
+                "peak_source": src, "avg_launch_us": ffn_avg, "launches_timed": len(ffn_us)}
+    if kernels is not None and att_us:
+        Hq, Hkv, d = c["heads"], c["kv_heads"], c["head_dim"]
+        N = (Hq + 2 * Hkv) * d
+        L = c["prompt"] + c["gen"]
+        nbytes = (N * D * 2 + 2 * c["batch"] * Hkv * L * d * 2 + M * D * (4 + 2)
+                  + 2 * M * Hq * d * 2)
+        hbm, src = _peak(peaks, "hbm_gbs", 6650.0)
+        a_us = statistics.fmean(att_us)
+        kernels["qkv_attention_in_decode"] = {
+            "case": f"layer 0 of every cached step: RMSNorm + q/k/v projection {N}x{D} (split-K "
+                    f"weight stream) + RoPE + block-slot K/V store + DualCache attention over "
+                    f"L = {L} (graph-replayed, events around the call)",
+            "bytes_per_call": nbytes, "us_per_call": a_us, "bound": "hbm",
+            "achieved": nbytes / a_us / 1e3, "peak": hbm, "unit": "GB/s",
+            "frac": nbytes / a_us / 1e3 / hbm, "peak_source": src, "calls_timed": len(att_us)}
+    if kernels is not None and full_us:
+        Hq, d, L, b = c["heads"], c["head_dim"], c["prompt"] + c["gen"], c["batch"]
+        flops = 4.0 * b * Hq * L * L * d
+        tfp, src = _peak(peaks, "bf16_tflops_sustained", 1400.0)
+        f_us = statistics.fmean(full_us)
+        kernels["full_attention_in_refresh"] = {
+            "case": f"layer 0 of every refresh: bidirectional attention of all {L} positions "
+                    f"({Hq} q heads / {c['kv_heads']} kv heads x {d}, batch {b}; graph-replayed, "
+                    f"events around the call)",
+            "flops_per_call": flops, "us_per_call": f_us, "bound": "tensor",
+            "achieved": flops / f_us / 1e6, "peak": tfp, "unit": "TFLOP/s",
+            "frac": flops / f_us / 1e6 / tfp, "peak_source": src + " (inside a long step)",
+            "calls_timed": len(full_us)}
+    nsteps = sum(kinds.values())
+    blocks = args.steps
+    wl = WORKLOAD
+    if args.cache != "dual" or args.planted_bias:
+        wl += f" [cache={args.cache}{', planted bias' if args.planted_bias else ''}]"
+    return {
+        "metric": METRIC, "value": toks_all / (ms_max / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random init)",
+        "config": {"workload": wl, "step": "one block: its refresh forward, then "
+                                           f"{cached} steps until no position of the block "
+                                           "is masked",
+                   "batch": c["batch"], "prompt": c["prompt"], "gen": c["gen"],
+                   "block": c["block"], "tau": c["tau"], "cache": args.cache,
+                   "planted_bias": bool(args.planted_bias),
+                   "layers": c["layers"], "hidden": c["hidden"], "vocab": c["vocab"],
+                   "parallelism": f"replicas x{world}",
+                   "blocks_timed": blocks, "decode_steps_timed": nsteps,
+                   "steps_by_kind": kinds, "tokens_decoded": toks,
+                   "tokens_per_decode_step": toks / max(nsteps, 1),
+                   "host_ms_per_step": {k: statistics.median(v) for k, v in step_ms.items()},
+                   "host_ms_per_step_mean": {k: statistics.fmean(v) for k, v in step_ms.items()},
+                   "weights_gb": round(w.nbytes() / 1e9, 2),
+                   "graph_capture_s": round(capture_s, 2),
+                   "l2": f"no flush: {w.nbytes() / 1e9:.0f} GB of weights (> 126 MB L2) are "
+                         f"streamed every step"},
+        "gpu_launches": launches,
+        "roofline": roof,
+        "kernels": kernels,
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "path": e2e["path"]},
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+
+
+def run_e2e(torch, ctx, w, c, args, rank):
+    """One whole decode through the library's decode entry point (fdl_generate)
+    from a pinned host prompt to a host copy of the sequence: the binding
+    copies the prompt in, the library runs every block, the binding copies the
+    sequence out; CUDA events around the whole call. The bytes per step are per
+    block (the bench's step)."""
+    from block_kv_cache_b200 import synth
+    hp = torch.from_numpy(synth.prompt_ids(7 + rank, c["batch"], c["prompt"],
+                                           c["mask_id"])).pin_memory()
+    bias = planted_bias(torch, c, rank) if args.planted_bias else (None, None)
+    m = w.native()
+    kw = dict(block=c["block"], tau=c["tau"], cache=args.cache, bias_tok=bias[0],
+              bias_val=bias[1])
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
-    dec.begin(hp, c["tau"])
-    toks = 0
-    for _ in range(steps):
-        toks += dec.step()
-        if dec.done:
-            break
-    hx.copy_(dec.x, non_blocking=True)
+    x, steps = ctx.generate(m, hp, c["gen"], **kw)
     e1.record()
     torch.cuda.synchronize()
-    n = max(dec.steps, 1)
-    return {"ms": e0.elapsed_time(e1), "toks": toks,
-            "h2d": hp.numel() * 4 / n, "d2h": 8 * c["batch"] + hx.numel() * 4 / n}
+    m.close()
+    blocks = c["gen"] // c["block"]
+    return {"ms": e0.elapsed_time(e1), "toks": c["batch"] * c["gen"],
+            "h2d": hp.numel() * 4 / blocks,
+            "d2h": (x.numel() * 4 + steps * c["batch"] * 4) / blocks,
+            "path": f"fdl_generate (the library's decode loop) on a host prompt: {steps} decode "
+                    f"steps, one whole decode of {blocks} blocks"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
 class OracleSample:
-    """A bounded sample of one decode step computed by the CPU oracle (float64
-    NumPy): one transformer layer of a cached block step of one sequence (its
-    block rows over its cache) and the full LM-head confidence of the block; a
-    sequence's step is extrapolated as layers x layer + LM head. The rows of a
-    batch are independent, so the batch's tokens per second equal one
-    sequence's (batch tokens per step, batch times the work)."""
+    """A bounded sample of one block of the decode computed by the CPU oracle
+    (float64 NumPy), for one sequence (the rows of a batch are independent, so
+    a batch's tokens per second equal one sequence's):
+      * a cached step: one transformer layer of the block's rows over the
+        sequence's cache, then the full LM-head confidence of the block and the
+        select; extrapolated as layers x layer + LM head;
+      * the refresh: one layer of the full forward on a slice of REFRESH_ROWS
+        query rows (their projections, attention over all L positions, FFN),
+        whose cost is linear in the rows, extrapolated as layers x L / rows x
+        slice + LM head.
+    A block of the random-init workload decodes one position per step: one
+    refresh and block - 1 cached steps."""
+    REFRESH_ROWS = 128
 
     def __init__(self, seed=0):
         from oracle import fastdllm as O
@@ -364,26 +570,43 @@ class OracleSample:
         self.k = g.standard_normal((c["kv_heads"], L, c["head_dim"]))
         self.v = g.standard_normal((c["kv_heads"], L, c["head_dim"]))
         self.h = g.standard_normal((c["block"], c["hidden"]))
+        self.hr = g.standard_normal((self.REFRESH_ROWS, c["hidden"]))
         self.lm = synth.lmhead_case(rows=c["block"], hidden=c["hidden"], vocab=c["vocab"],
                                     seed=seed, w_seed=0, mask_id=c["mask_id"])
 
-    def step_seconds(self):
-        O, P, c = self.O, self.P, CFG
+    def _layer(self, h, pos):
+        O, P = self.O, self.P
         Lw = P.layers[0]
-        s = c["prompt"]
-        t0 = time.perf_counter()
-        hn = O.rms_norm(self.h, Lw["attn_norm"], P.rms_eps)
-        q, k, v = O._layer_qkv(P, Lw, hn, np.arange(s, s + c["block"]))
-        self.k[:, s:s + c["block"]] = np.transpose(k, (1, 0, 2))
-        self.v[:, s:s + c["block"]] = np.transpose(v, (1, 0, 2))
+        hn = O.rms_norm(h, Lw["attn_norm"], P.rms_eps)
+        q, k, v = O._layer_qkv(P, Lw, hn, pos)
+        self.k[:, pos] = np.transpose(k, (1, 0, 2))
+        self.v[:, pos] = np.transpose(v, (1, 0, 2))
         o, _ = O.attention(q, self.k, self.v)
-        O._layer_rest(P, Lw, self.h, o)
-        t_layer = time.perf_counter() - t0
-        t0 = time.perf_counter()
+        O._layer_rest(P, Lw, h, o)
+
+    def _head(self):
+        O, c = self.O, CFG
         r = O.lmhead_confidence(self.lm.h, self.lm.w, self.lm.bias_tok, self.lm.bias_val)
         O.select_positions(r.conf[:c["block"]], np.ones(c["block"], bool), c["tau"])
+
+    def block_seconds(self):
+        """(block s, cached step s, refresh s, layer of a cached step s, refresh
+        slice s, LM head s)."""
+        c = CFG
+        L = c["prompt"] + c["gen"]
+        s = c["prompt"]
+        t0 = time.perf_counter()
+        self._layer(self.h, np.arange(s, s + c["block"]))
+        t_layer = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        self._head()
         t_head = time.perf_counter() - t0
-        return c["layers"] * t_layer + t_head, t_layer, t_head
+        t0 = time.perf_counter()
+        self._layer(self.hr, np.arange(0, self.REFRESH_ROWS))
+        t_slice = time.perf_counter() - t0
+        cached = c["layers"] * t_layer + t_head
+        refresh = c["layers"] * t_slice * (L / self.REFRESH_ROWS) + t_head
+        return refresh + (c["block"] - 1) * cached, cached, refresh, t_layer, t_slice, t_head
 
 
 def _threads():
@@ -394,22 +617,28 @@ def _threads():
         return os.cpu_count()
 
 
+def _sample_text(est, n):
+    med = lambda i: statistics.median(e[i] for e in est)
+    c = CFG
+    L = c["prompt"] + c["gen"]
+    return (f"{n} samples, float64 NumPy, one sequence: a cached step = {c['layers']} x one "
+            f"layer of the block's {c['block']} rows over a {L}-row cache ({med(3):.3f} s) + the "
+            f"full LM head ({med(5):.3f} s); the refresh = {c['layers']} x {L // 128} x one layer "
+            f"on a {OracleSample.REFRESH_ROWS}-row slice ({med(4):.3f} s) + the LM head; a "
+            f"block = refresh + {c['block'] - 1} cached steps (one position per step, as on the "
+            f"GPU with random weights)")
+
+
 def cpu_baseline(budget_s=20.0):
     smp = OracleSample()
     t0 = time.perf_counter()
     est, n = [], 0
     while time.perf_counter() - t0 < budget_s or n == 0:
-        est.append(smp.step_seconds())
+        est.append(smp.block_seconds())
         n += 1
-    step_s = statistics.median(e[0] for e in est)
-    return {"value": 1.0 / step_s, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
-            "host_cpus": os.cpu_count(),
-            "sample": f"{n} samples of one layer of a cached block step of one sequence "
-                      f"({CFG['block']} rows over a {CFG['prompt'] + CFG['gen']}-row cache) + "
-                      f"the full LM head, float64 NumPy; step time extrapolated as "
-                      f"{CFG['layers']} x layer ({statistics.median(e[1] for e in est):.3f} s)"
-                      f" + LM head ({statistics.median(e[2] for e in est):.3f} s), 1 token "
-                      f"per step as on the GPU"}
+    block_s = statistics.median(e[0] for e in est)
+    return {"value": CFG["block"] / block_s, "unit": "tokens/s", "cores": _threads(),
+            "kind": "oracle", "host_cpus": os.cpu_count(), "sample": _sample_text(est, n)}
 
 
 def run_reference(args):
@@ -419,26 +648,25 @@ def run_reference(args):
         return
     smp = OracleSample()
     for _ in range(args.warmup):
-        smp.step_seconds()
+        smp.block_seconds()
     t0 = time.perf_counter()
-    ext = 0.0
-    for _ in range(args.steps):
-        ext += smp.step_seconds()[0]
+    est = [smp.block_seconds() for _ in range(args.steps)]
     wall = time.perf_counter() - t0
-    val = args.steps / ext
+    ext = sum(e[0] for e in est)
+    val = CFG["block"] * args.steps / ext
     out = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": ext * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded random init)",
-           "config": {"workload": WORKLOAD, "batch": CFG["batch"], "prompt": CFG["prompt"],
+           "config": {"workload": WORKLOAD, "step": "one block: its refresh forward, then "
+                                                    "cached steps until it is decoded",
+                      "batch": CFG["batch"], "prompt": CFG["prompt"],
                       "gen": CFG["gen"], "block": CFG["block"], "tau": CFG["tau"],
                       "layers": CFG["layers"], "parallelism": "cpu oracle"},
            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": _threads(),
                             "kind": "oracle", "host_cpus": os.cpu_count(),
-                            "sample": f"each step: one layer of a cached block step of one "
-                                      f"sequence + the full LM head, extrapolated to "
-                                      f"{CFG['layers']} layers ({wall:.1f} s of CPU time for "
-                                      f"{args.steps} steps)"},
+                            "sample": _sample_text(est, args.steps) +
+                            f" ({wall:.1f} s of CPU time for {args.steps} blocks)"},
            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -450,6 +678,11 @@ def main():
     CFG.clear()
     CFG.update(CONFIGS[args.config])
     WORKLOAD = CFG["workload"]
+    for k in ("block", "gen", "tau"):
+        v = getattr(args, k)
+        if v is not None and v != CFG[k]:
+            CFG[k] = v
+            WORKLOAD += f" [{k} {v}]"
     if args.impl == "reference":
         run_reference(args)
     else:

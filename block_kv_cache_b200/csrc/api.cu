@@ -27,6 +27,10 @@ struct fdl_ctx {
 static const size_t kAccBytes = (size_t)256 * 32768 * 4;
 static const size_t kSyncBytes = 256;
 
+namespace fdl {
+void noalloc_forget(int dev);
+}
+
 namespace {
 
 thread_local char g_msg[512] = "";
@@ -144,6 +148,7 @@ int fdl_create(fdl_ctx** out, int device) {
         delete c;
         return cuda_fail(e, "fdl_create: device buffers");
     }
+    fdl::noalloc_forget(device);
     *out = c;
     return FDL_OK;
 }
@@ -538,8 +543,10 @@ int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
     if (desc->head_dim != 64 && desc->head_dim != 128)
         return fail(FDL_EUNSUPPORTED, "full_attention: head_dim %d", desc->head_dim);
     if (desc->batch < 1 || desc->n_q_heads < 1 || desc->n_kv_heads < 1 ||
-        desc->n_q_heads % desc->n_kv_heads || desc->seq_len < 32 || desc->seq_len % 32)
-        return fail(FDL_EINVAL, "full_attention: bad shape (seq_len a multiple of 32)");
+        desc->n_q_heads % desc->n_kv_heads || desc->block_start < 0 ||
+        desc->seq_len - desc->block_start < 32 || (desc->seq_len - desc->block_start) % 32)
+        return fail(FDL_EINVAL, "full_attention: bad shape (batch, heads; seq_len - block_start "
+                    "a positive multiple of 32)");
     if (!q || !k_cache || !v_cache || !out) return fail(FDL_EINVAL, "full_attention: NULL");
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return fail(FDL_EINVAL, "full_attention: buffers must be 16-byte aligned");
@@ -547,8 +554,9 @@ int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
     const float scale = desc->scale == 0.f ? 1.0f / sqrtf((float)desc->head_dim) : desc->scale;
     cudaError_t e = fdl::launch_full_attention_bf16(desc->batch, desc->n_q_heads,
                                                     desc->n_kv_heads, desc->head_dim,
-                                                    desc->seq_len, scale, q, k_cache, v_cache,
-                                                    out, ctx->sm_count, ctx->d_err,
+                                                    desc->seq_len, desc->seq_len -
+                                                    desc->block_start, scale, q, k_cache,
+                                                    v_cache, out, ctx->sm_count, ctx->d_err,
                                                     (cudaStream_t)stream);
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "full_attention launch");
 }
@@ -585,10 +593,24 @@ __global__ void block_rows_kernel(int32_t* __restrict__ maps, int b, int L, int 
     }
 }
 
+// PrefixCache row maps of the block at s: tail[i * n + j] = i * L + s + j for
+// j < n = L - s (rows [s, L) of sequence i in the [b * L] token rows) and
+// blk[i * B + j] = i * n + j (the block's rows among those b * n rows).
+__global__ void tail_rows_kernel(int32_t* __restrict__ tail, int32_t* __restrict__ blk, int b,
+                                 int L, int s, int B) {
+    const int n = L - s;
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < b * n; e += gridDim.x * blockDim.x) {
+        const int i = e / n, j = e % n;
+        tail[e] = i * L + s + j;
+        if (j < B) blk[i * B + j] = i * n + j;
+    }
+}
+
 // Byte offsets of the generate workspace (256-byte aligned pieces).
 struct GenLayout {
     size_t kc, vc, h_full, x_full, q_full, o_full, f_full, h_blk, x_blk, q_blk, o_blk, f_blk,
-        xn, conf, tok, masked, counts, maps, rope, lm_ws, total;
+        xn, conf, tok, masked, counts, maps, tail_map, tail_blk, bias_tok, bias_val, rope, lm_ws,
+        total;
     size_t kv_layer;    // bytes of one layer's K (or V) cache
     size_t lm_bytes;
 };
@@ -623,6 +645,10 @@ GenLayout gen_layout(const fdl_model_desc& d, int b, int L, int B, size_t lm_byt
     g.masked = take(rf);
     g.counts = take((size_t)2 * b * 4);
     g.maps = take((size_t)nblk * rb * 4);
+    g.tail_map = take(rf * 4);       // PrefixCache: rows [s, L) of every sequence
+    g.tail_blk = take(rb * 4);       // ... and the block's rows among them
+    g.bias_tok = take(rb * 4);       // the planted bias of the current block's rows
+    g.bias_val = take(rb * 4);
     g.rope = take((size_t)L * hd * 4);
     g.lm_bytes = lm_bytes;
     g.lm_ws = take(lm_bytes);
@@ -691,17 +717,27 @@ size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* m, int batch,
 }
 
 int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b, int P, int gen,
-                 int B, float tau, int32_t* x, int* steps_out, void* ws, size_t ws_bytes,
-                 void* stream) {
+                 int B, float tau, const fdl_generate_opts* opts, int32_t* x, int* steps_out,
+                 void* ws, size_t ws_bytes, void* stream) {
     if (!ctx || !m) return fail(FDL_EINVAL, "generate: ctx or model is NULL");
     if (!prompt || !x || !steps_out) return fail(FDL_EINVAL, "generate: NULL buffer");
     if (b < 1 || B < 1 || B > 128 || P < 0 || gen < B || P % B || gen % B)
         return fail(FDL_EINVAL, "generate: need batch >= 1, 1 <= block <= 128, prompt_len and "
                     "gen_len (>= block) multiples of block");
     if (!(tau >= 0.f && tau <= 1.f)) return fail(FDL_EINVAL, "generate: tau must be in [0, 1]");
+    const int mode = opts ? opts->cache : FDL_CACHE_DUAL;
+    if (mode != FDL_CACHE_DUAL && mode != FDL_CACHE_PREFIX && mode != FDL_CACHE_NONE)
+        return fail(FDL_EINVAL, "generate: unknown cache mode %d", mode);
+    const int32_t* bias_tok = opts ? opts->bias_tok : nullptr;
+    const float* bias_val = opts ? opts->bias_val : nullptr;
+    if ((bias_tok == nullptr) != (bias_val == nullptr))
+        return fail(FDL_EINVAL, "generate: bias_tok and bias_val go together");
     const fdl_model_desc& d = m->d;
     const int L = P + gen, D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads;
     const int hd = 128, rf = b * L, rb = b * B;
+    if (mode == FDL_CACHE_PREFIX && L % 32)
+        return fail(FDL_EINVAL, "generate: the PrefixCache mode needs prompt_len + gen_len and "
+                    "the block starts at multiples of 32");
     const GenLayout g = gen_layout(d, b, L, B, lm_ws_bytes(ctx, d, rb));
     if (!ws || ws_bytes < g.total)
         return fail(FDL_EWORKSPACE, "generate: workspace of %zu bytes needed", g.total);
@@ -720,6 +756,10 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
     int32_t* remaining = (int32_t*)at(g.counts);
     int32_t* n_decoded = remaining + b;
     int32_t* maps = (int32_t*)at(g.maps);
+    int32_t* tail_map = (int32_t*)at(g.tail_map);
+    int32_t* tail_blk = (int32_t*)at(g.tail_blk);
+    int32_t* blk_bias_tok = bias_tok ? (int32_t*)at(g.bias_tok) : nullptr;
+    float* blk_bias_val = bias_tok ? (float*)at(g.bias_val) : nullptr;
     float* rope = (float*)at(g.rope);
     const int nblk = (L + B - 1) / B;
 
@@ -746,22 +786,26 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
     if (e != cudaSuccess) return cuda_fail(e, "generate: set-up");
 
     const fdl_lmhead_desc lmd{rb, D, d.vocab, FDL_BF16};
+    // The layers over rows = b * n token rows at positions [pos0, pos0 + n) of
+    // every sequence. full: their K/V go into the caches and they attend over
+    // the whole cache (refresh: pos0 = 0, n = L; PrefixCache step: pos0 = s,
+    // n = L - s); otherwise the fused DualCache step of the block rows.
     auto layers = [&](float* h, void* xb, void* q, void* o, void* f, int rows, bool full,
-                      int s) -> int {
+                      int pos0, int n) -> int {
         int rc = FDL_OK;
         for (int li = 0; li < d.n_layers && rc == FDL_OK; ++li) {
             const fdl_layer_weights& W = m->layers[li];
             void* kl = kc + g.kv_layer * li;
             void* vl = vc + g.kv_layer * li;
             if (full) {
-                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, L, 0, L};
-                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, 0, 1, FDL_BF16, 0.f};
+                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
+                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
                 rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
                 if (!rc) rc = fdl_qkv_rope_store(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl, vl,
                                                  stream);
                 if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
             } else {
-                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, B, s, L};
+                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
                 rc = fdl_qkv_attention(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv, W.bias,
                                        rope, q, kl, vl, o, stream);
             }
@@ -777,25 +821,49 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
     for (int blk = 0; blk < gen / B; ++blk) {
         const int s = P + blk * B;
         const int32_t* row_map = maps + (size_t)(s / B) * rb;
-        for (bool refresh = true;; refresh = false) {
+        if (bias_tok) {
+            // this block's planted bias, [b, gen] -> [b, B] contiguous
+            e = cudaMemcpy2DAsync(blk_bias_tok, (size_t)B * 4, bias_tok + (s - P), (size_t)gen * 4,
+                                  (size_t)B * 4, b, cudaMemcpyDeviceToDevice, st);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2DAsync(blk_bias_val, (size_t)B * 4, bias_val + (s - P),
+                                      (size_t)gen * 4, (size_t)B * 4, b,
+                                      cudaMemcpyDeviceToDevice, st);
+            if (e != cudaSuccess) return cuda_fail(e, "generate: bias");
+        }
+        if (mode == FDL_CACHE_PREFIX) {
+            tail_rows_kernel<<<64, 256, 0, st>>>(tail_map, tail_blk, b, L, s, B);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e, "generate: row maps");
+        }
+        for (bool first = true;; first = false) {
             int rc;
-            if (refresh) {
+            if (first || mode == FDL_CACHE_NONE) {
                 // full forward over every position: all K/V caches rewritten
                 rc = fdl_embed(ctx, rf, D, x, nullptr, m->embed, h_full, stream);
                 if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full),
-                                     at(g.f_full), rf, true, 0);
+                                     at(g.f_full), rf, true, 0, L);
                 if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, row_map, m->final_norm, d.rms_eps,
                                           at(g.xn), stream);
+            } else if (mode == FDL_CACHE_PREFIX) {
+                // PrefixCache step: the block and the suffix over the cached prefix
+                const int n = L - s;
+                rc = fdl_embed(ctx, b * n, D, x, tail_map, m->embed, h_full, stream);
+                if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full),
+                                     at(g.f_full), b * n, true, s, n);
+                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, tail_blk, m->final_norm,
+                                          d.rms_eps, at(g.xn), stream);
             } else {
-                // cached step: only the block's rows
+                // DualCache step: only the block's rows
                 rc = fdl_embed(ctx, rb, D, x, row_map, m->embed, h_blk, stream);
                 if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), rb,
-                                     false, s);
+                                     false, s, B);
                 if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_blk, nullptr, m->final_norm, d.rms_eps,
                                           at(g.xn), stream);
             }
-            if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head, nullptr, nullptr,
-                                                conf, tok, at(g.lm_ws), g.lm_bytes, stream);
+            if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head, blk_bias_tok,
+                                                blk_bias_val, conf, tok, at(g.lm_ws), g.lm_bytes,
+                                                stream);
             const fdl_unmask_desc ud{b, L, s, B, tau};
             if (!rc) rc = fdl_threshold_unmask(ctx, &ud, conf, tok, x, masked, remaining, n_decoded,
                                                stream);

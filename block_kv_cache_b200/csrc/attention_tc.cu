@@ -982,16 +982,19 @@ cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQ
 }
 
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
-                                       int seq_len, float scale, const void* q, const void* k,
-                                       const void* v, void* out, int sm_count, int* dev_err,
-                                       cudaStream_t st) {
-    // query blocks of Bq rows: as many whole heads of a GQA group per 256 rows
+                                       int seq_len, int n_q, float scale, const void* q,
+                                       const void* k, const void* v, void* out, int sm_count,
+                                       int* dev_err, cudaStream_t st) {
+    // The n_q query rows of a sequence (the last n_q positions; all of them at
+    // a refresh) in query blocks of Bq rows: as many whole heads of a GQA group
+    // per 256 rows. Each query block is one "sequence" of the attention kernel
+    // whose K/V are its sequence's (q_per_kv blocks per sequence).
     const int grp = n_q_heads / n_kv_heads;
     int bq = grp == 1 ? 256 : grp == 2 ? 128 : grp <= 4 ? 64 : 32;
-    while (bq > 32 && seq_len % bq) bq /= 2;
-    if (seq_len % bq) return cudaErrorInvalidValue;
-    AttnShape s{batch * (seq_len / bq), n_q_heads, n_kv_heads, head_dim, seq_len, 0, bq, scale,
-                1, seq_len / bq};
+    while (bq > 32 && n_q % bq) bq /= 2;
+    if (n_q < 1 || n_q > seq_len || n_q % bq) return cudaErrorInvalidValue;
+    AttnShape s{batch * (n_q / bq), n_q_heads, n_kv_heads, head_dim, seq_len, 0, bq, scale,
+                1, n_q / bq};
     return launch_attention_bf16(s, q, k, v, out, nullptr, nullptr, sm_count, dev_err, st);
 }
 

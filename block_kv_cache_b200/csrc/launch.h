@@ -38,12 +38,13 @@ bool qkv_attention_fusable(const AttnShape& s, int sm_count);
 cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQKV& pq, void* out,
                                       int sm_count, int* err, cudaStream_t st);
 
-// Full bidirectional attention of every position of every sequence (the
-// refresh forward): q, out [b, L, Hq, d] bf16; caches [b, Hkv, L, d].
+// Full bidirectional attention of the last n_q positions of every sequence
+// over all seq_len positions (n_q = seq_len: the refresh forward; n_q = L - s:
+// a PrefixCache step): q, out [b, n_q, Hq, d] bf16; caches [b, Hkv, L, d].
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
-                                       int seq_len, float scale, const void* q, const void* k,
-                                       const void* v, void* out, int sm_count, int* dev_err,
-                                       cudaStream_t st);
+                                       int seq_len, int n_q, float scale, const void* q,
+                                       const void* k, const void* v, void* out, int sm_count,
+                                       int* dev_err, cudaStream_t st);
 
 cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len,
                             int elem_bytes, const void* k_new, const void* v_new,

@@ -58,6 +58,17 @@ cudaError_t scratch_address(int dev, void** out) {
 
 }  // namespace
 
+namespace fdl {
+// Drop the cached address of `dev` (called by fdl_create): after a device
+// reset the module is loaded again and the array may sit elsewhere, and any
+// context used after a reset is a new one.
+void noalloc_forget(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_scratch_addr[dev] = nullptr;
+}
+}  // namespace fdl
+
 extern "C" FDL_API int fdl_lmhead_confidence_noalloc(fdl_ctx* ctx, const fdl_lmhead_desc* desc,
                                                      const void* h, const void* w,
                                                      const int32_t* bias_tok,

@@ -41,7 +41,7 @@ class AttnDesc(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 
 class LMHeadDesc(ctypes.Structure):
@@ -80,6 +80,15 @@ class LayerWeights(ctypes.Structure):
 class ModelWeights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
                 ("lm_head", ctypes.c_void_p), ("layers", ctypes.POINTER(LayerWeights))]
+
+
+FDL_CACHE_DUAL, FDL_CACHE_PREFIX, FDL_CACHE_NONE = 0, 1, 2
+CACHE_MODES = {"dual": FDL_CACHE_DUAL, "prefix": FDL_CACHE_PREFIX, "none": FDL_CACHE_NONE}
+
+
+class GenerateOpts(ctypes.Structure):
+    _fields_ = [("cache", ctypes.c_int), ("bias_tok", ctypes.c_void_p),
+                ("bias_val", ctypes.c_void_p)]
 
 
 class FdlError(RuntimeError):
@@ -137,7 +146,8 @@ def load() -> ctypes.CDLL:
     L.fdl_model_destroy.argtypes = [vp]
     L.fdl_generate_workspace_bytes.argtypes = [vp, vp, i, i, i]
     L.fdl_generate_workspace_bytes.restype = sz
-    L.fdl_generate.argtypes = [vp, vp, vp, i, i, i, i, fl, vp, ctypes.POINTER(i), vp, sz, vp]
+    L.fdl_generate.argtypes = [vp, vp, vp, i, i, i, i, fl, ctypes.POINTER(GenerateOpts), vp,
+                               ctypes.POINTER(i), vp, sz, vp]
     for name in EXPORTS:
         getattr(L, name).restype = getattr(L, name).restype or i
     _lib = L
@@ -414,21 +424,37 @@ class Context:
                                         _stream(stream)))
         return out
 
-    def generate(self, model: Model, prompt, gen_len, *, block=32, tau=0.9, stream=None):
-        """The whole DualCache decode in the library (fdl_generate): prompt
-        [b, P] int32 CUDA tensor. Returns (x [b, P + gen_len] int32, steps)."""
+    def generate(self, model: Model, prompt, gen_len, *, block=32, tau=0.9, cache="dual",
+                 bias_tok=None, bias_val=None, stream=None):
+        """The whole decode in the library (fdl_generate). prompt [b, P] int32,
+        a CUDA tensor or a host tensor (then copied to the device first, and
+        the result copied back to a host tensor: the public call with host
+        buffers). cache: "dual", "prefix" or "none"; bias_tok / bias_val [b,
+        gen_len] (CUDA, int32 / float32): optional planted logit bias of the
+        generated positions. Returns (x [b, P + gen_len] int32, steps)."""
+        on_host = not prompt.is_cuda
+        dev = torch.device("cuda", self.device)
+        if on_host:
+            prompt = prompt.to(dev, non_blocking=True)
         _need(prompt, "prompt", torch.int32, 2)
         b, P = prompt.shape
+        if bias_tok is not None:
+            _need(bias_tok, "bias_tok", torch.int32, 2)
+            _need(bias_val, "bias_val", torch.float32, 2)
         L = load()
         n = L.fdl_generate_workspace_bytes(self._h, model._h, b, P + gen_len, int(block))
         if n == 0:
             raise ValueError("generate: bad shape")
-        ws = torch.empty(n, dtype=torch.uint8, device=prompt.device)
-        x = torch.empty((b, P + gen_len), dtype=torch.int32, device=prompt.device)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        x = torch.empty((b, P + gen_len), dtype=torch.int32, device=dev)
         steps = ctypes.c_int(0)
+        opts = GenerateOpts(CACHE_MODES[cache], None if bias_tok is None else bias_tok.data_ptr(),
+                            None if bias_val is None else bias_val.data_ptr())
         _check(L.fdl_generate(self._h, model._h, _ptr(prompt), b, P, int(gen_len), int(block),
-                              float(tau), _ptr(x), ctypes.byref(steps), _ptr(ws), n,
-                              _stream(stream)))
+                              float(tau), ctypes.byref(opts), _ptr(x), ctypes.byref(steps),
+                              _ptr(ws), n, _stream(stream)))
+        if on_host:
+            x = x.cpu()
         return x, steps.value
 
     def linear_residual(self, x, w, h, *, stream=None):
@@ -466,12 +492,21 @@ class Context:
                               _ptr(w_gu), _ptr(w_down), _ptr(f), _ptr(h), _stream(stream)))
         return f
 
-    def full_attention(self, q, k_cache, v_cache, *, out=None, scale=0.0, stream=None):
-        """Bidirectional attention of every position: q, out [b, L, Hq, d]."""
+    def full_attention(self, q, k_cache, v_cache, *, q_start=0, out=None, scale=0.0,
+                       stream=None):
+        """Bidirectional attention of the positions [q_start, L) over all L
+        positions of the caches: q, out [b, L - q_start, Hq, d] (q_start = 0:
+        every position, the refresh; q_start = s: the block and the suffix of a
+        PrefixCache step)."""
         _need(q, "q", torch.bfloat16, 4)
-        b, L, Hq, d = q.shape
-        hkv = k_cache.shape[1]
-        desc = AttnDesc(b, Hq, hkv, d, L, 0, 1, FDL_BF16, float(scale))
+        _need(k_cache, "k_cache", torch.bfloat16, 4)
+        _need(v_cache, "v_cache", torch.bfloat16, 4)
+        b, nq, Hq, d = q.shape
+        hkv, L = k_cache.shape[1], k_cache.shape[2]
+        if nq != L - int(q_start):
+            raise ValueError(f"full_attention: q has {nq} rows per sequence, the caches "
+                             f"{L} - q_start {q_start}")
+        desc = AttnDesc(b, Hq, hkv, d, L, int(q_start), nq, FDL_BF16, float(scale))
         if out is None:
             out = torch.empty_like(q)
         _check(load().fdl_full_attention(self._h, ctypes.byref(desc), _ptr(q), _ptr(k_cache),

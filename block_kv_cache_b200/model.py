@@ -21,7 +21,9 @@ epilogue finds both halves of a feature in one tile.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
+import time
 from dataclasses import dataclass
 
 import numpy as np
@@ -148,14 +150,33 @@ class DeviceWeights:
         return n
 
 
+CACHE_MODES = ("dual", "prefix", "none")
+
+
 class BlockDecoder:
-    """DualCache + threshold decoding of `batch` sequences of length seq_len."""
+    """Block decoding with the threshold rule of `batch` sequences of length
+    seq_len, with one of three cache modes (Fast-dLLM README usage flags and
+    evaluation table):
+      "dual"   (--use_cache --if_cache_position): DualCache; a cached step runs
+               only the block's rows over [cached prefix | block | cached suffix];
+      "prefix" (--use_cache): PrefixCache; a cached step runs the block and the
+               masked suffix (rows [s, L)) over [cached prefix | fresh rows];
+      "none"   (no cache): every step is a full forward over all positions.
+    In every mode a block's first step is the full forward (the refresh).
+
+    With bias_tok / bias_val ([b, gen] int32 / f32 on the device), the LM head
+    adds bias_val to the logit of token bias_tok at each generated position
+    (a synthetic planted-token bias, so that confidences can exceed the
+    threshold with random weights)."""
 
     def __init__(self, ctx: fdllm.Context, w: DeviceWeights, batch: int, seq_len: int,
-                 block: int = 32, device="cuda"):
+                 block: int = 32, device="cuda", cache: str = "dual", bias_tok=None,
+                 bias_val=None):
+        assert cache in CACHE_MODES
         sh = w.shape
         self.ctx, self.w, self.sh = ctx, w, sh
         self.b, self.L, self.B = batch, seq_len, block
+        self.cache = cache
         dev = device
         D, d = sh.hidden, sh.head_dim
         self.rope = torch.from_numpy(fdllm.rope_table(sh.rope_theta, seq_len, d)).to(dev)
@@ -186,49 +207,87 @@ class BlockDecoder:
         self.x = torch.empty((batch, seq_len), dtype=torch.int32, device=dev)
         self.masked = torch.empty((batch, seq_len), dtype=torch.uint8, device=dev)
         self.graphs = {}
-        self.graph_timers = {}          # graph key -> [(event, event)] around the FFN calls
+        self.graph_timers = {}          # graph key -> {call: [(event, event)]} of layer 0
+        self.call_us = {}               # (step kind, call) -> µs of each replay (step())
         self._launches = {}             # graph key -> kernels per replay
         self._timers = None
-        # rows of block k of every sequence in the flattened [b * L] token rows
         nblk = (seq_len + block - 1) // block
         i = np.arange(block)
-        maps = np.stack([(np.arange(batch)[:, None] * seq_len + k * block + i[None, :]).reshape(-1)
+        bi = np.arange(batch)[:, None]
+        # rows of block k of every sequence in the flattened [b * L] token rows
+        maps = np.stack([(bi * seq_len + k * block + i[None, :]).reshape(-1)
                          for k in range(nblk)]).astype(np.int32)
         self.row_maps = torch.from_numpy(np.minimum(maps, batch * seq_len - 1)).to(dev)
+        # PrefixCache: rows [s, L) of every sequence in the [b * L] token rows
+        # (tail_maps[k]), and the block's rows within those b * (L - s) rows
+        self.tail_maps, self.tail_blk = [], []
+        if cache == "prefix":
+            for k in range(nblk):
+                n = seq_len - k * block
+                j = np.arange(n)
+                self.tail_maps.append(torch.from_numpy(
+                    (bi * seq_len + k * block + j[None, :]).reshape(-1).astype(np.int32)).to(dev))
+                self.tail_blk.append(torch.from_numpy(
+                    (bi * n + i[None, :]).reshape(-1).astype(np.int32)).to(dev))
+        # planted bias per generated position, sliced per block ([nblk, b * B])
+        self.bias = None
+        if bias_tok is not None:
+            gen = bias_tok.shape[1]
+            P0 = seq_len - gen
+            assert gen % block == 0 and P0 % block == 0
+            bt = bias_tok.view(batch, gen // block, block).transpose(0, 1).contiguous()
+            bv = bias_val.view(batch, gen // block, block).transpose(0, 1).contiguous()
+            self.bias = (P0 // block, bt.view(gen // block, rb), bv.view(gen // block, rb))
         lmd = fdllm.LMHeadDesc(rb, D, sh.vocab, fdllm.FDL_BF16)
         self.ws_lm = torch.empty(max(ctx.lmhead_workspace_bytes(lmd), 16), dtype=torch.uint8,
                                  device=dev)
 
     # ------------------------------------------------------------------ layers
+    @contextlib.contextmanager
+    def _timed(self, name, on):
+        """CUDA events around one call (layer 0 only: events in a graph cut the
+        overlap of neighbouring kernels)."""
+        if not on:
+            yield
+            return
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        e0.record()
+        yield
+        e1.record()
+        self._timers.setdefault(name, []).append((e0, e1))
+
     def _layers(self, h, x, q, o, f, rows, rows_per_seq, pos0, full):
+        """The layers over `rows` = b * rows_per_seq token rows at positions
+        pos0 + [0, rows_per_seq) of every sequence. full: those rows' K/V are
+        written into the caches and the rows attend over the whole cache
+        (refresh: pos0 = 0; PrefixCache step: pos0 = s); otherwise the fused
+        DualCache step of the block rows."""
         ctx, sh = self.ctx, self.sh
         for li, Lw in enumerate(self.w.layers):
+            timed = self._timers is not None and li == 0
             if full:
-                ctx.rmsnorm(h, Lw["attn_norm"], sh.rms_eps, out=x)
-                ctx.qkv_rope_store(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
+                ctx.rmsnorm(h, Lw["attn_norm"], sh.rms_eps, out=x, rows=rows)
+                ctx.qkv_rope_store(x[:rows], Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
                                    n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
                                    bias=Lw["bias"])
-                ctx.full_attention(q.view(self.b, self.L, sh.n_q_heads, sh.head_dim),
-                                   self.kc[li], self.vc[li],
-                                   out=o.view(self.b, self.L, sh.n_q_heads, sh.head_dim))
+                with self._timed("full_attention", timed):
+                    ctx.full_attention(
+                        q[:rows].view(self.b, rows_per_seq, sh.n_q_heads, sh.head_dim),
+                        self.kc[li], self.vc[li], q_start=pos0,
+                        out=o[:rows].view(self.b, rows_per_seq, sh.n_q_heads, sh.head_dim))
             else:
                 # norm + block-slot projection + DualCache attention of the block rows
-                ctx.qkv_attention(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
-                                  o.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
-                                  n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq, pos0=pos0,
-                                  bias=Lw["bias"], h=h, norm_w=Lw["attn_norm"], eps=sh.rms_eps)
-            ctx.linear_residual(o.view(rows, -1), Lw["wo"], h)
-            # timing events around layer 0's FFN call only: events in the graph
-            # cut the overlap of neighbouring kernels
-            timed = self._timers is not None and li == 0
-            if timed:
-                e0 = torch.cuda.Event(enable_timing=True, external=True)
-                e1 = torch.cuda.Event(enable_timing=True, external=True)
-                e0.record()
-            ctx.ffn(x, Lw["w_gu"], Lw["wd"], h, f=f, norm_w=Lw["ffn_norm"], eps=sh.rms_eps)
-            if timed:
-                e1.record()
-                self._timers.append((e0, e1))
+                with self._timed("qkv_attention", timed):
+                    ctx.qkv_attention(x, Lw["w_qkv"], self.rope, q, self.kc[li], self.vc[li],
+                                      o.view(self.b, self.B, sh.n_q_heads, sh.head_dim),
+                                      n_q_heads=sh.n_q_heads, rows_per_seq=rows_per_seq,
+                                      pos0=pos0, bias=Lw["bias"], h=h, norm_w=Lw["attn_norm"],
+                                      eps=sh.rms_eps)
+            ctx.linear_residual(o[:rows].view(rows, -1), Lw["wo"], h[:rows])
+            with self._timed("ffn", timed):
+                ctx.ffn(x[:rows], Lw["w_gu"], Lw["wd"], h[:rows], f=f[:rows],
+                        norm_w=Lw["ffn_norm"], eps=sh.rms_eps)
 
     def refresh(self, x_ids, s):
         """Full forward over all positions of x_ids [b, L] (int32, device): rewrites
@@ -239,7 +298,7 @@ class BlockDecoder:
                      self.L, 0, True)
         self.ctx.rmsnorm(self.h_full, self.w.final_norm, self.sh.rms_eps, out=self.xn,
                          row_map=self._row_map(s))
-        self._confidence()
+        self._confidence(s)
 
     def block_step(self, x_ids, s):
         """Cached DualCache step for block [s, s+B) of x_ids [b, L]."""
@@ -248,14 +307,31 @@ class BlockDecoder:
         self._layers(self.h_blk, self.x_blk, self.q_blk, self.o_blk, self.f_blk, rows, self.B,
                      s, False)
         self.ctx.rmsnorm(self.h_blk, self.w.final_norm, self.sh.rms_eps, out=self.xn)
-        self._confidence()
+        self._confidence(s)
+
+    def prefix_step(self, x_ids, s):
+        """Cached PrefixCache step for block [s, s+B): rows [s, L) of every
+        sequence go through the layers over the cached prefix."""
+        k = s // self.B
+        n = self.L - s
+        rows = self.b * n
+        self.ctx.embed(x_ids, self.w.embed, out=self.h_full, row_map=self.tail_maps[k])
+        self._layers(self.h_full, self.x_full, self.q_full, self.o_full, self.f_full, rows, n,
+                     s, True)
+        self.ctx.rmsnorm(self.h_full, self.w.final_norm, self.sh.rms_eps, out=self.xn,
+                         row_map=self.tail_blk[k])
+        self._confidence(s)
 
     def _row_map(self, s):
         assert s % self.B == 0, "blocks start at multiples of the block size"
         return self.row_maps[s // self.B]
 
-    def _confidence(self):
-        self.ctx.lmhead_confidence(self.xn, self.w.lm_head, conf=self.conf, tok=self.tok,
+    def _confidence(self, s):
+        bt = bv = None
+        if self.bias is not None:
+            k = s // self.B - self.bias[0]
+            bt, bv = self.bias[1][k], self.bias[2][k]
+        self.ctx.lmhead_confidence(self.xn, self.w.lm_head, bt, bv, conf=self.conf, tok=self.tok,
                                    ws=self.ws_lm)
 
     def unmask(self, x_ids, masked, s, tau):
@@ -263,12 +339,25 @@ class BlockDecoder:
                                   x_ids, masked, s, tau, remaining=self.remaining,
                                   n_decoded=self.n_decoded)
 
+    def _forward(self, kind, x_ids, s):
+        if kind == "refresh":
+            self.refresh(x_ids, s)
+        elif kind == "prefix":
+            self.prefix_step(x_ids, s)
+        else:
+            self.block_step(x_ids, s)
+
+    def cached_kind(self):
+        """The kind of a block's steps after its first: the cache mode's step."""
+        return {"dual": "cached", "prefix": "prefix", "none": "refresh"}[self.cache]
+
     # ------------------------------------------------------------------ decode
     def generate(self, prompt, gen_len, tau=0.9, record=None):
         """Decode gen_len tokens after prompt [b, P] (host or device int32) with
-        DualCache and the threshold rule. Returns (x [b, L] int32 device, steps).
-        If `record` is a list, each step appends (kind, s, x_before, masked_before,
-        conf, tok) as host arrays (for step-wise checks)."""
+        the decoder's cache mode and the threshold rule. Returns (x [b, L] int32
+        device, steps). If `record` is a list, each step appends (kind, s,
+        x_before, masked_before, conf, tok, xn) as host arrays (for step-wise
+        checks; xn holds the final-norm rows the LM head consumed, as float32)."""
         b, P = prompt.shape
         assert P + gen_len == self.L and gen_len % self.B == 0
         dev = self.h_full.device
@@ -284,43 +373,38 @@ class BlockDecoder:
             while True:
                 if record is not None:
                     xb, mb = x.cpu().numpy(), masked.cpu().numpy()
-                if kind == "refresh":
-                    self.refresh(x, s)
-                else:
-                    self.block_step(x, s)
+                self._forward(kind, x, s)
                 if record is not None:
                     record.append((kind, s, xb, mb, self.conf.cpu().numpy().copy(),
-                                   self.tok.cpu().numpy().copy()))
+                                   self.tok.cpu().numpy().copy(),
+                                   self.xn.float().cpu().numpy()))
                 self.unmask(x, masked, s, tau)
                 steps += 1
                 host_rem.copy_(self.remaining, non_blocking=True)
                 torch.cuda.current_stream().synchronize()
                 if int(host_rem.max()) == 0:
                     break
-                kind = "cached"
+                kind = self.cached_kind()
         return x, steps
 
     # ------------------------------------------------------- graph-replayed decode
     def _step_calls(self, kind, s, tau):
-        if kind == "refresh":
-            self.refresh(self.x, s)
-        else:
-            self.block_step(self.x, s)
+        self._forward(kind, self.x, s)
         self.unmask(self.x, self.masked, s, tau)
         self.counts_host.copy_(self.counts, non_blocking=True)
 
-    def capture(self, kind, s, tau, time_ffn=False):
+    def capture(self, kind, s, tau, time_calls=False):
         """CUDA graph of one decode step (forward, unmask, counter read-back) for
         block start s; kernels read and write the decoder's own x / masked. With
-        time_ffn, timing events bracket layer 0's FFN call."""
+        time_calls, timing events bracket layer 0's attention and FFN calls."""
         key = (kind, s, float(tau))
         if key not in self.graphs:
             g = torch.cuda.CUDAGraph(keep_graph=True)   # the graph stays readable
-            self._timers = [] if time_ffn else None
+            self._timers = {} if time_calls else None
             with torch.cuda.graph(g):
                 self._step_calls(kind, s, tau)
             g.instantiate()
-            self.graph_timers[key] = self._timers or []
+            self.graph_timers[key] = self._timers or {}
             self._timers = None
             self.graphs[key] = g
         return self.graphs[key]
@@ -333,14 +417,15 @@ class BlockDecoder:
         return self._launches[key]
 
     def last_timers(self):
-        """Event pairs of the graph replayed by the last step()."""
-        return self.graph_timers.get(self._last_key, [])
+        """{call: [(event, event)]} of the graph replayed by the last step()."""
+        return self.graph_timers.get(self._last_key, {})
 
-    def capture_all(self, prompt_len, gen_len, tau, time_ffn=False):
+    def capture_all(self, prompt_len, gen_len, tau, time_calls=False):
         for blk in range(gen_len // self.B):
             s = prompt_len + blk * self.B
-            self.capture("refresh", s, tau, time_ffn)
-            self.capture("cached", s, tau, time_ffn)
+            self.capture("refresh", s, tau, time_calls)
+            if self.cache != "none":
+                self.capture(self.cached_kind(), s, tau, time_calls)
         torch.cuda.synchronize()
 
     def begin(self, prompt, tau):
@@ -361,6 +446,9 @@ class BlockDecoder:
         self.last_kind = self.kind
         self.capture(self.kind, s, self.tau).replay()
         torch.cuda.current_stream().synchronize()
+        for name, pairs in self.graph_timers.get(self._last_key, {}).items():
+            us = self.call_us.setdefault((self.kind, name), [])
+            us.extend(a.elapsed_time(b) * 1e3 for a, b in pairs)
         rem = int(self.counts_host[0].max())
         nd = int(self.counts_host[1].sum())
         self.steps += 1
@@ -370,8 +458,21 @@ class BlockDecoder:
             if self.P + self.blk * self.B >= self.L:
                 self.done = True
         else:
-            self.kind = "cached"
+            self.kind = self.cached_kind()
         return nd
+
+    def block(self):
+        """Decode the current block to its end (one refresh, then the cache
+        mode's steps until no position of the block is masked). Returns
+        (tokens decoded, [(kind, block start, host ms)] per step)."""
+        toks, steps = 0, []
+        blk = self.blk
+        while not self.done and self.blk == blk:
+            s = self.P + self.blk * self.B
+            t0 = time.perf_counter()
+            toks += self.step()
+            steps.append((self.last_kind, s, (time.perf_counter() - t0) * 1e3))
+        return toks, steps
 
     # ------------------------------------------------------------------ profiling
     def profile_step(self, kind, s, tau, reps=5):

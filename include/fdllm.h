@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define FDL_ABI_VERSION 3
+#define FDL_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define FDL_API __attribute__((visibility("default")))
@@ -198,7 +198,9 @@ FDL_API int fdl_lmhead_confidence(fdl_ctx* ctx, const fdl_lmhead_desc* desc,
  * vocabulary of 126464) are rejected with FDL_EINVAL before anything runs.
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream
- * capture. All calls share the one array and it keeps the last call's
+ * capture. fdl_create drops the cached address of its device, so after a
+ * cudaDeviceReset (which invalidates every context and the address) the
+ * first call on a new context looks it up again. All calls share the one array and it keeps the last call's
  * contents; each call writes every entry it later reads. Calls whose
  * executions overlap on the GPU (different streams, or different contexts
  * on one device) race on the array and must be ordered by the caller.
@@ -356,10 +358,15 @@ FDL_API int fdl_ffn(fdl_ctx* ctx, int rows, int hidden, int ffn, const float* no
                     void* x, const void* w_gu, const void* w_down, void* f, float* h,
                     void* stream);
 
-/* Full bidirectional attention of every position (the refresh forward after
- * a block completes): out[b, i, h, :] = softmax over all j of q_i . k_j.
- *   q, out [b, L, Hq, d] bf16; caches [b, Hkv, L, d] bf16 (desc->dtype must
- *   be FDL_BF16; block_start/block_len are ignored). L % 32 == 0.
+/* Full bidirectional attention of the positions [s, L), s = desc->block_start,
+ * over all L positions of the caches: out[b, i, h, :] = sum_j softmax_j(scale *
+ * q_i . k_j) v_j over every j in [0, L). s = 0 is the refresh forward after a
+ * block completes (ICLR reviews, review 4 question 2: all K/V are recomputed);
+ * s = the block start is the attention of a PrefixCache step, where the block
+ * and the masked suffix are recomputed over the cached prefix (README usage
+ * flag --use_cache without --if_cache_position).
+ *   q, out [b, L - s, Hq, d] bf16; caches [b, Hkv, L, d] bf16 (desc->dtype
+ *   must be FDL_BF16; block_len is ignored). L - s a positive multiple of 32.
  * Errors: FDL_EINVAL, FDL_EUNSUPPORTED, FDL_ECUDA. */
 FDL_API int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
                                const void* k_cache, const void* v_cache, void* out,
@@ -427,14 +434,41 @@ FDL_API int fdl_model_destroy(fdl_model* model);
 FDL_API size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* model, int batch,
                                             int seq_len, int block);
 
+/* Which K/V a decode step after a block's first reuses (Fast-dLLM README,
+ * usage flags and the evaluation table's "+cache" columns; aibase news
+ * "Innovations" 1). A block's first step is always the full forward that
+ * rewrites every layer's cache. */
+typedef enum {
+    FDL_CACHE_DUAL = 0,    /* DualCache (--use_cache --if_cache_position): only the block's
+                              rows are recomputed; prefix and masked suffix come from the cache */
+    FDL_CACHE_PREFIX = 1,  /* PrefixCache (--use_cache): the block and the suffix, rows [s, L),
+                              are recomputed over the cached prefix */
+    FDL_CACHE_NONE = 2     /* no cache: every step is a full forward over all positions */
+} fdl_cache_mode;
+
+typedef struct {
+    int cache;                /* fdl_cache_mode */
+    /* Optional planted logit bias per generated position (a synthetic workload
+     * device: with random weights no confidence reaches a threshold, and a bias
+     * on one token per position makes the parallel rule fire): at the LM head of
+     * every step, the logit of token bias_tok[i, p - prompt_len] of position p
+     * of sequence i gets + bias_val[i, p - prompt_len]. */
+    const int32_t* bias_tok;  /* [batch, gen_len] int32 device, entries in [0, V), or NULL */
+    const float* bias_val;    /* [batch, gen_len] f32 device; required iff bias_tok */
+} fdl_generate_opts;
+
 /* Decode gen_len positions after the prompts of `batch` sequences.
  *   prompt  [batch, prompt_len] int32 device (token ids)
  *   out_x   [batch, prompt_len + gen_len] int32 device (written: the prompts,
  *           then the decoded tokens)
  *   block   positions per block, 1..128; prompt_len and gen_len multiples of it
- *   tau     threshold in [0, 1]
+ *           (FDL_CACHE_PREFIX: prompt_len + gen_len and every block start also
+ *           multiples of 32)
+ *   tau     threshold in [0, 1] (tau = 1 decodes exactly one position per step)
+ *   opts    cache mode and optional planted bias; NULL = FDL_CACHE_DUAL, no bias
  *   *steps_out (host) the decode steps taken (refresh steps included)
- *   ws      device workspace of fdl_generate_workspace_bytes bytes
+ *   ws      device workspace of fdl_generate_workspace_bytes bytes, 256-byte
+ *           aligned
  * Every step reads `batch` 4-byte counters back to the host to decide
  * between the next cached step and the next block; the call returns when the
  * decode is complete (the stream is synchronised). The kernels and their
@@ -443,8 +477,9 @@ FDL_API size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* model
  * fdl_linear_residual, fdl_ffn, fdl_lmhead_confidence, fdl_threshold_unmask).
  * Errors: FDL_EINVAL, FDL_EWORKSPACE, FDL_ECUDA, or those of the calls. */
 FDL_API int fdl_generate(fdl_ctx* ctx, const fdl_model* model, const int32_t* prompt, int batch,
-                         int prompt_len, int gen_len, int block, float tau, int32_t* out_x,
-                         int* steps_out, void* ws, size_t ws_bytes, void* stream);
+                         int prompt_len, int gen_len, int block, float tau,
+                         const fdl_generate_opts* opts, int32_t* out_x, int* steps_out, void* ws,
+                         size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -24,6 +24,7 @@ pytestmark = pytest.mark.gpu
 BF16_TOL = 2e-2
 CONF_MODEL_TOL = 2e-2
 TOK_GAP = 0.05
+CONF_TOL = 1e-5
 
 
 @pytest.fixture(scope="module")
@@ -200,8 +201,13 @@ def test_qkv_attention(ctx, batch, Hq, Hkv, bias, B, pos0, L, D, norm):
             assert rel(og[sq], o_ref) <= BF16_TOL, (rep, sq)
 
 
-@pytest.mark.parametrize("b,Hq,Hkv,L", [(1, 32, 32, 256), (2, 28, 4, 128), (2, 8, 2, 96)])
+@pytest.mark.parametrize("b,Hq,Hkv,L", [(1, 32, 32, 256), (2, 28, 4, 128), (2, 8, 2, 96),
+                                        (1, 32, 32, 2048),     # LLaDA-8B refresh: 8 query blocks
+                                        (2, 28, 4, 1024)])     # Dream-7B refresh, two sequences
 def test_full_attention(ctx, b, Hq, Hkv, L):
+    """Bidirectional attention of every position (the refresh), against the
+    oracle for every query row; the L = 2048 MHA case runs the 256-row query
+    blocks (eight per head) of the LLaDA-8B refresh."""
     g = synth.rng(b * Hq + L)
     d = 128
     q = bf_vals(g.standard_normal((b, L, Hq, d)))
@@ -220,26 +226,46 @@ def _small_params(seed, n_layers=2, hq=2, hkv=2, bias=False):
                               qkv_bias=bias, w_std=0.06, lm_std=0.15)
 
 
-def _replay_check(P, rec, x_final, B, tau):
-    """Oracle replay of a recorded GPU decode (see module docstring)."""
+def _replay_check(P, rec, x_final, B, tau, tok_gap=TOK_GAP, bias=None):
+    """Oracle replay of a recorded GPU decode (see module docstring), step kind
+    by step kind: a refresh is the full forward (and rebuilds the oracle's
+    caches), a DualCache step the block forward, a PrefixCache step the
+    forward of the block and suffix over the cached prefix. At every step
+    also the LM-head boundary on its own: the oracle's confidences of the
+    GPU's final-norm rows (the exact LM-head input) within CONF_TOL of the
+    GPU's, token ids exact where the oracle's top-2 logit gap exceeds 1e-3.
+    bias = (bias_tok, bias_val, prompt_len): the planted bias [b, gen] of the
+    generated positions, added by the LM head."""
     b = rec[0][2].shape[0]
     caches = [None] * b
     max_err = 0.0
-    for n, (kind, s, xb, mb, conf, tok) in enumerate(rec):
+    for n, (kind, s, xb, mb, conf, tok, xn) in enumerate(rec):
         conf = conf.reshape(b, B)
         tok = tok.reshape(b, B)
+        xn = xn.reshape(b, B, -1)
         for i in range(b):
             if kind == "refresh":
-                logits, kv = O.full_forward(P, xb[i])
+                hf, kv = O.full_hidden(P, xb[i])
                 caches[i] = [(k.copy(), v.copy()) for k, v in kv]
-                lg = logits[s:s + B]
+                hb = hf[s:s + B]
+            elif kind == "cached":
+                hb = O.block_hidden(P, xb[i, s:s + B], s, caches[i])
             else:
-                lg = O.block_forward(P, xb[i, s:s + B], s, caches[i])
-            c = O.confidence_from_logits(lg)
+                assert kind == "prefix"
+                hb = O.prefix_hidden(P, xb[i, s:], s, caches[i])[:B]
+            bt = bv = None
+            if bias is not None:
+                bt = bias[0][i, s - bias[2]:s - bias[2] + B]
+                bv = bias[1][i, s - bias[2]:s - bias[2] + B]
+            c = O.lmhead_confidence(hb, P.lm_head, bt, bv)
             max_err = max(max_err, float(np.abs(conf[i] - c.conf).max()))
-            sure = c.gap > TOK_GAP
+            sure = c.gap > tok_gap
             assert np.array_equal(tok[i][sure], c.tok[sure]), (n, i)
-        # decisions on the GPU's confidences, bit-exact
+            cb = O.lmhead_confidence(xn[i], P.lm_head, bt, bv)
+            assert np.abs(conf[i] - cb.conf).max() <= CONF_TOL, (n, i)
+            sure = cb.gap > 1e-3
+            assert np.array_equal(tok[i][sure], cb.tok[sure]), (n, i)
+    # decisions on the GPU's confidences, bit-exact
         xa, ma, _, nd = O.threshold_unmask(xb, mb, conf, tok, s, B, tau)
         x_next = rec[n + 1][2] if n + 1 < len(rec) else x_final
         m_next = rec[n + 1][3] if n + 1 < len(rec) else None
@@ -267,6 +293,117 @@ def test_decode_matches_oracle_step_by_step(ctx, seed, tau, hq, hkv, bias):
     if tau == 1.0:
         assert steps == gen                              # one token per step
     _replay_check(P, rec, xf, B, tau)
+
+
+@pytest.mark.parametrize("cache,seed,tau,hq,hkv,bias", [("prefix", 3, 0.9, 2, 2, False),
+                                                        ("prefix", 4, 0.5, 4, 2, True),
+                                                        ("none", 5, 0.7, 2, 1, False)])
+def test_cache_modes_match_oracle_step_by_step(ctx, cache, seed, tau, hq, hkv, bias):
+    """PrefixCache (block and suffix recomputed over the cached prefix) and
+    no-cache decoding (a full forward every step), replayed by the oracle on
+    the GPU's own trajectory like the DualCache decode."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(seed, hq=hq, hkv=hkv, bias=bias)
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B = 2, 64, 64, 32
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B, cache=cache)
+    prompt = synth.prompt_ids(seed, b, Lp, P.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
+    ctx.device_status()
+    kinds = {r[0] for r in rec}
+    assert kinds == ({"refresh", "prefix"} if cache == "prefix" else {"refresh"})
+    _replay_check(P, rec, x.cpu().numpy(), B, tau)
+
+
+def test_planted_bias_decode_matches_oracle(ctx):
+    """With a planted logit bias on one token per generated position (the
+    synthetic way to make the threshold rule fire with random weights), the
+    DualCache decode decodes several positions per step and the oracle's
+    replay (with the same bias in its LM head) agrees at every step."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(6, hq=4, hkv=2, bias=True)
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B, tau = 2, 64, 64, 32, 0.9
+    g = synth.rng(66)
+    bt = g.integers(0, P.mask_id, (b, gen)).astype(np.int32)
+    bv = g.uniform(0.0, 16.0, (b, gen)).astype(np.float32)
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B, bias_tok=torch.from_numpy(bt).cuda(),
+                       bias_val=torch.from_numpy(bv).cuda())
+    prompt = synth.prompt_ids(6, b, Lp, P.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
+    ctx.device_status()
+    assert steps < gen // 2                          # the rule fires: > 2 positions per step
+    _replay_check(P, rec, x.cpu().numpy(), B, tau, bias=(bt, bv, Lp))
+
+
+@pytest.mark.parametrize("cache", ["prefix", "none"])
+def test_native_generate_cache_modes_equal_the_python_decoder(ctx, cache):
+    """fdl_generate in the PrefixCache and no-cache modes, with a planted bias,
+    takes the same steps and decodes the same tokens as the Python decoder of
+    the same mode (the same kernels in the same order)."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    P = _small_params(7, hq=4, hkv=2, bias=True)
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B, tau = 2, 64, 64, 32, 0.9
+    g = synth.rng(67)
+    bt = torch.from_numpy(g.integers(0, P.mask_id, (b, gen)).astype(np.int32)).cuda()
+    bv = torch.from_numpy(g.uniform(0.0, 16.0, (b, gen)).astype(np.float32)).cuda()
+    prompt = synth.prompt_ids(7, b, Lp, P.mask_id)
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B, cache=cache, bias_tok=bt, bias_val=bv)
+    x_py, steps_py = dec.generate(prompt, gen, tau=tau)
+    x_nat, steps_nat = ctx.generate(w.native(), torch.from_numpy(prompt), gen, block=B, tau=tau,
+                                    cache=cache, bias_tok=bt, bias_val=bv)
+    ctx.device_status()
+    assert not x_nat.is_cuda                         # host prompt in, host sequence out
+    assert steps_nat == steps_py
+    assert np.array_equal(x_nat.numpy(), x_py.cpu().numpy())
+
+
+# Two layers at the full widths of the two model families, so that a decode the
+# oracle replays runs the fused split-K calls (RMSNorm prologue, per-CTA query
+# tiles of the q/k/v epilogue, SwiGLU prologue behind grid barriers) and the
+# whole-vocabulary LM head. The LM head's weights are drawn with a wider
+# spread (logit std about 8) so that some confidences exceed tau and steps
+# decode several positions. Logits then carry an error of a few hundredths
+# from the bf16 activations of two layers (the 2e-2 confidence bound at
+# confidence ~0.5 allows ~0.04), so token ids are compared where the oracle's
+# top-2 gap exceeds 0.2, five times that.
+WIDE_TOK_GAP = 0.2
+WIDE_MODELS = {
+    # LLaDA-8B widths: MHA 32 x 128, FFN 12288, vocab 126464, mask id 126336
+    "llada": dict(vocab=126464, hidden=4096, n_q_heads=32, n_kv_heads=32, ffn=12288,
+                  qkv_bias=False, mask_id=126336, batch=1),
+    # Dream-7B (Qwen2.5-7B) widths: GQA 28/4 with q/k/v bias, FFN 18944, vocab 152064
+    "dream": dict(vocab=152064, hidden=3584, n_q_heads=28, n_kv_heads=4, ffn=18944,
+                  qkv_bias=True, mask_id=152063, batch=2),
+}
+
+
+@pytest.mark.parametrize("name", sorted(WIDE_MODELS))
+def test_two_layer_full_width_decode_matches_oracle(ctx, name):
+    """A 2-layer model at the full widths, prompt 64 + gen 64, block 32, tau
+    0.9: every step replayed by the oracle on the GPU's own trajectory
+    (confidences within 2e-2, decisions bit-exact given the GPU's
+    confidences) and, at every step, the LM-head boundary within 1e-5 on the
+    GPU's own final-norm rows."""
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    m = WIDE_MODELS[name]
+    D = m["hidden"]
+    P = synth.model_params(vocab=m["vocab"], hidden=D, n_layers=2, n_q_heads=m["n_q_heads"],
+                           n_kv_heads=m["n_kv_heads"], head_dim=128, ffn=m["ffn"], seed=71,
+                           dtype="bf16", qkv_bias=m["qkv_bias"], lm_std=8.0 / np.sqrt(D))
+    P.mask_id = m["mask_id"]
+    w = DeviceWeights.from_params(P)
+    b, Lp, gen, B, tau = m["batch"], 64, 64, 32, 0.9
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B)
+    prompt = synth.prompt_ids(72, b, Lp, P.mask_id)
+    rec = []
+    x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
+    ctx.device_status()
+    assert steps == len(rec) and steps < gen          # some steps decoded several positions
+    _replay_check(P, rec, x.cpu().numpy(), B, tau, tok_gap=WIDE_TOK_GAP)
 
 
 @pytest.mark.parametrize("seed,tau,hq,hkv,bias", [(0, 0.9, 2, 2, False), (1, 0.5, 4, 2, True),
@@ -326,7 +463,7 @@ def test_tau_one_single_layer_gpu_equals_sequential(ctx):
     x, steps = dec.generate(prompt, 64, tau=1.0, record=rec)
     assert steps == 64
     # each step decodes exactly the position the sequential rule picks
-    for kind, s, xb, mb, conf, tok in rec:
+    for kind, s, xb, mb, conf, tok, _ in rec:
         logits, _ = O.full_forward(P, xb[0])
         c = O.confidence_from_logits(logits[s:s + 32])
         cand = mb[0, s:s + 32] != 0
@@ -360,7 +497,7 @@ def test_dream_shape_full_decode(ctx):
     xf = x.cpu().numpy()
     assert steps == len(rec) and gen // B <= steps <= gen
     total = np.zeros(b, np.int64)
-    for n, (kind, s, xb, mb, conf, tok) in enumerate(rec):
+    for n, (kind, s, xb, mb, conf, tok, _) in enumerate(rec):
         conf, tok = conf.reshape(b, B), tok.reshape(b, B)
         xa, ma, _, nd = O.threshold_unmask(xb, mb, conf, tok, s, B, tau)
         x_next = rec[n + 1][2] if n + 1 < len(rec) else xf

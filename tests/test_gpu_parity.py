@@ -180,7 +180,16 @@ def test_lmhead_bf16_llada_vocab(ctx, rows):
     # hidden 4096, vocab 126464, mask id 126336; batch = rows / 32
     c = llada_lmhead_case(rows)
     conf, tok = run_lmhead(ctx, c)
-    sample = np.arange(rows) if rows <= 64 else synth.rng(rows).choice(rows, 64, replace=False)
+    # every row up to 64; beyond, the first and last row of every 128-row tile
+    # (the MMA's M) plus random rows, 64 in all
+    if rows <= 64:
+        sample = np.arange(rows)
+    else:
+        edges = np.unique(np.concatenate([np.arange(0, rows, 128),
+                                          np.minimum(np.arange(127, rows + 127, 128), rows - 1)]))
+        rest = np.setdiff1d(np.arange(rows), edges)
+        extra = synth.rng(rows).choice(rest, 64 - len(edges), replace=False)
+        sample = np.sort(np.concatenate([edges, extra]))
     ref = O.lmhead_confidence(c.h[sample], c.w, c.bias_tok[sample], c.bias_val[sample])
     err = np.abs(conf[sample] - ref.conf).max()
     assert err <= CONF_TOL, err
