@@ -91,6 +91,11 @@ def parse():
     p.add_argument("--no-kernels", dest="kernels", action="store_false",
                    help="skip the per-kernel roofline cases")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-loop", choices=["device", "host"], default="device",
+                   help="fdl_generate's loop for the e2e decode")
+    p.add_argument("--sweep", action="store_true",
+                   help="instead of the bench line: the block / tau / gen / cache-mode grid "
+                        "with the planted bias, one JSON line per point")
     p.add_argument("--profile-steps", action="store_true",
                    help="also print the per-call time of a cached step and of a refresh")
     p.add_argument("--config", choices=sorted(CONFIGS), default="llada",
@@ -512,18 +517,24 @@ def result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max, 
 
 
 def run_e2e(torch, ctx, w, c, args, rank):
-    """One whole decode through the library's decode entry point (fdl_generate)
-    from a pinned host prompt to a host copy of the sequence: the binding
-    copies the prompt in, the library runs every block, the binding copies the
-    sequence out; CUDA events around the whole call. The bytes per step are per
+    """Whole decodes through the library's decode entry point (fdl_generate)
+    from a pinned host prompt to a host copy of the sequence: the binding copies
+    the prompt in, the library runs every block, the binding copies the sequence
+    out; CUDA events around the whole call. With the device loop (default) the
+    decode is one CUDA graph (each block's cached steps in a conditional WHILE
+    node) that the context keeps: one untimed call captures it, as a server
+    would once per shape, then one call is timed. The bytes per step are per
     block (the bench's step)."""
     from block_kv_cache_b200 import synth
     hp = torch.from_numpy(synth.prompt_ids(7 + rank, c["batch"], c["prompt"],
                                            c["mask_id"])).pin_memory()
     bias = planted_bias(torch, c, rank) if args.planted_bias else (None, None)
     m = w.native()
+    device_loop = args.e2e_loop == "device"
     kw = dict(block=c["block"], tau=c["tau"], cache=args.cache, bias_tok=bias[0],
-              bias_val=bias[1])
+              bias_val=bias[1], device_loop=device_loop)
+    if device_loop:
+        ctx.generate(m, hp, c["gen"], **kw)           # captures and keeps the decode graph
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -531,13 +542,16 @@ def run_e2e(torch, ctx, w, c, args, rank):
     x, steps = ctx.generate(m, hp, c["gen"], **kw)
     e1.record()
     torch.cuda.synchronize()
+    ctx.device_status()
     m.close()
     blocks = c["gen"] // c["block"]
+    d2h = x.numel() * 4 + (4 if device_loop else steps * c["batch"] * 4)
     return {"ms": e0.elapsed_time(e1), "toks": c["batch"] * c["gen"],
-            "h2d": hp.numel() * 4 / blocks,
-            "d2h": (x.numel() * 4 + steps * c["batch"] * 4) / blocks,
-            "path": f"fdl_generate (the library's decode loop) on a host prompt: {steps} decode "
-                    f"steps, one whole decode of {blocks} blocks"}
+            "h2d": hp.numel() * 4 / blocks, "d2h": d2h / blocks,
+            "path": f"fdl_generate (the library's decode loop, "
+                    f"{'device loop: one CUDA graph per decode' if device_loop else 'host loop'}"
+                    f") on a host prompt: {steps} decode steps, one whole decode of {blocks} "
+                    f"blocks"}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -672,6 +686,71 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+# ----------------------------------------------------------------------------- sweeps
+# The pages' ablations on synthetic inputs: block size, threshold and
+# generation length (ICLR reviews, reviews 1-2: the block-size ablation), and
+# the README evaluation table's four columns: the base decode (no cache, one
+# position per step), +cache (DualCache, one position per step), +parallel
+# (no cache, threshold rule) and both. All with the planted logit bias, so
+# that the threshold rule fires as it would on a trained model's confident
+# positions; tau = 1 decodes exactly one position per step.
+SWEEP_GRID = (
+    [dict(block=b, tau=0.9, gen=1024, cache="dual") for b in (8, 16, 32, 64, 128)]
+    + [dict(block=32, tau=t, gen=1024, cache="dual") for t in (0.7, 1.0)]
+    + [dict(block=32, tau=0.9, gen=g, cache="dual") for g in (256, 512)]
+    + [dict(block=32, tau=t, gen=g, cache=m) for g in (256, 512)
+       for m, t in (("none", 1.0), ("dual", 1.0), ("none", 0.9), ("prefix", 0.9),
+                    ("prefix", 1.0))]
+)
+
+
+def run_sweep(args):
+    """One whole decode per grid point (every step graph captured before the
+    timed decode), CUDA events around it; one JSON line per point."""
+    import torch
+    from block_kv_cache_b200 import fdllm, synth
+    from block_kv_cache_b200.model import BlockDecoder, DeviceWeights
+    torch.cuda.set_device(0)
+    base = dict(CFG)
+    ctx = fdllm.Context(0)
+    w = DeviceWeights.random(shape(), seed=1234)
+    for pt in SWEEP_GRID:
+        c = dict(base, **pt)
+        L = c["prompt"] + c["gen"]
+        bias = planted_bias(torch, c, 0)
+        dec = BlockDecoder(ctx, w, c["batch"], L, c["block"], cache=c["cache"],
+                           bias_tok=bias[0], bias_val=bias[1])
+        prompt = torch.from_numpy(synth.prompt_ids(7, c["batch"], c["prompt"],
+                                                   c["mask_id"])).cuda()
+        dec.capture_all(c["prompt"], c["gen"], c["tau"])
+        dec.begin(prompt, c["tau"])                 # untimed: every graph replayed once
+        while not dec.done:
+            dec.block()
+        dec.begin(prompt, c["tau"])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        kinds, toks = {}, 0
+        e0.record()
+        while not dec.done:
+            n, steps = dec.block()
+            toks += n
+            for kind, _, _ in steps:
+                kinds[kind] = kinds.get(kind, 0) + 1
+        e1.record()
+        torch.cuda.synchronize()
+        ctx.device_status()
+        ms = e0.elapsed_time(e1)
+        nsteps = sum(kinds.values())
+        print(json.dumps({"sweep": pt, "tokens": toks, "decode_steps": nsteps,
+                          "tokens_per_step": toks / nsteps, "ms": ms,
+                          "tokens_per_s": toks / (ms / 1e3), "steps_by_kind": kinds}),
+              flush=True)
+        dec.graphs.clear()
+        del dec
+        torch.cuda.empty_cache()
+    ctx.close()
+
+
 def main():
     global WORKLOAD
     args = parse()
@@ -685,6 +764,8 @@ def main():
             WORKLOAD += f" [{k} {v}]"
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_gpu(args)
 

@@ -47,11 +47,20 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not _stale():
+# Instrumented build: kernels record per-CTA event clocks (csrc/timeline.cuh),
+# readable through fdl_timeline_<file>(); a separate library, loaded only when
+# FDLLM_LIB names it.
+LIB_TIMELINE = os.path.join(HERE, "libfdllm_timeline.so")
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          timeline: bool = False) -> str:
+    lib = LIB_TIMELINE if timeline else LIB
+    if not force and not timeline and not _stale():
         return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC, *sources(),
+    tmp = lib + ".tmp"
+    flags = ["-DFDL_TIMELINE"] if timeline else []
+    cmd = [_nvcc(), *NVCC_FLAGS, *flags, *(extra or []), "-I", INCLUDE, "-I", CSRC, *sources(),
            "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
@@ -60,10 +69,11 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
     if verbose and (r.stdout or r.stderr):
         print(r.stdout + r.stderr, file=sys.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    extra = [a for a in sys.argv[1:] if a not in ("--force", "-v")]
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, extra=extra))
+    extra = [a for a in sys.argv[1:] if a not in ("--force", "-v", "--timeline")]
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, extra=extra,
+                timeline="--timeline" in sys.argv))

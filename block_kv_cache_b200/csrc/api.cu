@@ -11,21 +11,41 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <vector>
+
+// The executable graph of the last device-loop decode of a context, kept for
+// the next decode with the same key (fdl_generate with device_loop).
+struct GenGraph {
+    cudaGraphExec_t exec = nullptr;
+    cudaStream_t cap = nullptr, body = nullptr;   // capture streams (non-blocking)
+    // key: everything the captured kernels' arguments depend on
+    uint64_t model = 0;                           // fdl_model id
+    const void* ws = nullptr;
+    size_t ws_bytes = 0;
+    int b = 0, P = 0, gen = 0, B = 0, mode = 0;
+    float tau = 0.f;
+    const void* bias_tok = nullptr;
+    const void* bias_val = nullptr;
+};
 
 struct fdl_ctx {
     int device;
     int sm_count;
-    int* d_err;              // device error word (4 bytes)
+    int* d_err;              // device error word (4 bytes), then at +8 the u64 wait limit
     float* d_acc;            // split-K accumulator of the projections, kept all zeros
     size_t acc_bytes;
     unsigned* d_sync;        // grid-barrier words of the fused kernels (zeroed)
+    GenGraph* gen;           // cached device-loop decode graph, or NULL
 };
 
 // Split-K accumulator of the few-token projections (zeroed at creation; every
 // kernel that adds into it leaves it zeroed again): room for 256 rows x 32768.
 static const size_t kAccBytes = (size_t)256 * 32768 * 4;
 static const size_t kSyncBytes = 256;
+// Default limit of the kernels' progress waits (the device-side default too).
+static const uint64_t kDefaultWaitNs = 2000000000ull;
+static const uint64_t kMaxWaitNs = 60000000000ull;
 
 namespace fdl {
 void noalloc_forget(int dev);
@@ -105,6 +125,8 @@ int check_lm(const fdl_lmhead_desc* d) {
 
 }  // namespace
 
+void release_gen_graph(fdl_ctx* ctx);
+
 extern "C" {
 
 int fdl_abi_version(void) { return FDL_ABI_VERSION; }
@@ -133,9 +155,15 @@ int fdl_create(fdl_ctx** out, int device) {
     c->d_err = nullptr;
     c->d_acc = nullptr;
     c->d_sync = nullptr;
+    c->gen = nullptr;
     c->acc_bytes = kAccBytes;
-    e = cudaMalloc(&c->d_err, sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, sizeof(int));
+    // 16 bytes: the error word, then (8-byte aligned) the limit of the
+    // kernels' progress waits in ns
+    const uint64_t limit = kDefaultWaitNs;
+    e = cudaMalloc(&c->d_err, 16);
+    if (e == cudaSuccess) e = cudaMemset(c->d_err, 0, 16);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(reinterpret_cast<char*>(c->d_err) + 8, &limit, 8, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMalloc(&c->d_acc, kAccBytes);
     if (e == cudaSuccess) e = cudaMemset(c->d_acc, 0, kAccBytes);
     if (e == cudaSuccess) e = cudaMalloc(&c->d_sync, kSyncBytes);
@@ -156,11 +184,25 @@ int fdl_create(fdl_ctx** out, int device) {
 int fdl_destroy(fdl_ctx* ctx) {
     if (!ctx) return FDL_OK;
     DeviceGuard g(ctx->device);
+    release_gen_graph(ctx);
     if (ctx->d_err) cudaFree(ctx->d_err);
     if (ctx->d_acc) cudaFree(ctx->d_acc);
     if (ctx->d_sync) cudaFree(ctx->d_sync);
     delete ctx;
     return FDL_OK;
+}
+
+int fdl_set_wait_timeout(fdl_ctx* ctx, uint64_t ns) {
+    if (!ctx) return fail(FDL_EINVAL, "set_wait_timeout: ctx is NULL");
+    if (ns < 1 || ns > kMaxWaitNs)
+        return fail(FDL_EINVAL, "set_wait_timeout: %llu ns outside [1, %llu]",
+                    (unsigned long long)ns, (unsigned long long)kMaxWaitNs);
+    DeviceGuard g(ctx->device);
+    if (!g.ok) return fail(FDL_ECUDA, "set_wait_timeout: cannot select device");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpy(reinterpret_cast<char*>(ctx->d_err) + 8, &ns, 8, cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "set_wait_timeout");
 }
 
 int fdl_get_device_status(fdl_ctx* ctx, void* stream) {
@@ -304,6 +346,15 @@ int fdl_threshold_unmask(fdl_ctx* ctx, const fdl_unmask_desc* desc, const float*
 }
 
 }  // extern "C"
+
+void release_gen_graph(fdl_ctx* ctx) {
+    if (!ctx->gen) return;
+    if (ctx->gen->exec) cudaGraphExecDestroy(ctx->gen->exec);
+    if (ctx->gen->cap) cudaStreamDestroy(ctx->gen->cap);
+    if (ctx->gen->body) cudaStreamDestroy(ctx->gen->body);
+    delete ctx->gen;
+    ctx->gen = nullptr;
+}
 
 namespace fdl {
 // Device id of a context (for library-internal entry points in other files).
@@ -565,6 +616,7 @@ int fdl_full_attention(fdl_ctx* ctx, const fdl_attn_desc* desc, const void* q,
 
 // ---- the whole decode ------------------------------------------------------------
 struct fdl_model {
+    uint64_t id;              // unique per fdl_model_create (keys the cached decode graph)
     fdl_model_desc d;
     const void* embed;
     const float* final_norm;
@@ -610,7 +662,7 @@ __global__ void tail_rows_kernel(int32_t* __restrict__ tail, int32_t* __restrict
 struct GenLayout {
     size_t kc, vc, h_full, x_full, q_full, o_full, f_full, h_blk, x_blk, q_blk, o_blk, f_blk,
         xn, conf, tok, masked, counts, maps, tail_map, tail_blk, bias_tok, bias_val, rope, lm_ws,
-        total;
+        x, steps, total;
     size_t kv_layer;    // bytes of one layer's K (or V) cache
     size_t lm_bytes;
 };
@@ -652,8 +704,247 @@ GenLayout gen_layout(const fdl_model_desc& d, int b, int L, int B, size_t lm_byt
     g.rope = take((size_t)L * hd * 4);
     g.lm_bytes = lm_bytes;
     g.lm_ws = take(lm_bytes);
+    g.x = take(rf * 4);              // the decode's token ids (copied out at the end)
+    g.steps = take(16);              // decode steps taken (device loop)
     g.total = off;
     return g;
+}
+
+// One decode of fdl_generate: its shapes, the workspace pieces, and the
+// issuing of a block's set-up and of one decode step on a given stream (used by
+// the host loop and, captured, by the device loop).
+struct GenRun {
+    fdl_ctx* ctx;
+    const fdl_model* m;
+    int b, P, gen, B, L, mode;
+    float tau;
+    const int32_t* bias_tok;
+    const float* bias_val;
+    GenLayout g;
+    char* base;
+
+    void* at(size_t off) const { return static_cast<void*>(base + off); }
+    int32_t* x() const { return (int32_t*)at(g.x); }
+    uint8_t* masked() const { return (uint8_t*)at(g.masked); }
+    int32_t* remaining() const { return (int32_t*)at(g.counts); }
+    int32_t* maps() const { return (int32_t*)at(g.maps); }
+
+    // per block, before its first step: the planted bias of its rows and, for
+    // the PrefixCache, its row maps
+    int block_prep(int blk, cudaStream_t st) const {
+        const int s = P + blk * B;
+        cudaError_t e = cudaSuccess;
+        if (bias_tok) {
+            // this block's planted bias, [b, gen] -> [b, B] contiguous
+            e = cudaMemcpy2DAsync(at(g.bias_tok), (size_t)B * 4, bias_tok + (s - P),
+                                  (size_t)gen * 4, (size_t)B * 4, b, cudaMemcpyDeviceToDevice, st);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2DAsync(at(g.bias_val), (size_t)B * 4, bias_val + (s - P),
+                                      (size_t)gen * 4, (size_t)B * 4, b,
+                                      cudaMemcpyDeviceToDevice, st);
+        }
+        if (e == cudaSuccess && mode == FDL_CACHE_PREFIX) {
+            tail_rows_kernel<<<64, 256, 0, st>>>((int32_t*)at(g.tail_map),
+                                                 (int32_t*)at(g.tail_blk), b, L, s, B);
+            e = cudaGetLastError();
+        }
+        return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: block set-up");
+    }
+
+    // The layers over rows = b * n token rows at positions [pos0, pos0 + n) of
+    // every sequence. full: their K/V go into the caches and they attend over
+    // the whole cache (refresh: pos0 = 0, n = L; PrefixCache step: pos0 = s,
+    // n = L - s); otherwise the fused DualCache step of the block rows.
+    int layers(float* h, void* xb, void* q, void* o, void* f, int rows, bool full, int pos0,
+               int n, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        const int D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads, hd = 128;
+        void* stream = (void*)st;
+        const float* rope = (const float*)at(g.rope);
+        int rc = FDL_OK;
+        for (int li = 0; li < d.n_layers && rc == FDL_OK; ++li) {
+            const fdl_layer_weights& W = m->layers[li];
+            void* kl = base + g.kc + g.kv_layer * li;
+            void* vl = base + g.vc + g.kv_layer * li;
+            const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
+            if (full) {
+                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
+                rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
+                if (!rc) rc = fdl_qkv_rope_store(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl, vl,
+                                                 stream);
+                if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
+            } else {
+                rc = fdl_qkv_attention(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv, W.bias,
+                                       rope, q, kl, vl, o, stream);
+            }
+            if (!rc) rc = fdl_linear_residual(ctx, rows, D, Hq * hd, o, W.wo, h, stream);
+            if (!rc) rc = fdl_ffn(ctx, rows, D, F, W.ffn_norm, d.rms_eps, xb, W.w_gu, W.w_down, f,
+                                  h, stream);
+        }
+        return rc;
+    }
+
+    // One decode step of block blk: the forward (the refresh when `first` or
+    // without a cache, else the cache mode's step), the LM head with the
+    // confidence reduction, and the threshold unmask (remaining[] written).
+    int step(int blk, bool first, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        const int D = d.hidden, rf = b * L, rb = b * B, s = P + blk * B;
+        void* stream = (void*)st;
+        const int32_t* row_map = maps() + (size_t)(s / B) * rb;
+        float* h_full = (float*)at(g.h_full);
+        float* h_blk = (float*)at(g.h_blk);
+        int rc;
+        if (first || mode == FDL_CACHE_NONE) {
+            // full forward over every position: all K/V caches rewritten
+            rc = fdl_embed(ctx, rf, D, x(), nullptr, m->embed, h_full, stream);
+            if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full), at(g.f_full),
+                                 rf, true, 0, L, st);
+            if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, row_map, m->final_norm, d.rms_eps,
+                                      at(g.xn), stream);
+        } else if (mode == FDL_CACHE_PREFIX) {
+            // PrefixCache step: the block and the suffix over the cached prefix
+            const int n = L - s;
+            rc = fdl_embed(ctx, b * n, D, x(), (const int32_t*)at(g.tail_map), m->embed, h_full,
+                           stream);
+            if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full), at(g.f_full),
+                                 b * n, true, s, n, st);
+            if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, (const int32_t*)at(g.tail_blk),
+                                      m->final_norm, d.rms_eps, at(g.xn), stream);
+        } else {
+            // DualCache step: only the block's rows
+            rc = fdl_embed(ctx, rb, D, x(), row_map, m->embed, h_blk, stream);
+            if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), rb,
+                                 false, s, B, st);
+            if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_blk, nullptr, m->final_norm, d.rms_eps,
+                                      at(g.xn), stream);
+        }
+        const fdl_lmhead_desc lmd{rb, D, d.vocab, FDL_BF16};
+        if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head,
+                                            bias_tok ? (const int32_t*)at(g.bias_tok) : nullptr,
+                                            bias_tok ? (const float*)at(g.bias_val) : nullptr,
+                                            (float*)at(g.conf), (int32_t*)at(g.tok), at(g.lm_ws),
+                                            g.lm_bytes, stream);
+        const fdl_unmask_desc ud{b, L, s, B, tau};
+        if (!rc) rc = fdl_threshold_unmask(ctx, &ud, (const float*)at(g.conf),
+                                           (const int32_t*)at(g.tok), x(), masked(), remaining(),
+                                           remaining() + b, stream);
+        return rc;
+    }
+};
+
+// After a step of the device loop: count it, and set the block's loop
+// condition to "a sequence still has a masked position in the block".
+__global__ void loop_cond_kernel(cudaGraphConditionalHandle h, const int32_t* __restrict__ rem,
+                                 int b, int32_t* __restrict__ steps) {
+    if (threadIdx.x != 0) return;
+    int any = 0;
+    for (int i = 0; i < b; ++i) any |= rem[i] > 0;
+    cudaGraphSetConditional(h, any ? 1u : 0u);
+    *steps += 1;
+}
+
+bool same_key(const GenGraph* c, const GenRun& r, size_t ws_bytes) {
+    return c && c->exec && c->model == r.m->id && c->ws == r.base && c->ws_bytes == ws_bytes &&
+           c->b == r.b && c->P == r.P && c->gen == r.gen && c->B == r.B && c->mode == r.mode &&
+           c->tau == r.tau && c->bias_tok == r.bias_tok && c->bias_val == r.bias_val;
+}
+
+// Capture the whole decode as one CUDA graph: per block its set-up and first
+// step (the refresh), then a conditional WHILE node whose body is one cached
+// step; a small kernel after every step sets the condition from the counts of
+// masked positions left, so the block's steps repeat on the device with no
+// host round trip. Captured on the context's own non-blocking streams.
+int build_gen_graph(const GenRun& r, GenGraph* c, cudaGraphExec_t* out) {
+    *out = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (!c->cap) e = cudaStreamCreateWithFlags(&c->cap, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !c->body) e = cudaStreamCreateWithFlags(&c->body, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "generate: capture streams");
+    cudaStream_t cs = c->cap;
+    e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return cuda_fail(e, "generate: begin capture");
+    int32_t* steps = (int32_t*)r.at(r.g.steps);
+    int rc = FDL_OK;
+    cudaGraph_t graph = nullptr;
+    for (int blk = 0; rc == FDL_OK && blk < r.gen / r.B; ++blk) {
+        cudaStreamCaptureStatus status;
+        const cudaGraphNode_t* deps = nullptr;
+        size_t ndeps = 0;
+        e = cudaStreamGetCaptureInfo(cs, &status, nullptr, &graph, &deps, &ndeps);
+        cudaGraphConditionalHandle h = 0;
+        if (e == cudaSuccess) e = cudaGraphConditionalHandleCreate(&h, graph, 0, 0);
+        if (e != cudaSuccess) { rc = cuda_fail(e, "generate: condition"); break; }
+        rc = r.block_prep(blk, cs);
+        if (!rc) rc = r.step(blk, true, cs);
+        if (rc) break;
+        loop_cond_kernel<<<1, 32, 0, cs>>>(h, r.remaining(), r.b, steps);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaStreamGetCaptureInfo(cs, &status, nullptr, &graph, &deps, &ndeps);
+        cudaGraphNodeParams cp = {};
+        cp.type = cudaGraphNodeTypeConditional;
+        cp.conditional.handle = h;
+        cp.conditional.type = cudaGraphCondTypeWhile;
+        cp.conditional.size = 1;
+        cudaGraphNode_t node = nullptr;
+        if (e == cudaSuccess) e = cudaGraphAddNode(&node, graph, deps, ndeps, &cp);
+        if (e == cudaSuccess)
+            e = cudaStreamUpdateCaptureDependencies(cs, &node, 1, cudaStreamSetCaptureDependencies);
+        if (e != cudaSuccess) { rc = cuda_fail(e, "generate: loop node"); break; }
+        // the body: one cached step, then the condition again
+        cudaGraph_t body = cp.conditional.phGraph_out[0];
+        e = cudaStreamBeginCaptureToGraph(c->body, body, nullptr, nullptr, 0,
+                                          cudaStreamCaptureModeThreadLocal);
+        if (e != cudaSuccess) { rc = cuda_fail(e, "generate: body capture"); break; }
+        rc = r.step(blk, false, c->body);
+        if (!rc) {
+            loop_cond_kernel<<<1, 32, 0, c->body>>>(h, r.remaining(), r.b, steps);
+            e = cudaGetLastError();
+        }
+        cudaGraph_t body_out = nullptr;
+        const cudaError_t e2 = cudaStreamEndCapture(c->body, &body_out);
+        if (!rc && e == cudaSuccess) e = e2;
+        if (!rc && e != cudaSuccess) rc = cuda_fail(e, "generate: body");
+    }
+    cudaGraph_t whole = nullptr;
+    const cudaError_t e3 = cudaStreamEndCapture(cs, &whole);
+    if (!rc && e3 != cudaSuccess) rc = cuda_fail(e3, "generate: end capture");
+    if (!rc) {
+        e = cudaGraphInstantiate(out, whole, 0);
+        if (e != cudaSuccess) rc = cuda_fail(e, "generate: instantiate");
+    }
+    if (whole) cudaGraphDestroy(whole);
+    return rc;
+}
+
+int run_device_loop(const GenRun& r, cudaStream_t st) {
+    fdl_ctx* ctx = r.ctx;
+    const size_t ws_bytes = r.g.total;
+    if (!same_key(ctx->gen, r, ws_bytes)) {
+        if (!ctx->gen) ctx->gen = new GenGraph;
+        GenGraph* c = ctx->gen;
+        if (c->exec) {
+            cudaGraphExecDestroy(c->exec);
+            c->exec = nullptr;
+        }
+        cudaGraphExec_t exec = nullptr;
+        const int rc = build_gen_graph(r, c, &exec);
+        if (rc) return rc;
+        c->exec = exec;
+        c->model = r.m->id;
+        c->ws = r.base;
+        c->ws_bytes = ws_bytes;
+        c->b = r.b;
+        c->P = r.P;
+        c->gen = r.gen;
+        c->B = r.B;
+        c->mode = r.mode;
+        c->tau = r.tau;
+        c->bias_tok = r.bias_tok;
+        c->bias_val = r.bias_val;
+    }
+    const cudaError_t e = cudaGraphLaunch(ctx->gen->exec, st);
+    return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: graph launch");
 }
 
 bool model_desc_ok(const fdl_model_desc* d) {
@@ -685,7 +976,9 @@ int fdl_model_create(const fdl_model_desc* desc, const fdl_model_weights* w, fdl
         return fail(FDL_EINVAL, "model_create: NULL weight pointer");
     if (!aligned16(w->embed) || !aligned16(w->final_norm) || !aligned16(w->lm_head))
         return fail(FDL_EINVAL, "model_create: weights must be 16-byte aligned");
+    static std::atomic<uint64_t> next_id{1};
     fdl_model* m = new fdl_model;
+    m->id = next_id++;
     m->d = *desc;
     m->embed = w->embed;
     m->final_norm = w->final_norm;
@@ -717,167 +1010,101 @@ size_t fdl_generate_workspace_bytes(fdl_ctx* ctx, const fdl_model* m, int batch,
 }
 
 int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b, int P, int gen,
-                 int B, float tau, const fdl_generate_opts* opts, int32_t* x, int* steps_out,
+                 int B, float tau, const fdl_generate_opts* opts, int32_t* out_x, int* steps_out,
                  void* ws, size_t ws_bytes, void* stream) {
     if (!ctx || !m) return fail(FDL_EINVAL, "generate: ctx or model is NULL");
-    if (!prompt || !x || !steps_out) return fail(FDL_EINVAL, "generate: NULL buffer");
+    if (!prompt || !out_x || !steps_out) return fail(FDL_EINVAL, "generate: NULL buffer");
     if (b < 1 || B < 1 || B > 128 || P < 0 || gen < B || P % B || gen % B)
         return fail(FDL_EINVAL, "generate: need batch >= 1, 1 <= block <= 128, prompt_len and "
                     "gen_len (>= block) multiples of block");
     if (!(tau >= 0.f && tau <= 1.f)) return fail(FDL_EINVAL, "generate: tau must be in [0, 1]");
-    const int mode = opts ? opts->cache : FDL_CACHE_DUAL;
-    if (mode != FDL_CACHE_DUAL && mode != FDL_CACHE_PREFIX && mode != FDL_CACHE_NONE)
-        return fail(FDL_EINVAL, "generate: unknown cache mode %d", mode);
-    const int32_t* bias_tok = opts ? opts->bias_tok : nullptr;
-    const float* bias_val = opts ? opts->bias_val : nullptr;
-    if ((bias_tok == nullptr) != (bias_val == nullptr))
+    GenRun r;
+    r.ctx = ctx;
+    r.m = m;
+    r.b = b;
+    r.P = P;
+    r.gen = gen;
+    r.B = B;
+    r.tau = tau;
+    r.mode = opts ? opts->cache : FDL_CACHE_DUAL;
+    const bool device_loop = opts && opts->device_loop;
+    if (r.mode != FDL_CACHE_DUAL && r.mode != FDL_CACHE_PREFIX && r.mode != FDL_CACHE_NONE)
+        return fail(FDL_EINVAL, "generate: unknown cache mode %d", r.mode);
+    r.bias_tok = opts ? opts->bias_tok : nullptr;
+    r.bias_val = opts ? opts->bias_val : nullptr;
+    if ((r.bias_tok == nullptr) != (r.bias_val == nullptr))
         return fail(FDL_EINVAL, "generate: bias_tok and bias_val go together");
     const fdl_model_desc& d = m->d;
-    const int L = P + gen, D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads;
-    const int hd = 128, rf = b * L, rb = b * B;
-    if (mode == FDL_CACHE_PREFIX && L % 32)
+    r.L = P + gen;
+    if (r.mode == FDL_CACHE_PREFIX && r.L % 32)
         return fail(FDL_EINVAL, "generate: the PrefixCache mode needs prompt_len + gen_len and "
                     "the block starts at multiples of 32");
-    const GenLayout g = gen_layout(d, b, L, B, lm_ws_bytes(ctx, d, rb));
-    if (!ws || ws_bytes < g.total)
-        return fail(FDL_EWORKSPACE, "generate: workspace of %zu bytes needed", g.total);
+    const int rf = b * r.L, rb = b * B;
+    r.g = gen_layout(d, b, r.L, B, lm_ws_bytes(ctx, d, rb));
+    if (!ws || ws_bytes < r.g.total)
+        return fail(FDL_EWORKSPACE, "generate: workspace of %zu bytes needed", r.g.total);
     if (((uintptr_t)ws & 255u) != 0) return fail(FDL_EINVAL, "generate: ws must be 256-byte aligned");
+    r.base = static_cast<char*>(ws);
     DeviceGuard guard(ctx->device);
+    if (!guard.ok) return fail(FDL_ECUDA, "generate: cannot select device");
     cudaStream_t st = (cudaStream_t)stream;
-    char* base = static_cast<char*>(ws);
-    auto at = [&](size_t off) { return static_cast<void*>(base + off); };
-    char* kc = base + g.kc;
-    char* vc = base + g.vc;
-    float* h_full = (float*)at(g.h_full);
-    float* h_blk = (float*)at(g.h_blk);
-    float* conf = (float*)at(g.conf);
-    int32_t* tok = (int32_t*)at(g.tok);
-    uint8_t* masked = (uint8_t*)at(g.masked);
-    int32_t* remaining = (int32_t*)at(g.counts);
-    int32_t* n_decoded = remaining + b;
-    int32_t* maps = (int32_t*)at(g.maps);
-    int32_t* tail_map = (int32_t*)at(g.tail_map);
-    int32_t* tail_blk = (int32_t*)at(g.tail_blk);
-    int32_t* blk_bias_tok = bias_tok ? (int32_t*)at(g.bias_tok) : nullptr;
-    float* blk_bias_val = bias_tok ? (float*)at(g.bias_val) : nullptr;
-    float* rope = (float*)at(g.rope);
-    const int nblk = (L + B - 1) / B;
+    int32_t* x = r.x();
+    const int nblk = (r.L + B - 1) / B;
 
     // state: x = prompts then mask ids, masked = the generated positions
     cudaError_t e = cudaSuccess;
     fill_i32_kernel<<<148, 256, 0, st>>>(x, (size_t)rf, d.mask_id);
     if (e == cudaSuccess && P > 0)
-        e = cudaMemcpy2DAsync(x, (size_t)L * 4, prompt, (size_t)P * 4, (size_t)P * 4, b,
+        e = cudaMemcpy2DAsync(x, (size_t)r.L * 4, prompt, (size_t)P * 4, (size_t)P * 4, b,
                               cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(masked, 0, (size_t)rf, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(r.masked(), 0, (size_t)rf, st);
     if (e == cudaSuccess)
-        e = cudaMemset2DAsync(masked + P, (size_t)L, 1, (size_t)gen, b, st);
-    block_rows_kernel<<<64, 256, 0, st>>>(maps, b, L, B, nblk);
+        e = cudaMemset2DAsync(r.masked() + P, (size_t)r.L, 1, (size_t)gen, b, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(r.at(r.g.steps), 0, 16, st);
+    block_rows_kernel<<<64, 256, 0, st>>>(r.maps(), b, r.L, B, nblk);
     if (e == cudaSuccess) e = cudaGetLastError();
     {
-        std::vector<float> host_rope((size_t)L * hd);
-        int rc = fdl_rope_table((double)d.rope_theta, L, hd, host_rope.data());
+        std::vector<float> host_rope((size_t)r.L * 128);
+        int rc = fdl_rope_table((double)d.rope_theta, r.L, 128, host_rope.data());
         if (rc) return rc;
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(rope, host_rope.data(), host_rope.size() * 4,
+            e = cudaMemcpyAsync(r.at(r.g.rope), host_rope.data(), host_rope.size() * 4,
                                 cudaMemcpyHostToDevice, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);   // host_rope goes out of scope
     }
     if (e != cudaSuccess) return cuda_fail(e, "generate: set-up");
 
-    const fdl_lmhead_desc lmd{rb, D, d.vocab, FDL_BF16};
-    // The layers over rows = b * n token rows at positions [pos0, pos0 + n) of
-    // every sequence. full: their K/V go into the caches and they attend over
-    // the whole cache (refresh: pos0 = 0, n = L; PrefixCache step: pos0 = s,
-    // n = L - s); otherwise the fused DualCache step of the block rows.
-    auto layers = [&](float* h, void* xb, void* q, void* o, void* f, int rows, bool full,
-                      int pos0, int n) -> int {
-        int rc = FDL_OK;
-        for (int li = 0; li < d.n_layers && rc == FDL_OK; ++li) {
-            const fdl_layer_weights& W = m->layers[li];
-            void* kl = kc + g.kv_layer * li;
-            void* vl = vc + g.kv_layer * li;
-            if (full) {
-                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
-                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
-                rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
-                if (!rc) rc = fdl_qkv_rope_store(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl, vl,
-                                                 stream);
-                if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
-            } else {
-                const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
-                rc = fdl_qkv_attention(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv, W.bias,
-                                       rope, q, kl, vl, o, stream);
-            }
-            if (!rc) rc = fdl_linear_residual(ctx, rows, D, Hq * hd, o, W.wo, h, stream);
-            if (!rc) rc = fdl_ffn(ctx, rows, D, F, W.ffn_norm, d.rms_eps, xb, W.w_gu, W.w_down, f,
-                                  h, stream);
-        }
-        return rc;
-    };
-
-    std::vector<int32_t> host_rem(b);
     int steps = 0;
-    for (int blk = 0; blk < gen / B; ++blk) {
-        const int s = P + blk * B;
-        const int32_t* row_map = maps + (size_t)(s / B) * rb;
-        if (bias_tok) {
-            // this block's planted bias, [b, gen] -> [b, B] contiguous
-            e = cudaMemcpy2DAsync(blk_bias_tok, (size_t)B * 4, bias_tok + (s - P), (size_t)gen * 4,
-                                  (size_t)B * 4, b, cudaMemcpyDeviceToDevice, st);
-            if (e == cudaSuccess)
-                e = cudaMemcpy2DAsync(blk_bias_val, (size_t)B * 4, bias_val + (s - P),
-                                      (size_t)gen * 4, (size_t)B * 4, b,
-                                      cudaMemcpyDeviceToDevice, st);
-            if (e != cudaSuccess) return cuda_fail(e, "generate: bias");
-        }
-        if (mode == FDL_CACHE_PREFIX) {
-            tail_rows_kernel<<<64, 256, 0, st>>>(tail_map, tail_blk, b, L, s, B);
-            e = cudaGetLastError();
-            if (e != cudaSuccess) return cuda_fail(e, "generate: row maps");
-        }
-        for (bool first = true;; first = false) {
-            int rc;
-            if (first || mode == FDL_CACHE_NONE) {
-                // full forward over every position: all K/V caches rewritten
-                rc = fdl_embed(ctx, rf, D, x, nullptr, m->embed, h_full, stream);
-                if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full),
-                                     at(g.f_full), rf, true, 0, L);
-                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, row_map, m->final_norm, d.rms_eps,
-                                          at(g.xn), stream);
-            } else if (mode == FDL_CACHE_PREFIX) {
-                // PrefixCache step: the block and the suffix over the cached prefix
-                const int n = L - s;
-                rc = fdl_embed(ctx, b * n, D, x, tail_map, m->embed, h_full, stream);
-                if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full),
-                                     at(g.f_full), b * n, true, s, n);
-                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_full, tail_blk, m->final_norm,
-                                          d.rms_eps, at(g.xn), stream);
-            } else {
-                // DualCache step: only the block's rows
-                rc = fdl_embed(ctx, rb, D, x, row_map, m->embed, h_blk, stream);
-                if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), rb,
-                                     false, s, B);
-                if (!rc) rc = fdl_rmsnorm(ctx, rb, D, h_blk, nullptr, m->final_norm, d.rms_eps,
-                                          at(g.xn), stream);
-            }
-            if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head, blk_bias_tok,
-                                                blk_bias_val, conf, tok, at(g.lm_ws), g.lm_bytes,
-                                                stream);
-            const fdl_unmask_desc ud{b, L, s, B, tau};
-            if (!rc) rc = fdl_threshold_unmask(ctx, &ud, conf, tok, x, masked, remaining, n_decoded,
-                                               stream);
+    if (device_loop) {
+        int rc = run_device_loop(r, st);
+        if (rc) return rc;
+        int32_t dev_steps = 0;
+        e = cudaMemcpyAsync(&dev_steps, r.at(r.g.steps), 4, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return cuda_fail(e, "generate: step count");
+        steps = dev_steps;
+    } else {
+        std::vector<int32_t> host_rem(b);
+        for (int blk = 0; blk < gen / B; ++blk) {
+            int rc = r.block_prep(blk, st);
             if (rc) return rc;
-            ++steps;
-            e = cudaMemcpyAsync(host_rem.data(), remaining, (size_t)b * 4, cudaMemcpyDeviceToHost,
-                                st);
-            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-            if (e != cudaSuccess) return cuda_fail(e, "generate: counters");
-            int rem = 0;
-            for (int i = 0; i < b; ++i) rem = host_rem[i] > rem ? host_rem[i] : rem;
-            if (rem == 0) break;
+            for (bool first = true;; first = false) {
+                rc = r.step(blk, first, st);
+                if (rc) return rc;
+                ++steps;
+                e = cudaMemcpyAsync(host_rem.data(), r.remaining(), (size_t)b * 4,
+                                    cudaMemcpyDeviceToHost, st);
+                if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+                if (e != cudaSuccess) return cuda_fail(e, "generate: counters");
+                int rem = 0;
+                for (int i = 0; i < b; ++i) rem = host_rem[i] > rem ? host_rem[i] : rem;
+                if (rem == 0) break;
+            }
         }
     }
+    e = cudaMemcpyAsync(out_x, x, (size_t)rf * 4, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "generate: output");
     *steps_out = steps;
     return FDL_OK;
 }

@@ -43,6 +43,7 @@
 #include "gemm.h"
 #include "launch.h"
 #include "sm100.cuh"
+#include "timeline.cuh"
 
 namespace fdl {
 
@@ -313,6 +314,9 @@ __device__ __forceinline__ void qkv_zero_q(const ProQKV& pro, const AttnArgs& a,
     }
 }
 
+// Timeline events (timeline builds): 0 entry, 1 after the dependency wait and
+// the prologue, 2 first S MMA issued, 3 last PV committed, 4 first P tile
+// written, 5 epilogue start, 6 split merge done, 7 exit.
 template <int D, int MT, class Pro>
 __global__ void __launch_bounds__(Att4<D, MT>::THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -341,6 +345,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11 + 4 * STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+    constexpr int tlk = Pro::kActive ? 1 : (MT == 2 ? 2 : 0);
+    if (threadIdx.x == 0) FDL_TL(tlk, 0);
     const int split = blockIdx.x;                    // == rank in the cluster
     const int g = blockIdx.y / a.n_chunks, chunk = blockIdx.y % a.n_chunks;
     const int bb = blockIdx.z;
@@ -451,6 +457,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         __syncthreads();
     }
     pdl_trigger();
+    if (threadIdx.x == 0) FDL_TL(tlk, 1);
     bool ok = *abort_flag == 0;
 
     if (warp == S::TMA_WARP) {
@@ -521,18 +528,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             if (!ok) {
                 // gave up: every copy requested into this CTA's shared memory must
                 // land before the CTA exits (the last STAGES of each operand)
-                volatile int no_abort = 0;
                 for (int u = (nk > STAGES ? nk - STAGES : 0); u < nk; ++u)
-                    mbar_wait(k_full(u % STAGES), (u / STAGES) & 1, &no_abort, a.err);
+                    mbar_wait_drain(k_full(u % STAGES), (u / STAGES) & 1, a.err);
                 for (int u = (nv > STAGES ? nv - STAGES : 0); u < nv; ++u)
-                    mbar_wait(v_full(u % STAGES), (u / STAGES) & 1, &no_abort, a.err);
+                    mbar_wait_drain(v_full(u % STAGES), (u / STAGES) & 1, a.err);
                 for (int u = nv; u < STAGES && u < nt; ++u)   // early V not yet counted
                     if ((early >> u) & 1u)
-                        mbar_wait(v_full(u), 0, &no_abort, a.err);
+                        mbar_wait_drain(v_full(u), 0, a.err);
                 for (int u = nk; u < STAGES && u < nt; ++u)
                     if ((early >> u) & 1u)
-                        mbar_wait(k_full(u), 0, &no_abort, a.err);
-                if (q_issued) mbar_wait(bar_q, 0, &no_abort, a.err);
+                        mbar_wait_drain(k_full(u), 0, a.err);
+                if (q_issued) mbar_wait_drain(bar_q, 0, a.err);
             }
         }
     } else if (warp == S::MMA_WARP) {
@@ -565,6 +571,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                             }
                         umma_commit(o_done(pbuf));
                         umma_commit(v_empty(su));
+                        if (npv + 1 == nt) FDL_TL(tlk, 3);
                         ++npv;
                         moved = true;
                     }
@@ -588,6 +595,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                             }
                         umma_commit(s_full(b2));
                         umma_commit(k_empty(st));
+                        if (ns == 0) FDL_TL(tlk, 2);
                         ++ns;
                         moved = true;
                     }
@@ -699,10 +707,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                 fence_proxy_async();
                 tc_fence_before();
                 mbar_arrive(p_full(b2));
+                if (t == 0 && threadIdx.x == 0) FDL_TL(tlk, 4);
             }
             // ----------------------------------------------------------- epilogue
             if (ok)
                 ok = mbar_wait_warp(o_done((nt - 1) & 1), ((nt - 1) >> 1) & 1, abort_flag, a.err);
+            if (threadIdx.x == 0) FDL_TL(tlk, 5);
             // the live softmax warps agree on running the epilogue; every wait
             // above is bounded, so all of them get here
             named_sync(1, live_threads);
@@ -772,8 +782,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if (!rcv_ready) cluster_wait();
         // every split's rows have landed (bounded; on the give-up path still wait
         // for what is in flight, so that no push lands after this CTA has left)
-        volatile int no_abort = 0;
-        const bool got = own == 0 || mbar_wait(bar_rcv, 0, &no_abort, a.err);
+        const bool got = own == 0 || mbar_wait_drain(bar_rcv, 0, a.err);
         const int items = got && *abort_flag == 0 ? own * (D / 8) : 0;
         for (int it = threadIdx.x; it < items; it += S::THREADS) {
             const int j = it / (D / 8), d8 = it % (D / 8);
@@ -874,6 +883,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         }
         cluster_sync();                    // no CTA leaves while others read its smem
     }
+    if (threadIdx.x == 0) FDL_TL(tlk, 6);
     // every split of this head has read the q sums (split 0 has received every
     // split's partial, or passed the cluster barrier above, or, with one split,
     // the barrier after the prologue)
@@ -885,6 +895,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         tc_fence_after();
         tmem_dealloc(tmem, S::TMEM_ALLOC);
     }
+    if (threadIdx.x == 0) FDL_TL(tlk, 7);
 }
 
 template <int D, int MT, class Pro>
@@ -999,3 +1010,5 @@ cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads,
 }
 
 }  // namespace fdl
+
+FDL_TL_READER(fdl_timeline_attention)

@@ -23,6 +23,9 @@
 #include "common.cuh"
 #include "gemm.h"
 #include "sm100.cuh"
+#include "timeline.cuh"
+
+#include <type_traits>
 
 namespace fdl {
 namespace {
@@ -296,6 +299,26 @@ struct ProRMSNorm {
     }
 };
 
+// Kind of an instrumented launch (timeline builds): which call it serves.
+template <class Epi, class Pro>
+__device__ __forceinline__ constexpr int sk_tl_kind() {
+    if constexpr (std::is_same<Epi, SkAccum>::value && std::is_same<Pro, ProRMSNorm>::value)
+        return 0;                                    // q/k/v or gate/up sums with the RMSNorm
+    else if constexpr (std::is_same<Epi, SkResid>::value && std::is_same<Pro, ProSwiGLU>::value)
+        return 1;                                    // down projection with the SwiGLU
+    else if constexpr (std::is_same<Epi, SkResid>::value)
+        return 2;                                    // O projection
+    else if constexpr (std::is_same<Epi, SkAccum>::value)
+        return 3;
+    else if constexpr (std::is_same<Epi, SkSwiGLU>::value)
+        return 4;
+    else
+        return 5;
+}
+
+// Timeline events of the skinny GEMM (timeline builds): 0 entry, 1 after the
+// dependency wait, 2 after the prologue's grid barrier, 3 first MMA issued,
+// 4 last MMA issued, 5 last epilogue chunk done, 7 exit.
 template <int NT, class Epi, class Pro>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -321,6 +344,8 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int k_iters = K / SK_BK;
     const int kps = (k_iters + splits - 1) / splits;        // k iterations per split
+    constexpr int tlk = sk_tl_kind<Epi, Pro>();
+    if (threadIdx.x == 0) FDL_TL(tlk, 0);
     if (threadIdx.x == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
             mbar_init(full_bar(s), 1);
@@ -360,11 +385,13 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
     }
     pdl_wait();
+    if (threadIdx.x == 0) FDL_TL(tlk, 1);
     if constexpr (Pro::kActive) {
         pro.work(blockIdx.x, gridDim.x);
         fence_proxy_async_global();                 // the TMA below reads what was written
         grid_barrier(pro.bar, abort_flag, err);
     }
+    if (threadIdx.x == 0) FDL_TL(tlk, 2);
     pdl_trigger();
 
     if (warp == 0) {
@@ -399,11 +426,10 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 // now, so that its barrier phase completes
                 for (int j = n; j < npre; ++j)
                     tma_load_3d(sB(j), &tmX, full_bar(j), 0, 0, pre_k[j] * 2);
-                volatile int no_abort = 0;
                 const int issued = n > npre ? n : npre;
                 for (int s = 0; s < S::STAGES && s < issued; ++s) {
                     const int j = s + ((issued - 1 - s) / S::STAGES) * S::STAGES;
-                    mbar_wait(full_bar(s), (uint32_t)((j / S::STAGES) & 1), &no_abort, err);
+                    mbar_wait_drain(full_bar(s), (uint32_t)((j / S::STAGES) & 1), err);
                 }
             }
         }
@@ -432,11 +458,13 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                         umma_bf16(d_tmem, a0 + (uint64_t)((kk & 3) * 2), b0 + (uint64_t)((kk & 3) * 2),
                                   idesc, (k > k0 || kk > 0) ? 1u : 0u);
                     }
+                    if (it == 0 && k == k0) FDL_TL(tlk, 3);
                     umma_commit(empty_bar(stage));
                     if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (ok) umma_commit(tfull_bar(acc));
             }
+            FDL_TL(tlk, 4);
         }
     } else {
         const int q = warp & 3;                     // TMEM lane quarter = 32 weight rows
@@ -460,6 +488,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             tc_fence_before();
             mbar_arrive(tempty_bar(acc));
         }
+        if (threadIdx.x == 64) FDL_TL(tlk, 5);
     }
     tc_fence_before();
     __syncthreads();
@@ -467,6 +496,7 @@ gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem_base, S::TMEM_COLS);
     }
+    if (threadIdx.x == 0) FDL_TL(tlk, 7);
 }
 
 template <int NT, class Epi, class Pro = NoPro>
@@ -656,3 +686,5 @@ cudaError_t launch_skinny_ffn(const GemmShape& g_gu, const void* x, const void* 
 }
 
 }  // namespace fdl
+
+FDL_TL_READER(fdl_timeline_skinny)

@@ -90,6 +90,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            int issued = 0;                              // loads requested (load u: stage u % STAGES)
             const uint64_t w_policy = l2_evict_first();
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x) {
                 const int m_tile = item % num_m, n_tile = item / num_m;
@@ -102,6 +103,7 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                          w_policy);
                     else
                         tma_load_2d(sB(stage), &tmB, full_bar(stage), k * BK, n_tile * BN);
+                    ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
@@ -111,6 +113,12 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 ok = mbar_wait(empty_bar(stage), phase ^ 1, abort_flag, err);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
+            if (!ok) {
+                // gave up: the loads still in flight (at most one per stage, the
+                // last STAGES requested) land before the CTA may leave
+                for (int u = issued > STAGES ? issued - STAGES : 0; u < issued; ++u)
+                    mbar_wait_drain(full_bar(u % STAGES), (uint32_t)((u / STAGES) & 1), err);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -119,6 +127,8 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0;
             bool ok = true;
             int it = 0;
+            int consumed = 0;                            // stages committed back (u: stage u % STAGES)
+            int tcommits = 0;                            // accumulators committed (i: acc i & 1)
             for (int item = blockIdx.x; ok && item < num_items; item += gridDim.x, ++it) {
                 const int acc = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
@@ -137,9 +147,24 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                   (k | kk) != 0);
                     }
                     umma_commit(empty_bar(stage));
+                    ++consumed;
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                if (ok) umma_commit(tfull_bar(acc));
+                if (ok) {
+                    umma_commit(tfull_bar(acc));
+                    ++tcommits;
+                }
+            }
+            if (!ok) {
+                // gave up: every MMA issued is followed by a commit on its stage's
+                // empty barrier (at most one outstanding per stage, the last
+                // STAGES) and each finished item by one on its accumulator's full
+                // barrier (at most the last two): once those arrivals have
+                // landed, no MMA writes TMEM and no arrival is on its way here
+                for (int u = consumed > STAGES ? consumed - STAGES : 0; u < consumed; ++u)
+                    mbar_wait_drain(empty_bar(u % STAGES), (uint32_t)((u / STAGES) & 1), err);
+                for (int i = tcommits > 2 ? tcommits - 2 : 0; i < tcommits; ++i)
+                    mbar_wait_drain(tfull_bar(i & 1), (uint32_t)((i >> 1) & 1), err);
             }
         }
     } else {

@@ -13,7 +13,20 @@ namespace sm100 {
 
 // A wait that has not completed after this long gives up and records
 // DEV_TIMEOUT; a correct launch of any kernel here finishes in milliseconds.
+// This is the default of the per-context limit of the progress waits (below)
+// and the fixed limit of the drain waits that follow a give-up.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+// The limit of the progress waits of a context: the 64-bit word 8 bytes after
+// the context's 4-byte device error word (set by fdl_create to kWaitTimeoutNs
+// and changed by fdl_set_wait_timeout). Read when a wait starts its clock.
+__device__ __forceinline__ uint64_t wait_limit_ns(const int* err) {
+    if (!err) return kWaitTimeoutNs;
+    // constant while a kernel runs (set with the device idle): read through the
+    // non-coherent cache, a hit in L1 after the first read on an SM
+    return __ldg(reinterpret_cast<const unsigned long long*>(
+        reinterpret_cast<const char*>(err) + 8));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -71,6 +84,7 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 struct PollBudget {
     uint32_t n = 0;
     uint64_t t0 = 0;
+    uint64_t limit = 0;
     __device__ __forceinline__ void reset() { n = 0; t0 = 0; }
     __device__ __forceinline__ bool idle(volatile int* abort, int* err) {
         if ((++n & 63u) != 0) return true;
@@ -78,7 +92,8 @@ struct PollBudget {
         const uint64_t now = globaltimer();
         if (t0 == 0) {
             t0 = now;
-        } else if (now - t0 > kWaitTimeoutNs) {
+            limit = wait_limit_ns(err);
+        } else if (now - t0 > limit) {
             *abort = 1;
             record_error(err, DEV_TIMEOUT);
             return false;
@@ -104,19 +119,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // time, or at once if another thread of the CTA has already given up.
 // The clock and the abort flag are consulted only every 64 polls, so a wait
 // that completes soon costs no more than the try_wait itself.
+// The clock starts at the first unsuccessful poll; with the default limit it
+// is read every 64 polls, with a limit under 1 ms (a shortened limit, set to
+// make waits run out) at every poll, so that a short wait can run out too.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           int* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    const uint64_t limit = wait_limit_ns(err);
+    const uint32_t every = limit < 1000000ull ? 0u : 63u;
+    uint32_t n = 0;
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((++n & every) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > limit) {
+                *abort = 1;
+                record_error(err, DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Wait of the give-up path: for an asynchronous operation this thread (or a
+// copy it requested) has already started and that completes by itself (a TMA
+// load landing, a tcgen05 commit arriving), so that nothing is still on its
+// way into the CTA's shared memory or TMEM when the CTA leaves. Ignores the
+// abort flag and has the fixed limit kWaitTimeoutNs (records DEV_TIMEOUT and
+// returns false if even that runs out).
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, int* err) {
     uint32_t n = 0;
     uint64_t t0 = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((++n & 63u) == 0) {
-            if (*abort) return false;
             const uint64_t now = globaltimer();
             if (t0 == 0) {
                 t0 = now;
             } else if (now - t0 > kWaitTimeoutNs) {
-                *abort = 1;
                 record_error(err, DEV_TIMEOUT);
                 return false;
             }
@@ -171,13 +212,14 @@ __device__ __forceinline__ bool grid_barrier(unsigned* bar, volatile int* abort,
             atom_add_release_gpu(cnt, first ? kBarrierQuantum - (nb - 1) : 1ull);
         const unsigned long long target = (old / kBarrierQuantum + 1) * kBarrierQuantum;
         uint32_t n = 0;
-        uint64_t t0 = 0;
+        uint64_t t0 = 0, limit = 0;
         while (ld_acquire_gpu(cnt) < target) {
             if ((++n & 63u) == 0) {
                 const uint64_t now = globaltimer();
                 if (t0 == 0) {
                     t0 = now;
-                } else if (now - t0 > kWaitTimeoutNs) {
+                    limit = wait_limit_ns(err);
+                } else if (now - t0 > limit) {
                     *abort = 1;
                     record_error(err, DEV_TIMEOUT);
                     break;

@@ -17,14 +17,17 @@ import os
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfdllm.so")
+# FDLLM_LIB may name another build of the library (the instrumented
+# libfdllm_timeline.so of `python -m block_kv_cache_b200.build --timeline`).
+LIB_PATH = os.environ.get("FDLLM_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                       "libfdllm.so")
 
 FDL_OK, FDL_EINVAL, FDL_EUNSUPPORTED, FDL_ECUDA, FDL_ETIMEOUT, FDL_EWORKSPACE, FDL_EDEVICE = (
     0, -1, -2, -3, -4, -5, -6)
 FDL_F32, FDL_BF16 = 0, 1
 
 EXPORTS = ("fdl_abi_version", "fdl_create", "fdl_destroy", "fdl_last_error",
-           "fdl_get_device_status", "fdl_attention_workspace_bytes",
+           "fdl_get_device_status", "fdl_set_wait_timeout", "fdl_attention_workspace_bytes",
            "fdl_dualcache_attention", "fdl_kv_store", "fdl_lmhead_workspace_bytes",
            "fdl_lmhead_confidence", "fdl_threshold_unmask",
            "fdl_lmhead_confidence_noalloc", "fdl_rope_table", "fdl_rmsnorm", "fdl_embed",
@@ -87,8 +90,8 @@ CACHE_MODES = {"dual": FDL_CACHE_DUAL, "prefix": FDL_CACHE_PREFIX, "none": FDL_C
 
 
 class GenerateOpts(ctypes.Structure):
-    _fields_ = [("cache", ctypes.c_int), ("bias_tok", ctypes.c_void_p),
-                ("bias_val", ctypes.c_void_p)]
+    _fields_ = [("cache", ctypes.c_int), ("device_loop", ctypes.c_int),
+                ("bias_tok", ctypes.c_void_p), ("bias_val", ctypes.c_void_p)]
 
 
 class FdlError(RuntimeError):
@@ -117,6 +120,7 @@ def load() -> ctypes.CDLL:
     L.fdl_destroy.argtypes = [vp]
     L.fdl_last_error.restype = ctypes.c_char_p
     L.fdl_get_device_status.argtypes = [vp, vp]
+    L.fdl_set_wait_timeout.argtypes = [vp, ctypes.c_uint64]
     L.fdl_attention_workspace_bytes.argtypes = [vp, ctypes.POINTER(AttnDesc)]
     L.fdl_attention_workspace_bytes.restype = sz
     L.fdl_dualcache_attention.argtypes = [vp, ctypes.POINTER(AttnDesc), vp, vp, vp, vp, vp,
@@ -261,6 +265,11 @@ class Context:
         if self._ws is None or self._ws.numel() < nbytes:
             self._ws = torch.empty(nbytes, dtype=torch.uint8, device=f"cuda:{self.device}")
         return self._ws
+
+    def set_wait_timeout(self, ns: int):
+        """Limit (ns) of the kernels' progress waits on this context
+        (fdl_set_wait_timeout)."""
+        _check(load().fdl_set_wait_timeout(self._h, int(ns)))
 
     def device_status(self, stream=None) -> int:
         """Synchronise and raise FdlError if a kernel recorded a device error."""
@@ -425,13 +434,16 @@ class Context:
         return out
 
     def generate(self, model: Model, prompt, gen_len, *, block=32, tau=0.9, cache="dual",
-                 bias_tok=None, bias_val=None, stream=None):
+                 bias_tok=None, bias_val=None, device_loop=False, stream=None):
         """The whole decode in the library (fdl_generate). prompt [b, P] int32,
         a CUDA tensor or a host tensor (then copied to the device first, and
         the result copied back to a host tensor: the public call with host
         buffers). cache: "dual", "prefix" or "none"; bias_tok / bias_val [b,
         gen_len] (CUDA, int32 / float32): optional planted logit bias of the
-        generated positions. Returns (x [b, P + gen_len] int32, steps)."""
+        generated positions. device_loop: the decode as one CUDA graph with the
+        steps sequenced on the device (kept in the context for the next call
+        with the same arguments; the workspace is kept by this Context so that
+        it does). Returns (x [b, P + gen_len] int32, steps)."""
         on_host = not prompt.is_cuda
         dev = torch.device("cuda", self.device)
         if on_host:
@@ -445,14 +457,18 @@ class Context:
         n = L.fdl_generate_workspace_bytes(self._h, model._h, b, P + gen_len, int(block))
         if n == 0:
             raise ValueError("generate: bad shape")
-        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        if getattr(self, "_gen_ws", None) is None or self._gen_ws.numel() < n:
+            self._gen_ws = None
+            self._gen_ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        ws = self._gen_ws
         x = torch.empty((b, P + gen_len), dtype=torch.int32, device=dev)
         steps = ctypes.c_int(0)
-        opts = GenerateOpts(CACHE_MODES[cache], None if bias_tok is None else bias_tok.data_ptr(),
+        opts = GenerateOpts(CACHE_MODES[cache], int(bool(device_loop)),
+                            None if bias_tok is None else bias_tok.data_ptr(),
                             None if bias_val is None else bias_val.data_ptr())
         _check(L.fdl_generate(self._h, model._h, _ptr(prompt), b, P, int(gen_len), int(block),
                               float(tau), ctypes.byref(opts), _ptr(x), ctypes.byref(steps),
-                              _ptr(ws), n, _stream(stream)))
+                              _ptr(ws), ws.numel(), _stream(stream)))
         if on_host:
             x = x.cpu()
         return x, steps.value

@@ -193,6 +193,59 @@ def run_ffn(a, ctx):
             "GBps": nbytes / us / 1e3, "TFLOPs": 6.0 * a.rows * a.n * a.k / us / 1e6}
 
 
+TL_EVENTS = {
+    "attention": ["entry", "after dependency wait + prologue", "first S MMA issued",
+                  "last PV committed", "first P tile written", "epilogue start",
+                  "split merge done", "exit"],
+    "skinny": ["entry", "after dependency wait", "after prologue barrier", "first MMA issued",
+               "last MMA issued", "last epilogue chunk", "-", "exit"],
+}
+TL_KINDS = {
+    "attention": ["DualCache (no prologue)", "DualCache with the q/k/v prologue",
+                  "full attention (two 128-row tiles)"],
+    "skinny": ["split-K sums with the RMSNorm prologue (q/k/v, gate/up)",
+               "down projection with the SwiGLU prologue", "residual (O projection)",
+               "split-K sums", "SwiGLU epilogue", "other"],
+}
+
+
+def timeline_summary():
+    """Per-CTA event clocks of the last launch of each kernel kind, read from
+    the instrumented library (FDLLM_LIB=.../libfdllm_timeline.so): for every
+    event, the median / min / max over CTAs of its time after the earliest
+    CTA entry of that launch (µs)."""
+    import ctypes
+    L = fdllm.load()
+    K, C, E = 8, 512, 8
+    out = {}
+    for name in ("attention", "skinny"):
+        fn = getattr(L, f"fdl_timeline_{name}", None)
+        if fn is None:
+            raise RuntimeError("not an instrumented library: set FDLLM_LIB to "
+                               "libfdllm_timeline.so")
+        buf = (ctypes.c_ulonglong * (K * C * E))()
+        if fn(buf) != 0:
+            raise RuntimeError("timeline read failed")
+        a = np.frombuffer(buf, dtype=np.uint64).reshape(K, C, E).astype(np.int64)
+        for k in range(K):
+            ctas = np.nonzero(a[k, :, 0])[0]
+            if len(ctas) == 0:
+                continue
+            t0 = a[k, ctas, 0].min()
+            ev = {}
+            for e in range(E):
+                v = a[k, ctas, e]
+                v = v[v > 0]
+                if len(v):
+                    d = (v - t0) / 1e3
+                    ev[TL_EVENTS[name][e]] = {"median": round(float(np.median(d)), 2),
+                                              "min": round(float(d.min()), 2),
+                                              "max": round(float(d.max()), 2), "ctas": int(len(v))}
+            kind = TL_KINDS[name][k] if k < len(TL_KINDS[name]) else str(k)
+            out[f"{name}: {kind}"] = ev
+    return out
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("op", choices=["lmhead", "attention", "full", "qkvattn", "swiglu", "resid",
@@ -214,6 +267,9 @@ def main():
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--graph", action="store_true", help="replay the timed calls as a CUDA graph")
     p.add_argument("--reps", type=int, default=5, help="graph replays timed (with --graph)")
+    p.add_argument("--timeline", action="store_true",
+                   help="also print the per-CTA event clocks of the last launch of each "
+                        "kernel kind (needs FDLLM_LIB=.../libfdllm_timeline.so)")
     a = p.parse_args()
     ctx = fdllm.Context(0)
     if a.op == "lmhead":
@@ -229,6 +285,8 @@ def main():
     else:
         r = run_linear(a, ctx)
     print(json.dumps(r), flush=True)
+    if a.timeline:
+        print(json.dumps({"timeline_us": timeline_summary()}), flush=True)
     ctx.close()
 
 

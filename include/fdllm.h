@@ -90,6 +90,18 @@ FDL_API const char* fdl_last_error(void);
  * FDL_OK, FDL_ETIMEOUT or FDL_EDEVICE accordingly. */
 FDL_API int fdl_get_device_status(fdl_ctx* ctx, void* stream);
 
+/* Limit, in ns, of the bounded waits with which the kernels launched on this
+ * context wait for progress (a TMA load, an MMA, another CTA, another
+ * warp's results); 2 s after fdl_create. A wait that runs out makes its CTA
+ * give up: it records FDL_ETIMEOUT in the device error word, waits (with the
+ * fixed 2 s limit) for the copies and tensor-core operations it has already
+ * started, frees its TMEM and returns, leaving the call's outputs undefined;
+ * the context must then be destroyed and created again. The library's own
+ * failure-detection test shortens the limit to make a wait run out on purpose.
+ * Synchronises the device; applies to kernels launched afterwards.
+ * ns in [1, 60e9]. Errors: FDL_EINVAL, FDL_ECUDA. */
+FDL_API int fdl_set_wait_timeout(fdl_ctx* ctx, uint64_t ns);
+
 /* ------------------------------------------------------------------------
  * (a) DualCache block attention
  * ------------------------------------------------------------------------ */
@@ -448,6 +460,16 @@ typedef enum {
 
 typedef struct {
     int cache;                /* fdl_cache_mode */
+    /* 0: the host runs the loop, reading the block's masked counts back after
+     * every step. 1: the whole decode is one CUDA graph: per block the refresh
+     * step, then a conditional WHILE node whose body is one cached step,
+     * repeated on the device while a sequence has a masked position left in
+     * the block (the condition is set by a small kernel after each step); the
+     * host synchronises once per decode. The executable graph is kept in the
+     * context and launched again by the next call with the same model,
+     * workspace, shapes, tau, cache mode and bias pointers; the first call
+     * captures and instantiates it. */
+    int device_loop;
     /* Optional planted logit bias per generated position (a synthetic workload
      * device: with random weights no confidence reaches a threshold, and a bias
      * on one token per position makes the parallel rule fire): at the LM head of
@@ -469,9 +491,11 @@ typedef struct {
  *   *steps_out (host) the decode steps taken (refresh steps included)
  *   ws      device workspace of fdl_generate_workspace_bytes bytes, 256-byte
  *           aligned
- * Every step reads `batch` 4-byte counters back to the host to decide
- * between the next cached step and the next block; the call returns when the
- * decode is complete (the stream is synchronised). The kernels and their
+ * With the host loop every step reads `batch` 4-byte counters back to decide
+ * between the next cached step and the next block; with opts->device_loop the
+ * steps are sequenced on the device. The call returns when the decode is
+ * complete (the stream is synchronised). prompt and out_x are only read at
+ * the start and written at the end (the decode state lives in ws). The kernels and their
  * order are those of the per-call functions above (fdl_embed, fdl_rmsnorm,
  * fdl_qkv_rope_store, fdl_full_attention, fdl_qkv_attention,
  * fdl_linear_residual, fdl_ffn, fdl_lmhead_confidence, fdl_threshold_unmask).

@@ -49,6 +49,7 @@ def test_null_arguments_rejected_without_device():
     assert L.fdl_generate(None, None, None, 1, 32, 32, 32, 0.9, None, None, None, None, 0,
                           None) == fdllm.FDL_EINVAL
     assert L.fdl_generate_workspace_bytes(None, None, 1, 64, 32) == 0
+    assert L.fdl_set_wait_timeout(None, 1000) == fdllm.FDL_EINVAL
     assert L.fdl_model_destroy(None) == fdllm.FDL_OK
     assert L.fdl_destroy(None) == fdllm.FDL_OK
 
