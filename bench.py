@@ -400,14 +400,15 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def planted_bias(torch, c, rank):
+def planted_bias(torch, c, rank, hi=16.0):
     """A planted logit bias per generated position (token drawn != mask id, value
-    ~ U(0, 16)): with random weights no confidence reaches tau, and this makes
-    the threshold rule fire, as a trained model's confident positions would."""
+    ~ U(0, hi); 16 is the LM-head workload's): with random weights no confidence
+    reaches tau, and this makes the threshold rule fire, as a trained model's
+    confident positions would."""
     from block_kv_cache_b200 import synth
     g = synth.rng(4242 + rank)
     bt = g.integers(0, c["mask_id"], (c["batch"], c["gen"])).astype(np.int32)
-    bv = g.uniform(0.0, 16.0, (c["batch"], c["gen"])).astype(np.float32)
+    bv = g.uniform(0.0, hi, (c["batch"], c["gen"])).astype(np.float32)
     return torch.from_numpy(bt).cuda(), torch.from_numpy(bv).cuda()
 
 
@@ -693,7 +694,10 @@ def run_reference(args):
 # position per step), +cache (DualCache, one position per step), +parallel
 # (no cache, threshold rule) and both. All with the planted logit bias, so
 # that the threshold rule fires as it would on a trained model's confident
-# positions; tau = 1 decodes exactly one position per step.
+# positions; tau = 1 decodes exactly one position per step. The bias is drawn
+# from U(0, 24): with the random LM head's logit spread about 7% of U(0, 16)
+# biases reach a confidence of 0.9, about 40% of U(0, 24) ones.
+SWEEP_BIAS_HI = 24.0
 SWEEP_GRID = (
     [dict(block=b, tau=0.9, gen=1024, cache="dual") for b in (8, 16, 32, 64, 128)]
     + [dict(block=32, tau=t, gen=1024, cache="dual") for t in (0.7, 1.0)]
@@ -717,7 +721,7 @@ def run_sweep(args):
     for pt in SWEEP_GRID:
         c = dict(base, **pt)
         L = c["prompt"] + c["gen"]
-        bias = planted_bias(torch, c, 0)
+        bias = planted_bias(torch, c, 0, SWEEP_BIAS_HI)
         dec = BlockDecoder(ctx, w, c["batch"], L, c["block"], cache=c["cache"],
                            bias_tok=bias[0], bias_val=bias[1])
         prompt = torch.from_numpy(synth.prompt_ids(7, c["batch"], c["prompt"],
@@ -741,7 +745,8 @@ def run_sweep(args):
         ctx.device_status()
         ms = e0.elapsed_time(e1)
         nsteps = sum(kinds.values())
-        print(json.dumps({"sweep": pt, "tokens": toks, "decode_steps": nsteps,
+        print(json.dumps({"sweep": pt, "bias_hi": SWEEP_BIAS_HI, "tokens": toks,
+                          "decode_steps": nsteps,
                           "tokens_per_step": toks / nsteps, "ms": ms,
                           "tokens_per_s": toks / (ms / 1e3), "steps_by_kind": kinds}),
               flush=True)

@@ -434,6 +434,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // so no empty wait). One tile only: a larger burst delays the loads of the
     // prologue that follows (measured).
     uint32_t early = 0;
+    if constexpr (!Pro::kActive) {
+        // the tensor maps are kernel parameters: fetch them while the
+        // preceding kernel finishes, so the first copies do not wait for them
+        if (warp == S::TMA_WARP && lane == 0) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
+    }
     if constexpr (Pro::kActive) {
         if (warp == S::TMA_WARP && lane == 0) {
             prefetch_tmap(&tmK);
@@ -469,7 +478,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             } else if (ok) {
                 q_issued = true;
                 const int head0 = g * grp + chunk * a.hc;
-                prefetch_tmap(&tmQ);
                 mbar_arrive_expect_tx(bar_q, (uint32_t)(S::DC * a.rows * 128));
                 for (int dc = 0; dc < S::DC; ++dc)
                     tma_load_3d(sb + S::OFF_Q + dc * S::Q_CHUNK, &tmQ, bar_q, dc * 64, head0,

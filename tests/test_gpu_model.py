@@ -364,12 +364,13 @@ def test_native_generate_cache_modes_equal_the_python_decoder(ctx, cache):
 # Two layers at the full widths of the two model families, so that a decode the
 # oracle replays runs the fused split-K calls (RMSNorm prologue, per-CTA query
 # tiles of the q/k/v epilogue, SwiGLU prologue behind grid barriers) and the
-# whole-vocabulary LM head. The LM head's weights are drawn with a wider
-# spread (logit std about 8) so that some confidences exceed tau and steps
-# decode several positions. Logits then carry an error of a few hundredths
-# from the bf16 activations of two layers (the 2e-2 confidence bound at
-# confidence ~0.5 allows ~0.04), so token ids are compared where the oracle's
-# top-2 gap exceeds 0.2, five times that.
+# whole-vocabulary LM head. The LM head has the LM-head workload's weight
+# distribution (W ~ N(0, 0.02)) and one planted logit bias ~ U(0, 24) per
+# generated position, so that confidences spread over (0, 1) and steps decode
+# several positions.
+# Logits carry an error of a few hundredths from the bf16 activations of two
+# layers (the 2e-2 confidence bound at confidence ~0.5 allows ~0.04), so token
+# ids are compared where the oracle's top-2 gap exceeds 0.2, five times that.
 WIDE_TOK_GAP = 0.2
 WIDE_MODELS = {
     # LLaDA-8B widths: MHA 32 x 128, FFN 12288, vocab 126464, mask id 126336
@@ -383,7 +384,7 @@ WIDE_MODELS = {
 
 @pytest.mark.parametrize("name", sorted(WIDE_MODELS))
 def test_two_layer_full_width_decode_matches_oracle(ctx, name):
-    """A 2-layer model at the full widths, prompt 64 + gen 64, block 32, tau
+    """A 2-layer model at the full widths, prompt 32 + gen 64, block 32, tau
     0.9: every step replayed by the oracle on the GPU's own trajectory
     (confidences within 2e-2, decisions bit-exact given the GPU's
     confidences) and, at every step, the LM-head boundary within 1e-5 on the
@@ -393,17 +394,27 @@ def test_two_layer_full_width_decode_matches_oracle(ctx, name):
     D = m["hidden"]
     P = synth.model_params(vocab=m["vocab"], hidden=D, n_layers=2, n_q_heads=m["n_q_heads"],
                            n_kv_heads=m["n_kv_heads"], head_dim=128, ffn=m["ffn"], seed=71,
-                           dtype="bf16", qkv_bias=m["qkv_bias"], lm_std=8.0 / np.sqrt(D))
+                           dtype="bf16", qkv_bias=m["qkv_bias"], lm_std=0.02)
     P.mask_id = m["mask_id"]
     w = DeviceWeights.from_params(P)
-    b, Lp, gen, B, tau = m["batch"], 64, 64, 32, 0.9
-    dec = BlockDecoder(ctx, w, b, Lp + gen, B)
+    # the oracle widens its operands to float64 at every use; widen the layer
+    # and LM-head weights once here instead (the same values)
+    for Lw in P.layers:
+        for k in list(Lw):
+            Lw[k] = Lw[k].astype(np.float64)
+    P.lm_head = P.lm_head.astype(np.float64)
+    b, Lp, gen, B, tau = m["batch"], 32, 64, 32, 0.9
+    g = synth.rng(73)
+    bt = g.integers(0, P.mask_id, (b, gen)).astype(np.int32)
+    bv = g.uniform(0.0, 24.0, (b, gen)).astype(np.float32)
+    dec = BlockDecoder(ctx, w, b, Lp + gen, B, bias_tok=torch.from_numpy(bt).cuda(),
+                       bias_val=torch.from_numpy(bv).cuda())
     prompt = synth.prompt_ids(72, b, Lp, P.mask_id)
     rec = []
     x, steps = dec.generate(prompt, gen, tau=tau, record=rec)
     ctx.device_status()
     assert steps == len(rec) and steps < gen          # some steps decoded several positions
-    _replay_check(P, rec, x.cpu().numpy(), B, tau, tok_gap=WIDE_TOK_GAP)
+    _replay_check(P, rec, x.cpu().numpy(), B, tau, tok_gap=WIDE_TOK_GAP, bias=(bt, bv, Lp))
 
 
 @pytest.mark.parametrize("seed,tau,hq,hkv,bias", [(0, 0.9, 2, 2, False), (1, 0.5, 4, 2, True),
