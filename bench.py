@@ -85,6 +85,8 @@ def parse():
     p.add_argument("--planted-bias", action="store_true",
                    help="a planted logit bias per generated position, so that the "
                         "threshold rule decodes several positions per step")
+    p.add_argument("--bias-hi", type=float, default=16.0,
+                   help="upper end of the planted bias U(0, hi) (default 16)")
     p.add_argument("--block", type=int, default=None, help="block size (default 32)")
     p.add_argument("--gen", type=int, default=None, help="generated length (default 1024)")
     p.add_argument("--tau", type=float, default=None, help="threshold (default 0.9)")
@@ -93,6 +95,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-loop", choices=["device", "host"], default="device",
                    help="fdl_generate's loop for the e2e decode")
+    p.add_argument("--compact", action="store_true",
+                   help="e2e decode with the host loop and compacted cached steps (only the "
+                        "sequences with masked positions left in the block)")
     p.add_argument("--sweep", action="store_true",
                    help="instead of the bench line: the block / tau / gen / cache-mode grid "
                         "with the planted bias, one JSON line per point")
@@ -322,7 +327,7 @@ def run_gpu(args):
     ctx = fdllm.Context(local)
     w = DeviceWeights.random(shape(), seed=1234)
     L = c["prompt"] + c["gen"]
-    bias = planted_bias(torch, c, rank) if args.planted_bias else (None, None)
+    bias = planted_bias(torch, c, rank, args.bias_hi) if args.planted_bias else (None, None)
     dec = BlockDecoder(ctx, w, c["batch"], L, c["block"], cache=args.cache, bias_tok=bias[0],
                        bias_val=bias[1])
     prompt = torch.from_numpy(synth.prompt_ids(7 + rank, c["batch"], c["prompt"],
@@ -496,6 +501,8 @@ def result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max, 
                    "batch": c["batch"], "prompt": c["prompt"], "gen": c["gen"],
                    "block": c["block"], "tau": c["tau"], "cache": args.cache,
                    "planted_bias": bool(args.planted_bias),
+                   **({"planted_bias_hi": args.bias_hi} if args.planted_bias else {}),
+                   **({"compact": True} if args.compact else {}),
                    "layers": c["layers"], "hidden": c["hidden"], "vocab": c["vocab"],
                    "parallelism": f"replicas x{world}",
                    "blocks_timed": blocks, "decode_steps_timed": nsteps,
@@ -529,11 +536,11 @@ def run_e2e(torch, ctx, w, c, args, rank):
     from block_kv_cache_b200 import synth
     hp = torch.from_numpy(synth.prompt_ids(7 + rank, c["batch"], c["prompt"],
                                            c["mask_id"])).pin_memory()
-    bias = planted_bias(torch, c, rank) if args.planted_bias else (None, None)
+    bias = planted_bias(torch, c, rank, args.bias_hi) if args.planted_bias else (None, None)
     m = w.native()
-    device_loop = args.e2e_loop == "device"
+    device_loop = args.e2e_loop == "device" and not args.compact
     kw = dict(block=c["block"], tau=c["tau"], cache=args.cache, bias_tok=bias[0],
-              bias_val=bias[1], device_loop=device_loop)
+              bias_val=bias[1], device_loop=device_loop, compact=args.compact)
     if device_loop:
         ctx.generate(m, hp, c["gen"], **kw)           # captures and keeps the decode graph
     torch.cuda.synchronize()
@@ -551,6 +558,7 @@ def run_e2e(torch, ctx, w, c, args, rank):
             "h2d": hp.numel() * 4 / blocks, "d2h": d2h / blocks,
             "path": f"fdl_generate (the library's decode loop, "
                     f"{'device loop: one CUDA graph per decode' if device_loop else 'host loop'}"
+                    f"{', compacted cached steps' if args.compact else ''}"
                     f") on a host prompt: {steps} decode steps, one whole decode of {blocks} "
                     f"blocks"}
 

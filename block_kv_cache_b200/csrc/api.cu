@@ -442,6 +442,12 @@ int check_qkv(const fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const vo
 }
 }  // namespace
 
+int qkv_attention_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h,
+                         const float* norm_w, float eps, void* x, const void* w,
+                         const float* bias, const float* rope, void* q_out, void* k_cache,
+                         void* v_cache, void* out, void* stream, const int32_t* seq_map,
+                         int kv_batch);
+
 extern "C" {
 
 int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
@@ -464,6 +470,20 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
 int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const float* norm_w,
                       float eps, void* x, const void* w, const float* bias, const float* rope,
                       void* q_out, void* k_cache, void* v_cache, void* out, void* stream) {
+    return qkv_attention_mapped(ctx, d, h, norm_w, eps, x, w, bias, rope, q_out, k_cache,
+                                v_cache, out, stream, nullptr, 0);
+}
+
+}  // extern "C"
+
+// fdl_qkv_attention over a compacted batch: the d->batch sequences of the rows
+// are sequences seq_map[0 .. d->batch) of caches that hold kv_batch sequences
+// (seq_map null: the identity, kv_batch = d->batch).
+int qkv_attention_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h,
+                         const float* norm_w, float eps, void* x, const void* w,
+                         const float* bias, const float* rope, void* q_out, void* k_cache,
+                         void* v_cache, void* out, void* stream, const int32_t* seq_map,
+                         int kv_batch) {
     int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
     if (rc) return rc;
     if (norm_w && (!h || !aligned16(h) || !aligned16(norm_w) || !(eps > 0.f)))
@@ -478,11 +498,16 @@ int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const
     DeviceGuard g(ctx->device);
     cudaStream_t st = (cudaStream_t)stream;
     const fdl::GemmShape gs{d->rows, (d->n_q_heads + 2 * d->n_kv_heads) * 128, d->hidden};
+    if (seq_map && kv_batch < d->batch)
+        return fail(FDL_EINVAL, "qkv_attention: the caches hold %d sequences, fewer than the "
+                    "%d of the batch", kv_batch, d->batch);
     const fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
                         (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
-                        d->rows_per_seq, d->pos0};
+                        d->rows_per_seq, d->pos0, seq_map};
     fdl::AttnShape as{d->batch, d->n_q_heads, d->n_kv_heads, 128, d->seq_len, d->pos0,
                       d->rows_per_seq, 1.0f / sqrtf(128.f), 1};
+    as.seq_map = seq_map;
+    as.kv_batch = seq_map ? kv_batch : 0;
     const fdl::NormIn ni{h, norm_w, eps};
     cudaError_t e;
     const int splits = fdl::skinny_ok(gs) ? fdl::skinny_qkv_splits(gs, ctx->acc_bytes,
@@ -508,6 +533,8 @@ int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const
     }
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv_attention launch");
 }
+
+extern "C" {
 
 int fdl_linear_residual(fdl_ctx* ctx, int rows, int out_features, int in_features,
                         const void* x, const void* w, float* h, void* stream) {
@@ -658,11 +685,40 @@ __global__ void tail_rows_kernel(int32_t* __restrict__ tail, int32_t* __restrict
     }
 }
 
+// A compacted DualCache step of the block at s: the sequences with masked
+// positions left in the block (remaining > 0), in order, become the batch;
+// seq_map[i] is the sequence of batch entry i, rows[i * B + j] the token row
+// of its block position j, and the block's planted bias rows are gathered to
+// match. One CTA; returns nothing (the host derives the same count from the
+// same counts).
+__global__ void compact_batch_kernel(const int32_t* __restrict__ remaining, int b, int L, int s,
+                                     int B, int32_t* __restrict__ seq_map,
+                                     int32_t* __restrict__ rows, const int32_t* __restrict__ btok,
+                                     const float* __restrict__ bval, int32_t* __restrict__ btok_c,
+                                     float* __restrict__ bval_c) {
+    __shared__ int n_act;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int i = 0; i < b; ++i)
+            if (remaining[i] > 0) seq_map[n++] = i;
+        n_act = n;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < n_act * B; e += blockDim.x) {
+        const int i = e / B, j = e % B, sq = seq_map[i];
+        rows[e] = sq * L + s + j;
+        if (btok) {
+            btok_c[e] = btok[sq * B + j];
+            bval_c[e] = bval[sq * B + j];
+        }
+    }
+}
+
 // Byte offsets of the generate workspace (256-byte aligned pieces).
 struct GenLayout {
     size_t kc, vc, h_full, x_full, q_full, o_full, f_full, h_blk, x_blk, q_blk, o_blk, f_blk,
         xn, conf, tok, masked, counts, maps, tail_map, tail_blk, bias_tok, bias_val, rope, lm_ws,
-        x, steps, total;
+        x, steps, seq_map, row_map_c, bias_tok_c, bias_val_c, total;
     size_t kv_layer;    // bytes of one layer's K (or V) cache
     size_t lm_bytes;
 };
@@ -706,6 +762,10 @@ GenLayout gen_layout(const fdl_model_desc& d, int b, int L, int B, size_t lm_byt
     g.lm_ws = take(lm_bytes);
     g.x = take(rf * 4);              // the decode's token ids (copied out at the end)
     g.steps = take(16);              // decode steps taken (device loop)
+    g.seq_map = take((size_t)b * 4); // compacted steps: the sequences still decoding,
+    g.row_map_c = take(rb * 4);      // ... their block rows among the token rows,
+    g.bias_tok_c = take(rb * 4);     // ... and their rows of the planted bias
+    g.bias_val_c = take(rb * 4);
     g.total = off;
     return g;
 }
@@ -755,8 +815,10 @@ struct GenRun {
     // every sequence. full: their K/V go into the caches and they attend over
     // the whole cache (refresh: pos0 = 0, n = L; PrefixCache step: pos0 = s,
     // n = L - s); otherwise the fused DualCache step of the block rows.
+    // With seq_map, a compacted DualCache step: the rows are those of nb
+    // sequences, batch entry i being sequence seq_map[i] of the caches.
     int layers(float* h, void* xb, void* q, void* o, void* f, int rows, bool full, int pos0,
-               int n, cudaStream_t st) const {
+               int n, cudaStream_t st, int nb = -1, const int32_t* seq_map = nullptr) const {
         const fdl_model_desc& d = m->d;
         const int D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads, hd = 128;
         void* stream = (void*)st;
@@ -766,7 +828,7 @@ struct GenRun {
             const fdl_layer_weights& W = m->layers[li];
             void* kl = base + g.kc + g.kv_layer * li;
             void* vl = base + g.vc + g.kv_layer * li;
-            const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, b, L, n, pos0, L};
+            const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, nb > 0 ? nb : b, L, n, pos0, L};
             if (full) {
                 const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
                 rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
@@ -774,14 +836,48 @@ struct GenRun {
                                                  stream);
                 if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
             } else {
-                rc = fdl_qkv_attention(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv, W.bias,
-                                       rope, q, kl, vl, o, stream);
+                rc = qkv_attention_mapped(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv,
+                                          W.bias, rope, q, kl, vl, o, stream, seq_map, b);
             }
             if (!rc) rc = fdl_linear_residual(ctx, rows, D, Hq * hd, o, W.wo, h, stream);
             if (!rc) rc = fdl_ffn(ctx, rows, D, F, W.ffn_norm, d.rms_eps, xb, W.w_gu, W.w_down, f,
                                   h, stream);
         }
         return rc;
+    }
+
+    // A cached DualCache step over only the n_act < b sequences that still
+    // have masked positions in the block (the others' rows would decode
+    // nothing): the same step on a compacted batch, whose rows read and write
+    // the caches, tokens and counts of the sequences they stand for.
+    int compact_step(int blk, int n_act, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        const int D = d.hidden, rc_rows = n_act * B, s = P + blk * B;
+        void* stream = (void*)st;
+        int32_t* smap = (int32_t*)at(g.seq_map);
+        int32_t* rows = (int32_t*)at(g.row_map_c);
+        compact_batch_kernel<<<1, 256, 0, st>>>(
+            remaining(), b, L, s, B, smap, rows, bias_tok ? (const int32_t*)at(g.bias_tok) : nullptr,
+            (const float*)at(g.bias_val), (int32_t*)at(g.bias_tok_c), (float*)at(g.bias_val_c));
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "generate: compaction");
+        float* h_blk = (float*)at(g.h_blk);
+        int rc = fdl_embed(ctx, rc_rows, D, x(), rows, m->embed, h_blk, stream);
+        if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), rc_rows,
+                             false, s, B, st, n_act, smap);
+        if (!rc) rc = fdl_rmsnorm(ctx, rc_rows, D, h_blk, nullptr, m->final_norm, d.rms_eps,
+                                  at(g.xn), stream);
+        const fdl_lmhead_desc lmd{rc_rows, D, d.vocab, FDL_BF16};
+        if (!rc) rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head,
+                                            bias_tok ? (const int32_t*)at(g.bias_tok_c) : nullptr,
+                                            bias_tok ? (const float*)at(g.bias_val_c) : nullptr,
+                                            (float*)at(g.conf), (int32_t*)at(g.tok), at(g.lm_ws),
+                                            g.lm_bytes, stream);
+        if (rc) return rc;
+        e = fdl::launch_threshold_unmask(n_act, L, s, B, tau, (const float*)at(g.conf),
+                                         (const int32_t*)at(g.tok), x(), masked(), remaining(),
+                                         remaining() + b, ctx->d_err, st, smap);
+        return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: unmask");
     }
 
     // One decode step of block blk: the forward (the refresh when `first` or
@@ -1028,12 +1124,15 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
     r.tau = tau;
     r.mode = opts ? opts->cache : FDL_CACHE_DUAL;
     const bool device_loop = opts && opts->device_loop;
+    const bool compact = opts && opts->compact;
     if (r.mode != FDL_CACHE_DUAL && r.mode != FDL_CACHE_PREFIX && r.mode != FDL_CACHE_NONE)
         return fail(FDL_EINVAL, "generate: unknown cache mode %d", r.mode);
     r.bias_tok = opts ? opts->bias_tok : nullptr;
     r.bias_val = opts ? opts->bias_val : nullptr;
     if ((r.bias_tok == nullptr) != (r.bias_val == nullptr))
         return fail(FDL_EINVAL, "generate: bias_tok and bias_val go together");
+    if (compact && (device_loop || r.mode != FDL_CACHE_DUAL))
+        return fail(FDL_EINVAL, "generate: compaction needs the DualCache mode and the host loop");
     const fdl_model_desc& d = m->d;
     r.L = P + gen;
     if (r.mode == FDL_CACHE_PREFIX && r.L % 32)
@@ -1088,17 +1187,19 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
         for (int blk = 0; blk < gen / B; ++blk) {
             int rc = r.block_prep(blk, st);
             if (rc) return rc;
+            int n_act = b;              // sequences with masked positions left in the block
             for (bool first = true;; first = false) {
-                rc = r.step(blk, first, st);
+                rc = !first && compact && n_act < b ? r.compact_step(blk, n_act, st)
+                                                    : r.step(blk, first, st);
                 if (rc) return rc;
                 ++steps;
                 e = cudaMemcpyAsync(host_rem.data(), r.remaining(), (size_t)b * 4,
                                     cudaMemcpyDeviceToHost, st);
                 if (e == cudaSuccess) e = cudaStreamSynchronize(st);
                 if (e != cudaSuccess) return cuda_fail(e, "generate: counters");
-                int rem = 0;
-                for (int i = 0; i < b; ++i) rem = host_rem[i] > rem ? host_rem[i] : rem;
-                if (rem == 0) break;
+                n_act = 0;
+                for (int i = 0; i < b; ++i) n_act += host_rem[i] > 0;
+                if (n_act == 0) break;
             }
         }
     }

@@ -164,6 +164,7 @@ struct AttnArgs {
     int push;           // splits push their partial rows to the owner's buffer
     float scale_log2;
     int* err;
+    const int32_t* seq_map;   // compacted batch: caches of sequence seq_map[bb], else bb
 };
 
 // ---- prologues: work every CTA does after the preceding kernel -----------------
@@ -198,6 +199,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
     constexpr int U = 2;
     const EpiQKV& p = pro.p;
     const int N = (p.n_q_heads + 2 * p.n_kv_heads) * 128;
+    const int kv_seq = p.cache_seq(bb);         // whose cache rows the block slot is
     for (int e0 = tid; e0 < n; e0 += U * nthreads) {
         float4 v[U][4], bs[U][4], cs[U][4];
 #pragma unroll
@@ -283,7 +285,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
             } else {
                 const int f = e - nq, kind = (f >> 3) & 1, pc = f & 7, row = kv0 + (f >> 4);
                 bf16* dst = (kind ? p.v_cache : p.k_cache) +
-                            (((size_t)bb * p.n_kv_heads + g) * p.seq_len + row) * 128 + pc * 8;
+                            (((size_t)kv_seq * p.n_kv_heads + g) * p.seq_len + row) * 128 + pc * 8;
                 *reinterpret_cast<uint4*>(dst) = w0;
                 *reinterpret_cast<uint4*>(dst + 64) = w1;
                 // only this thread reads these sums: zero them for the next call
@@ -409,7 +411,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (push) cluster_arrive();
     bool rcv_ready = !push;
     const uint32_t tmem = *tmem_slot;
-    const int krow0 = (bb / a.q_per_kv * a.Hkv + g) * a.L + k_begin;
+    const int kv_seq = a.seq_map ? __ldg(a.seq_map + bb) : bb / a.q_per_kv;
+    const int krow0 = (kv_seq * a.Hkv + g) * a.L + k_begin;
     const uint64_t kv_policy = l2_evict_first();
     // one copy per tile and operand: all D columns as DC sub-tiles
     auto load_k = [&](int t, int st) {
@@ -940,7 +943,8 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     const uint32_t qbox[3] = {64, (uint32_t)p.hc, (uint32_t)s.block_len};
     cudaError_t e = make_tmap_bf16(&tq, q, 3, qdims, qstr, qbox);
     if (e != cudaSuccess) return e;
-    const uint64_t kv_rows = (uint64_t)(s.batch / s.q_per_kv) * s.n_kv_heads * s.seq_len;
+    const uint64_t kv_rows =
+        (uint64_t)(s.kv_batch > 0 ? s.kv_batch : s.batch / s.q_per_kv) * s.n_kv_heads * s.seq_len;
     e = make_tmap_bf16_rows(&tk, k, kv_rows, D, ATT_KT, D / 64);
     if (e != cudaSuccess) return e;
     e = make_tmap_bf16_rows(&tv, v, kv_rows, D, ATT_KT, D / 64);
@@ -969,6 +973,7 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     }
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
+    a.seq_map = s.seq_map;
     const int hb = s.batch, hk = s.n_kv_heads;
     if (D == 128)
         return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, hb, hk, st, pro)

@@ -29,6 +29,12 @@ struct EpiQKV {              // N = (n_q_heads + 2 n_kv_heads) * 128
     int n_q_heads, n_kv_heads, seq_len;
     int rows_per_seq;        // row r belongs to sequence r / rows_per_seq ...
     int pos0;                // ... at position pos0 + r % rows_per_seq
+    // Compacted batch: the rows of sequence i write the cache rows of sequence
+    // seq_map[i] (null: of sequence i).
+    const int32_t* seq_map = nullptr;
+    __device__ __forceinline__ int cache_seq(int i) const {
+        return seq_map ? __ldg(seq_map + i) : i;
+    }
 };
 
 cudaError_t launch_gemm_resid(const GemmShape& g, const void* a, const void* w,

@@ -101,7 +101,7 @@ struct EpiQKVOp {
     __device__ void operator()(uint32_t tacc, int row, int M, int n0, int N) const {
         constexpr int D = 128;
         const int nq = p.n_q_heads * D, nk = p.n_kv_heads * D;
-        const int seq = row / p.rows_per_seq;
+        const int seq = row < M ? p.cache_seq(row / p.rows_per_seq) : 0;
         const int pos = p.pos0 + row % p.rows_per_seq;
 #pragma unroll 1
         for (int hc = 0; hc < BN; hc += D) {

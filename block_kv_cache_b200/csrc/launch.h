@@ -14,6 +14,11 @@ struct AttnShape {
     int bf16;     // 1: bf16 tensors (tcgen05 kernel), 0: f32 (SIMT kernel)
     int q_per_kv = 1;   // query blocks per sequence: batch counts query blocks,
                         // sequence index = batch index / q_per_kv (full attention)
+    // Compacted batch (q_per_kv == 1): query block i reads the caches of
+    // sequence seq_map[i], and the caches hold kv_batch sequences (null / 0:
+    // the identity and batch).
+    const int32_t* seq_map = nullptr;
+    int kv_batch = 0;
 };
 
 // Scratch for the split-KV partials of either attention kernel.
@@ -65,6 +70,7 @@ cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
                                     int block_len, float tau, const float* conf,
                                     const int32_t* tok, int32_t* x, uint8_t* masked,
                                     int32_t* remaining, int32_t* n_decoded,
-                                    int* dev_err, cudaStream_t st);
+                                    int* dev_err, cudaStream_t st,
+                                    const int32_t* seq_map = nullptr);
 
 }  // namespace fdl

@@ -6,7 +6,9 @@
 // candidate exceeds it, the single most confident candidate (lowest position
 // on ties) is decoded so that every step makes progress.
 //
-// One CTA per sequence, one thread per block position. The work is a few
+// One CTA per sequence, one thread per block position. With a compacted batch
+// (only the sequences that still have masked positions in the block), CTA i
+// reads row i of conf/tok and updates sequence seq_map[i]. The work is a few
 // compares per position, so the kernel is latency-bound; it reads B floats,
 // B ints and B bytes per sequence and writes at most B ints and B bytes.
 #include "common.cuh"
@@ -19,13 +21,15 @@ __global__ void __launch_bounds__(1024)
 threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restrict__ tok,
                         int32_t* __restrict__ x, uint8_t* __restrict__ masked,
                         int32_t* __restrict__ remaining, int32_t* __restrict__ n_decoded,
-                        int L, int s, int B, float tau, int* err) {
+                        int L, int s, int B, float tau, const int32_t* __restrict__ seq_map,
+                        int* err) {
     pdl_wait();
     pdl_trigger();
     __shared__ float s_val[32];
     __shared__ int s_idx[32];
     __shared__ int s_win;
-    const int b = blockIdx.x;
+    const int ci = blockIdx.x;                      // row of conf / tok
+    const int b = seq_map ? seq_map[ci] : ci;       // sequence updated
     const int j = threadIdx.x;
     const int lane = j & 31, warp = j >> 5, nwarps = blockDim.x >> 5;
 
@@ -33,7 +37,7 @@ threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restric
     float c = 0.f;
     if (j < B) {
         cand = masked[(size_t)b * L + s + j] != 0;
-        c = conf[(size_t)b * B + j];
+        c = conf[(size_t)ci * B + j];
     }
     const bool above = cand && (c > tau);          // NaN > tau is false
     const int any_above = __syncthreads_or(above);
@@ -64,7 +68,7 @@ threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restric
         sel = (j == s_win);
     }
     if (sel) {
-        x[(size_t)b * L + s + j] = tok[(size_t)b * B + j];
+        x[(size_t)b * L + s + j] = tok[(size_t)ci * B + j];
         masked[(size_t)b * L + s + j] = 0;
     }
     const int rem = __syncthreads_count(cand && !sel);
@@ -79,11 +83,11 @@ cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
                                     int block_len, float tau, const float* conf,
                                     const int32_t* tok, int32_t* x, uint8_t* masked,
                                     int32_t* remaining, int32_t* n_decoded,
-                                    int* dev_err, cudaStream_t st) {
+                                    int* dev_err, cudaStream_t st, const int32_t* seq_map) {
     int threads = ((block_len + 31) / 32) * 32;
     return launch_pdl(threshold_unmask_kernel, dim3(batch), dim3(threads), 0, st, 0, conf, tok, x,
                       masked, remaining, n_decoded, seq_len, block_start, block_len, tau,
-                      dev_err);
+                      seq_map, dev_err);
 }
 
 }  // namespace fdl

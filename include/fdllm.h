@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define FDL_ABI_VERSION 4
+#define FDL_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define FDL_API __attribute__((visibility("default")))
@@ -477,6 +477,14 @@ typedef struct {
      * of sequence i gets + bias_val[i, p - prompt_len]. */
     const int32_t* bias_tok;  /* [batch, gen_len] int32 device, entries in [0, V), or NULL */
     const float* bias_val;    /* [batch, gen_len] f32 device; required iff bias_tok */
+    /* 1 (FDL_CACHE_DUAL with the host loop only; else FDL_EINVAL): a cached
+     * step runs on the sequences that still have masked positions in the
+     * block, compacted into a smaller batch, instead of on all of them (the
+     * ones done with the block would decode nothing). Every sequence decodes
+     * the same tokens in the same steps as without compaction; the block's
+     * refresh still runs on the whole batch. 0: every step runs on the whole
+     * batch (lockstep). */
+    int compact;
 } fdl_generate_opts;
 
 /* Decode gen_len positions after the prompts of `batch` sequences.
@@ -487,7 +495,8 @@ typedef struct {
  *           (FDL_CACHE_PREFIX: prompt_len + gen_len and every block start also
  *           multiples of 32)
  *   tau     threshold in [0, 1] (tau = 1 decodes exactly one position per step)
- *   opts    cache mode and optional planted bias; NULL = FDL_CACHE_DUAL, no bias
+ *   opts    cache mode, loop, optional planted bias, compaction; NULL =
+ *           FDL_CACHE_DUAL, host loop, no bias, lockstep
  *   *steps_out (host) the decode steps taken (refresh steps included)
  *   ws      device workspace of fdl_generate_workspace_bytes bytes, 256-byte
  *           aligned

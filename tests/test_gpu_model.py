@@ -465,6 +465,80 @@ def test_native_device_loop_equals_host_loop(ctx, cache, bias):
         assert np.array_equal(x_d.cpu().numpy(), x_h.cpu().numpy())
 
 
+def _spread_bias(mask_id, b, gen, seed):
+    """Planted bias whose strength differs by sequence (sequence i gets
+    U(0, hi_i) with hi_i from 0 to 16), so that at tau < 1 the sequences of a
+    batch finish a block after different numbers of steps."""
+    g = synth.rng(seed)
+    hi = np.linspace(16.0, 0.0, b)[:, None]
+    tok = g.integers(0, mask_id, (b, gen)).astype(np.int32)
+    val = (g.uniform(0.0, 1.0, (b, gen)) * hi).astype(np.float32)
+    return torch.from_numpy(tok).cuda(), torch.from_numpy(val).cuda()
+
+
+@pytest.mark.parametrize("tau", [0.9, 0.5])
+def test_native_generate_compact_equals_lockstep(ctx, tau):
+    """fdl_generate with compaction (each cached step only on the sequences
+    that still have masked positions in the block) decodes the same tokens in
+    the same steps as the lockstep decode, on a batch whose sequences finish
+    their blocks after different numbers of steps (planted bias of a
+    different strength per sequence). At these shapes no projection splits K,
+    so both decodes are deterministic and the comparison is exact."""
+    from block_kv_cache_b200.model import DeviceWeights
+    P = _small_params(11, hq=4, hkv=2, bias=True)
+    w = DeviceWeights.from_params(P)
+    m = w.native()
+    b, Lp, gen, B = 5, 64, 96, 32
+    bias_tok, bias_val = _spread_bias(P.mask_id, b, gen, 71)
+    prompt = torch.from_numpy(synth.prompt_ids(12, b, Lp, P.mask_id)).cuda()
+    kw = dict(block=B, tau=tau, bias_tok=bias_tok, bias_val=bias_val)
+    x_l, s_l = ctx.generate(m, prompt, gen, **kw)
+    x_c, s_c = ctx.generate(m, prompt, gen, compact=True, **kw)
+    ctx.device_status()
+    assert s_c == s_l
+    assert np.array_equal(x_c.cpu().numpy(), x_l.cpu().numpy())
+    # the sequences did not finish in lockstep: compaction had work to skip
+    per_seq = [ctx.generate(m, prompt[i:i + 1].contiguous(), gen, block=B, tau=tau,
+                            bias_tok=bias_tok[i:i + 1].contiguous(),
+                            bias_val=bias_val[i:i + 1].contiguous())[1] for i in (0, b - 1)]
+    assert per_seq[0] < s_l and per_seq[1] <= s_l
+    # a single sequence decodes alone exactly as it does inside the batch
+    x_1, _ = ctx.generate(m, prompt[:1].contiguous(), gen, block=B, tau=tau,
+                          bias_tok=bias_tok[:1].contiguous(), bias_val=bias_val[:1].contiguous())
+    assert np.array_equal(x_1.cpu().numpy()[0], x_c.cpu().numpy()[0])
+
+
+def test_native_generate_compact_fused_shapes(ctx):
+    """Compaction on shapes that take the fused split-K calls (hidden 1024,
+    GQA 8/2 with bias; the compacted batch's sequence map reaches the split-K
+    q/k/v sums, the attention's block-slot writes and its cache reads): the
+    prompts are kept, every position is decoded, and the tokens agree with the
+    lockstep decode (exactly, unless the order of split-K atomic additions
+    tips a decision; at least 90 % of positions). Compaction is refused with
+    the device loop and outside the DualCache mode."""
+    from block_kv_cache_b200 import fdllm
+    from block_kv_cache_b200.model import DeviceWeights, ModelShape
+    sh = ModelShape(4096, 1024, 2, 8, 2, 1024, 4095, 128, qkv_bias=True)
+    w = DeviceWeights.random(sh, seed=6)
+    b, Lp, gen, B = 6, 64, 64, 32
+    prompt = torch.from_numpy(synth.prompt_ids(13, b, Lp, sh.mask_id)).cuda()
+    bias_tok, bias_val = _spread_bias(sh.mask_id, b, gen, 72)
+    bias_val = bias_val * 2.0
+    m = w.native()
+    kw = dict(block=B, tau=0.9, bias_tok=bias_tok, bias_val=bias_val)
+    x_l, s_l = ctx.generate(m, prompt, gen, **kw)
+    x_c, s_c = ctx.generate(m, prompt, gen, compact=True, **kw)
+    ctx.device_status()
+    xc, xl = x_c.cpu().numpy(), x_l.cpu().numpy()
+    assert np.array_equal(xc[:, :Lp], prompt.cpu().numpy())
+    assert (xc[:, Lp:] != sh.mask_id).all() and xc.min() >= 0 and xc.max() < sh.vocab
+    assert (xc[:, Lp:] == xl[:, Lp:]).mean() >= 0.9
+    assert s_c <= gen and s_l <= gen
+    for bad in (dict(compact=True, device_loop=True), dict(compact=True, cache="prefix")):
+        with pytest.raises(fdllm.FdlError):
+            ctx.generate(m, prompt, gen, **kw, **bad)
+
+
 def test_native_generate_fused_shapes(ctx):
     """fdl_generate on shapes that take the fused split-K calls (hidden 1024,
     GQA 8/2 with bias): the prompt is kept, every position is decoded, tau = 1
