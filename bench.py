@@ -445,8 +445,8 @@ def result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max, 
             ach, bound, unit = ffn_flops / ffn_avg / 1e6, "tensor", "TFLOP/s"
         # DRAM bytes read + written by the two kernels of one such call, from an
         # ncu capture of the same kernels at the LLaDA-8B shape (kernel_cases ffn
-        # --rows 32 --n 12288 --k 4096): 205.09 + 3.33 + 104.40 + 1.59 MB
-        traffic = (205_085_184 + 3_330_560 + 104_400_896 + 1_594_624
+        # --rows 32 --n 12288 --k 4096): 205.08 + 3.57 + 104.40 + 1.63 MB
+        traffic = (205_078_016 + 3_570_944 + 104_399_872 + 1_632_000
                    if (M, D, F) == (32, 4096, 12288) else None)
         roof = {"kernel": f"ffn call of layer 0 of a cached step (M={M}): RMSNorm, gate/up GEMM "
                           f"{2 * F}x{D}, SwiGLU, down GEMM {D}x{F} (with M <= 256 the RMSNorm "

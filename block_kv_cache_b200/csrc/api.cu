@@ -169,6 +169,7 @@ int fdl_create(fdl_ctx** out, int device) {
     if (e == cudaSuccess) e = cudaMalloc(&c->d_sync, kSyncBytes);
     if (e == cudaSuccess) e = cudaMemset(c->d_sync, 0, kSyncBytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) fdl::attn_tc_warm();   // host-side queries, no launch
     if (e != cudaSuccess) {
         if (c->d_err) cudaFree(c->d_err);
         if (c->d_acc) cudaFree(c->d_acc);

@@ -39,6 +39,8 @@
 //
 // Roofline: HBM. Algorithmic bytes per call = K and V once (2*b*Hkv*L*d*2)
 // + q and out (2*b*B*Hq*d*2).
+#include <atomic>
+
 #include "common.cuh"
 #include "gemm.h"
 #include "launch.h"
@@ -60,6 +62,15 @@ struct AttnPlan {
     int n_splits;  // cluster size
 };
 
+// At most `splits` splits of the key tiles (at least one tile each).
+void attn_set_splits(AttnPlan& p, int splits) {
+    if (splits > ATT_MAX_SPLITS) splits = ATT_MAX_SPLITS;
+    if (splits > p.tiles) splits = p.tiles;
+    if (splits < 1) splits = 1;
+    p.tps = (p.tiles + splits - 1) / splits;
+    p.n_splits = (p.tiles + p.tps - 1) / p.tps;
+}
+
 AttnPlan attn_tc_plan(const AttnShape& s, int sm_count) {
     AttnPlan p;
     const int grp = s.n_q_heads / s.n_kv_heads;
@@ -71,12 +82,7 @@ AttnPlan attn_tc_plan(const AttnShape& s, int sm_count) {
     p.mt = p.rows > 128 ? 2 : 1;
     p.tiles = (s.seq_len + ATT_KT - 1) / ATT_KT;
     const int units = s.batch * s.n_kv_heads * p.n_chunks;
-    int splits = sm_count / units;
-    if (splits < 1) splits = 1;
-    if (splits > ATT_MAX_SPLITS) splits = ATT_MAX_SPLITS;
-    if (splits > p.tiles) splits = p.tiles;
-    p.tps = (p.tiles + splits - 1) / splits;
-    p.n_splits = (p.tiles + p.tps - 1) / p.tps;
+    attn_set_splits(p, sm_count / units);
     return p;
 }
 
@@ -909,20 +915,91 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (threadIdx.x == 0) FDL_TL(tlk, 7);
 }
 
+// Clusters of s CTAs of this kernel that the GPU holds at once. A cluster
+// must fit in one GPC, so with one CTA per SM fewer clusters of 8 are resident
+// than 148 / 8 (measured: 16 clusters of 8 ran in two waves). Queried once per
+// cluster size, never while the stream is being captured (fdl_create warms the
+// values up); 0 while unknown.
 template <int D, int MT, class Pro>
-cudaError_t run_tc(const AttnPlan& p, const CUtensorMap& tq, const CUtensorMap& tk,
-                   const CUtensorMap& tv, const AttnArgs& a, int batch, int hkv,
+int cluster_capacity(int s, cudaStream_t st) {
+    using S = Att4<D, MT>;
+    static std::atomic<int> cap[ATT_MAX_SPLITS + 1];
+    if (s < 2 || s > ATT_MAX_SPLITS) return 0;
+    const int known = cap[s].load(std::memory_order_relaxed);
+    if (known > 0) return known;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    auto kfn = attn_tc_kernel<D, MT, Pro>;
+    if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::TOTAL) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s, 1, 1);
+    cfg.blockDim = dim3(S::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S::TOTAL;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = s;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cap[s].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+template <int D, int MT, class Pro>
+void warm_clusters() {
+    for (int s = 2; s <= ATT_MAX_SPLITS; ++s) (void)cluster_capacity<D, MT, Pro>(s, nullptr);
+}
+
+template <int D, int MT, class Pro>
+cudaError_t run_tc(AttnPlan p, const CUtensorMap& tq, const CUtensorMap& tk,
+                   const CUtensorMap& tv, AttnArgs a, int batch, int hkv,
                    cudaStream_t st, const Pro& pro) {
     using S = Att4<D, MT>;
     auto kfn = attn_tc_kernel<D, MT, Pro>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)S::TOTAL);
     if (e != cudaSuccess) return e;
+    // fewer splits while the grid's clusters would not all be resident at once
+    const int units = batch * hkv * p.n_chunks;
+    while (p.n_splits > 1) {
+        const int cap = cluster_capacity<D, MT, Pro>(p.n_splits, st);
+        if (cap <= 0 || units <= cap) break;
+        attn_set_splits(p, p.n_splits - 1);
+    }
+    a.tps = p.tps;
+    a.n_splits = p.n_splits;
+    // pushed merge when every split's rows for one owner fit its buffer
+    const int rpc = (p.rows + p.n_splits - 1) / p.n_splits;
+    a.push = MT == 1 && p.n_splits > 1 && p.n_splits * rpc * S::RCV_ROW <= S::RCV_BYTES ? 1 : 0;
     return launch_pdl(kfn, dim3(p.n_splits, hkv * p.n_chunks, batch), dim3(S::THREADS), S::TOTAL,
                       st, p.n_splits, tq, tk, tv, a, pro);
 }
 
 }  // namespace
+
+// The cluster capacities of every attention kernel, queried once per process
+// outside any stream capture (GPUs of one kind in a process).
+void attn_tc_warm() {
+    warm_clusters<128, 1, AttNoPro>();
+    warm_clusters<128, 2, AttNoPro>();
+    warm_clusters<64, 1, AttNoPro>();
+    warm_clusters<64, 2, AttNoPro>();
+    warm_clusters<128, 1, ProQKV>();
+    warm_clusters<128, 2, ProQKV>();
+}
 
 size_t attn_tc_workspace_bytes(const AttnShape&, int) {
     return 16;   // the splits merge on chip; no scratch is needed
@@ -965,12 +1042,7 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     a.q_per_kv = s.q_per_kv;
     a.blk0 = s.block_start;
     a.blk1 = s.block_start + s.block_len;
-    {
-        // pushed merge when every split's rows for one owner fit its buffer
-        const int rpc = (p.rows + p.n_splits - 1) / p.n_splits;
-        const int need = p.n_splits * rpc * (D + 4) * 4;
-        a.push = p.mt == 1 && p.n_splits > 1 && need <= Att4<128, 1>::RCV_BYTES ? 1 : 0;
-    }
+    a.push = 0;   // set by run_tc with the split count it launches
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
     a.seq_map = s.seq_map;

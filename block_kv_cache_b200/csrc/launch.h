@@ -21,6 +21,10 @@ struct AttnShape {
     int kv_batch = 0;
 };
 
+// Query the cluster capacities the attention launches use to size their split
+// count (once per process; call outside stream capture).
+void attn_tc_warm();
+
 // Scratch for the split-KV partials of either attention kernel.
 size_t attn_workspace_bytes(const AttnShape& s, int sm_count);
 size_t attn_tc_workspace_bytes(const AttnShape& s, int sm_count);
