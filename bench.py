@@ -95,9 +95,11 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-loop", choices=["device", "host"], default="device",
                    help="fdl_generate's loop for the e2e decode")
-    p.add_argument("--compact", action="store_true",
-                   help="e2e decode with the host loop and compacted cached steps (only the "
-                        "sequences with masked positions left in the block)")
+    p.add_argument("--batching", choices=["lockstep", "compact", "per_sequence"],
+                   default="lockstep",
+                   help="how the e2e decode moves a batch through its blocks (compact and "
+                        "per_sequence use the host loop): compacted cached steps, or every "
+                        "sequence at its own block")
     p.add_argument("--sweep", action="store_true",
                    help="instead of the bench line: the block / tau / gen / cache-mode grid "
                         "with the planted bias, one JSON line per point")
@@ -502,7 +504,7 @@ def result_line(args, c, world, w, dec, toks, toks_all, kinds, step_ms, ms_max, 
                    "block": c["block"], "tau": c["tau"], "cache": args.cache,
                    "planted_bias": bool(args.planted_bias),
                    **({"planted_bias_hi": args.bias_hi} if args.planted_bias else {}),
-                   **({"compact": True} if args.compact else {}),
+                   **({"batching": args.batching} if args.batching != "lockstep" else {}),
                    "layers": c["layers"], "hidden": c["hidden"], "vocab": c["vocab"],
                    "parallelism": f"replicas x{world}",
                    "blocks_timed": blocks, "decode_steps_timed": nsteps,
@@ -538,9 +540,9 @@ def run_e2e(torch, ctx, w, c, args, rank):
                                            c["mask_id"])).pin_memory()
     bias = planted_bias(torch, c, rank, args.bias_hi) if args.planted_bias else (None, None)
     m = w.native()
-    device_loop = args.e2e_loop == "device" and not args.compact
+    device_loop = args.e2e_loop == "device" and args.batching == "lockstep"
     kw = dict(block=c["block"], tau=c["tau"], cache=args.cache, bias_tok=bias[0],
-              bias_val=bias[1], device_loop=device_loop, compact=args.compact)
+              bias_val=bias[1], device_loop=device_loop, batching=args.batching)
     if device_loop:
         ctx.generate(m, hp, c["gen"], **kw)           # captures and keeps the decode graph
     torch.cuda.synchronize()
@@ -558,7 +560,7 @@ def run_e2e(torch, ctx, w, c, args, rank):
             "h2d": hp.numel() * 4 / blocks, "d2h": d2h / blocks,
             "path": f"fdl_generate (the library's decode loop, "
                     f"{'device loop: one CUDA graph per decode' if device_loop else 'host loop'}"
-                    f"{', compacted cached steps' if args.compact else ''}"
+                    f"{'' if args.batching == 'lockstep' else ', batching ' + args.batching}"
                     f") on a host prompt: {steps} decode steps, one whole decode of {blocks} "
                     f"blocks"}
 

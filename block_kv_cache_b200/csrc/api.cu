@@ -447,20 +447,37 @@ int qkv_attention_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h,
                          const float* norm_w, float eps, void* x, const void* w,
                          const float* bias, const float* rope, void* q_out, void* k_cache,
                          void* v_cache, void* out, void* stream, const int32_t* seq_map,
-                         int kv_batch);
+                         int kv_batch, const int32_t* pos0_map);
+int qkv_rope_store_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+                          const float* bias, const float* rope, void* q_out, void* k_cache,
+                          void* v_cache, void* stream, const int32_t* seq_map, int kv_batch);
 
 extern "C" {
 
 int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
                        const float* bias, const float* rope, void* q_out, void* k_cache,
                        void* v_cache, void* stream) {
+    return qkv_rope_store_mapped(ctx, d, x, w, bias, rope, q_out, k_cache, v_cache, stream,
+                                 nullptr, 0);
+}
+
+}  // extern "C"
+
+// fdl_qkv_rope_store with the rows of sequence i going to the caches of
+// sequence seq_map[i] of kv_batch (seq_map null: the identity).
+int qkv_rope_store_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const void* w,
+                          const float* bias, const float* rope, void* q_out, void* k_cache,
+                          void* v_cache, void* stream, const int32_t* seq_map, int kv_batch) {
     const int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
     if (rc) return rc;
+    if (seq_map && kv_batch < d->batch)
+        return fail(FDL_EINVAL, "qkv: the caches hold %d sequences, fewer than the %d of the "
+                    "batch", kv_batch, d->batch);
     DeviceGuard g(ctx->device);
     fdl::GemmShape gs{d->rows, (d->n_q_heads + 2 * d->n_kv_heads) * 128, d->hidden};
     fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
                   (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
-                  d->rows_per_seq, d->pos0};
+                  d->rows_per_seq, d->pos0, seq_map};
     cudaError_t e = fdl::skinny_ok(gs)
         ? fdl::launch_skinny_qkv(gs, x, w, p, ctx->d_acc, ctx->acc_bytes, ctx->sm_count,
                                  ctx->d_err, (cudaStream_t)stream)
@@ -468,23 +485,27 @@ int fdl_qkv_rope_store(fdl_ctx* ctx, const fdl_qkv_desc* d, const void* x, const
     return e == cudaSuccess ? FDL_OK : cuda_fail(e, "qkv launch");
 }
 
+extern "C" {
+
 int fdl_qkv_attention(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h, const float* norm_w,
                       float eps, void* x, const void* w, const float* bias, const float* rope,
                       void* q_out, void* k_cache, void* v_cache, void* out, void* stream) {
     return qkv_attention_mapped(ctx, d, h, norm_w, eps, x, w, bias, rope, q_out, k_cache,
-                                v_cache, out, stream, nullptr, 0);
+                                v_cache, out, stream, nullptr, 0, nullptr);
 }
 
 }  // extern "C"
 
 // fdl_qkv_attention over a compacted batch: the d->batch sequences of the rows
 // are sequences seq_map[0 .. d->batch) of caches that hold kv_batch sequences
-// (seq_map null: the identity, kv_batch = d->batch).
+// (seq_map null: the identity, kv_batch = d->batch); with pos0_map, sequence i's
+// block starts at pos0_map[i] instead of d->pos0 (the caller keeps every block
+// inside [0, seq_len)).
 int qkv_attention_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h,
                          const float* norm_w, float eps, void* x, const void* w,
                          const float* bias, const float* rope, void* q_out, void* k_cache,
                          void* v_cache, void* out, void* stream, const int32_t* seq_map,
-                         int kv_batch) {
+                         int kv_batch, const int32_t* pos0_map) {
     int rc = check_qkv(ctx, d, x, w, rope, q_out, k_cache, v_cache);
     if (rc) return rc;
     if (norm_w && (!h || !aligned16(h) || !aligned16(norm_w) || !(eps > 0.f)))
@@ -504,11 +525,12 @@ int qkv_attention_mapped(fdl_ctx* ctx, const fdl_qkv_desc* d, const float* h,
                     "%d of the batch", kv_batch, d->batch);
     const fdl::EpiQKV p{(fdl::bf16*)q_out, (fdl::bf16*)k_cache, (fdl::bf16*)v_cache, bias,
                         (const float2*)rope, d->n_q_heads, d->n_kv_heads, d->seq_len,
-                        d->rows_per_seq, d->pos0, seq_map};
+                        d->rows_per_seq, d->pos0, seq_map, pos0_map};
     fdl::AttnShape as{d->batch, d->n_q_heads, d->n_kv_heads, 128, d->seq_len, d->pos0,
                       d->rows_per_seq, 1.0f / sqrtf(128.f), 1};
     as.seq_map = seq_map;
     as.kv_batch = seq_map ? kv_batch : 0;
+    as.blk0_map = pos0_map;
     const fdl::NormIn ni{h, norm_w, eps};
     cudaError_t e;
     const int splits = fdl::skinny_ok(gs) ? fdl::skinny_qkv_splits(gs, ctx->acc_bytes,
@@ -715,11 +737,27 @@ __global__ void compact_batch_kernel(const int32_t* __restrict__ remaining, int 
     }
 }
 
+// The planted-bias rows of n sequences at their own blocks: row i * B + j is
+// position s_of[i] + j of sequence seq[i] (bias arrays [b, gen] from prompt_len
+// P on).
+__global__ void gather_bias_kernel(const int32_t* __restrict__ btok,
+                                   const float* __restrict__ bval, int gen, int P, int B,
+                                   const int32_t* __restrict__ seq,
+                                   const int32_t* __restrict__ s_of, int n,
+                                   int32_t* __restrict__ btok_c, float* __restrict__ bval_c) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n * B; e += gridDim.x * blockDim.x) {
+        const int i = e / B, j = e % B;
+        const size_t src = (size_t)seq[i] * gen + (s_of[i] - P) + j;
+        btok_c[e] = btok[src];
+        bval_c[e] = bval[src];
+    }
+}
+
 // Byte offsets of the generate workspace (256-byte aligned pieces).
 struct GenLayout {
     size_t kc, vc, h_full, x_full, q_full, o_full, f_full, h_blk, x_blk, q_blk, o_blk, f_blk,
         xn, conf, tok, masked, counts, maps, tail_map, tail_blk, bias_tok, bias_val, rope, lm_ws,
-        x, steps, seq_map, row_map_c, bias_tok_c, bias_val_c, total;
+        x, steps, seq_map, row_map_c, bias_tok_c, bias_val_c, ps_maps, total;
     size_t kv_layer;    // bytes of one layer's K (or V) cache
     size_t lm_bytes;
 };
@@ -767,6 +805,10 @@ GenLayout gen_layout(const fdl_model_desc& d, int b, int L, int B, size_t lm_byt
     g.row_map_c = take(rb * 4);      // ... their block rows among the token rows,
     g.bias_tok_c = take(rb * 4);     // ... and their rows of the planted bias
     g.bias_val_c = take(rb * 4);
+    // sequences at their own blocks: the maps of one step, written by the host
+    // (sequence ids, block starts, token rows of up to b whole sequences, and
+    // the block rows among them)
+    g.ps_maps = take(((size_t)2 * b + rf + rb) * 4);
     g.total = off;
     return g;
 }
@@ -816,10 +858,12 @@ struct GenRun {
     // every sequence. full: their K/V go into the caches and they attend over
     // the whole cache (refresh: pos0 = 0, n = L; PrefixCache step: pos0 = s,
     // n = L - s); otherwise the fused DualCache step of the block rows.
-    // With seq_map, a compacted DualCache step: the rows are those of nb
-    // sequences, batch entry i being sequence seq_map[i] of the caches.
+    // With seq_map, the rows are those of nb sequences, batch entry i being
+    // sequence seq_map[i] of the caches; with pos0_map (a DualCache step of
+    // sequences at their own blocks), entry i's block starts at pos0_map[i].
     int layers(float* h, void* xb, void* q, void* o, void* f, int rows, bool full, int pos0,
-               int n, cudaStream_t st, int nb = -1, const int32_t* seq_map = nullptr) const {
+               int n, cudaStream_t st, int nb = -1, const int32_t* seq_map = nullptr,
+               const int32_t* pos0_map = nullptr) const {
         const fdl_model_desc& d = m->d;
         const int D = d.hidden, F = d.ffn, Hq = d.n_q_heads, Hkv = d.n_kv_heads, hd = 128;
         void* stream = (void*)st;
@@ -831,14 +875,23 @@ struct GenRun {
             void* vl = base + g.vc + g.kv_layer * li;
             const fdl_qkv_desc qd{rows, D, Hq, Hkv, hd, nb > 0 ? nb : b, L, n, pos0, L};
             if (full) {
-                const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
                 rc = fdl_rmsnorm(ctx, rows, D, h, nullptr, W.attn_norm, d.rms_eps, xb, stream);
-                if (!rc) rc = fdl_qkv_rope_store(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl, vl,
-                                                 stream);
-                if (!rc) rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
+                if (!rc) rc = qkv_rope_store_mapped(ctx, &qd, xb, W.w_qkv, W.bias, rope, q, kl,
+                                                    vl, stream, seq_map, b);
+                if (!rc && !seq_map) {
+                    const fdl_attn_desc ad{b, Hq, Hkv, hd, L, pos0, n, FDL_BF16, 0.f};
+                    rc = fdl_full_attention(ctx, &ad, q, kl, vl, o, stream);
+                } else if (!rc) {
+                    // the whole-sequence forward of the nb sequences of seq_map
+                    const cudaError_t e = fdl::launch_full_attention_bf16(
+                        nb, Hq, Hkv, hd, L, n, 1.0f / sqrtf((float)hd), q, kl, vl, o,
+                        ctx->sm_count, ctx->d_err, st, seq_map, b);
+                    if (e != cudaSuccess) rc = cuda_fail(e, "generate: full attention");
+                }
             } else {
                 rc = qkv_attention_mapped(ctx, &qd, h, W.attn_norm, d.rms_eps, xb, W.w_qkv,
-                                          W.bias, rope, q, kl, vl, o, stream, seq_map, b);
+                                          W.bias, rope, q, kl, vl, o, stream, seq_map, b,
+                                          pos0_map);
             }
             if (!rc) rc = fdl_linear_residual(ctx, rows, D, Hq * hd, o, W.wo, h, stream);
             if (!rc) rc = fdl_ffn(ctx, rows, D, F, W.ffn_norm, d.rms_eps, xb, W.w_gu, W.w_down, f,
@@ -879,6 +932,72 @@ struct GenRun {
                                          (const int32_t*)at(g.tok), x(), masked(), remaining(),
                                          remaining() + b, ctx->d_err, st, smap);
         return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: unmask");
+    }
+
+    // Sequences at their own blocks. The host writes the step's maps into
+    // ps_maps: n sequence ids, their n block starts, then the token rows the
+    // step embeds, then (a refresh) the block rows among the forward's rows.
+    int32_t* ps_seq() const { return (int32_t*)at(g.ps_maps); }
+    int32_t* ps_start() const { return ps_seq() + b; }
+    int32_t* ps_rows() const { return ps_seq() + 2 * b; }
+    int32_t* ps_blk_rows() const { return ps_rows() + (size_t)b * L; }
+
+    // The step's maps to the device (stream-ordered; `host` may be reused once
+    // this returns) and the gather of the planted bias of the n sequences'
+    // blocks.
+    int ps_upload(const std::vector<int32_t>& host, int n, cudaStream_t st) const {
+        cudaError_t e = cudaMemcpyAsync(ps_seq(), host.data(), host.size() * 4,
+                                        cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess && bias_tok) {
+            gather_bias_kernel<<<32, 256, 0, st>>>(bias_tok, bias_val, gen, P, B, ps_seq(),
+                                                   ps_start(), n, (int32_t*)at(g.bias_tok_c),
+                                                   (float*)at(g.bias_val_c));
+            e = cudaGetLastError();
+        }
+        return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: step maps");
+    }
+
+    // LM head over the n sequences' block rows in xn, then the unmask of each
+    // at its own block.
+    int ps_decide(int n, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        const fdl_lmhead_desc lmd{n * B, d.hidden, d.vocab, FDL_BF16};
+        int rc = fdl_lmhead_confidence(ctx, &lmd, at(g.xn), m->lm_head,
+                                       bias_tok ? (const int32_t*)at(g.bias_tok_c) : nullptr,
+                                       bias_tok ? (const float*)at(g.bias_val_c) : nullptr,
+                                       (float*)at(g.conf), (int32_t*)at(g.tok), at(g.lm_ws),
+                                       g.lm_bytes, (void*)st);
+        if (rc) return rc;
+        const cudaError_t e = fdl::launch_threshold_unmask(
+            n, L, P, B, tau, (const float*)at(g.conf), (const int32_t*)at(g.tok), x(), masked(),
+            remaining(), remaining() + b, ctx->d_err, st, ps_seq(), ps_start());
+        return e == cudaSuccess ? FDL_OK : cuda_fail(e, "generate: unmask");
+    }
+
+    // The refresh of n sequences that have just moved to a new block: the full
+    // forward over all their positions (their caches rewritten), then the
+    // first step of their new blocks.
+    int ps_refresh(int n, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        float* h_full = (float*)at(g.h_full);
+        int rc = fdl_embed(ctx, n * L, d.hidden, x(), ps_rows(), m->embed, h_full, (void*)st);
+        if (!rc) rc = layers(h_full, at(g.x_full), at(g.q_full), at(g.o_full), at(g.f_full),
+                             n * L, true, 0, L, st, n, ps_seq());
+        if (!rc) rc = fdl_rmsnorm(ctx, n * B, d.hidden, h_full, ps_blk_rows(), m->final_norm,
+                                  d.rms_eps, at(g.xn), (void*)st);
+        return rc ? rc : ps_decide(n, st);
+    }
+
+    // A DualCache step of n sequences, each at its own block.
+    int ps_cached(int n, cudaStream_t st) const {
+        const fdl_model_desc& d = m->d;
+        float* h_blk = (float*)at(g.h_blk);
+        int rc = fdl_embed(ctx, n * B, d.hidden, x(), ps_rows(), m->embed, h_blk, (void*)st);
+        if (!rc) rc = layers(h_blk, at(g.x_blk), at(g.q_blk), at(g.o_blk), at(g.f_blk), n * B,
+                             false, P, B, st, n, ps_seq(), ps_start());
+        if (!rc) rc = fdl_rmsnorm(ctx, n * B, d.hidden, h_blk, nullptr, m->final_norm,
+                                  d.rms_eps, at(g.xn), (void*)st);
+        return rc ? rc : ps_decide(n, st);
     }
 
     // One decode step of block blk: the forward (the refresh when `first` or
@@ -1125,15 +1244,20 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
     r.tau = tau;
     r.mode = opts ? opts->cache : FDL_CACHE_DUAL;
     const bool device_loop = opts && opts->device_loop;
-    const bool compact = opts && opts->compact;
+    const int batching = opts ? opts->batching : FDL_BATCH_LOCKSTEP;
+    const bool compact = batching == FDL_BATCH_COMPACT;
+    const bool per_seq = batching == FDL_BATCH_PER_SEQUENCE;
+    if (batching != FDL_BATCH_LOCKSTEP && !compact && !per_seq)
+        return fail(FDL_EINVAL, "generate: unknown batching %d", batching);
     if (r.mode != FDL_CACHE_DUAL && r.mode != FDL_CACHE_PREFIX && r.mode != FDL_CACHE_NONE)
         return fail(FDL_EINVAL, "generate: unknown cache mode %d", r.mode);
     r.bias_tok = opts ? opts->bias_tok : nullptr;
     r.bias_val = opts ? opts->bias_val : nullptr;
     if ((r.bias_tok == nullptr) != (r.bias_val == nullptr))
         return fail(FDL_EINVAL, "generate: bias_tok and bias_val go together");
-    if (compact && (device_loop || r.mode != FDL_CACHE_DUAL))
-        return fail(FDL_EINVAL, "generate: compaction needs the DualCache mode and the host loop");
+    if ((compact || per_seq) && (device_loop || r.mode != FDL_CACHE_DUAL))
+        return fail(FDL_EINVAL, "generate: compacted or per-sequence batching needs the "
+                    "DualCache mode and the host loop");
     const fdl_model_desc& d = m->d;
     r.L = P + gen;
     if (r.mode == FDL_CACHE_PREFIX && r.L % 32)
@@ -1183,6 +1307,58 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) return cuda_fail(e, "generate: step count");
         steps = dev_steps;
+    } else if (per_seq) {
+        // Every sequence moves to its next block as soon as its own block is
+        // decoded: a step refreshes the sequences that have just moved on
+        // (their forward also decodes the first step of the new block) and
+        // takes one DualCache step of the others, each at its own block.
+        const int nblk_gen = gen / B;
+        std::vector<int32_t> host_rem(b), blk(b, 0), state(b, 0);   // 0 refresh, 1 cached, 2 done
+        std::vector<int32_t> up;
+        for (;;) {
+            int stepped = 0;
+            for (int kind = 0; kind < 2; ++kind) {
+                up.assign((size_t)2 * b, 0);
+                int n = 0;
+                for (int i = 0; i < b; ++i)
+                    if (state[i] == kind) {
+                        up[n] = i;
+                        up[b + n] = P + blk[i] * B;
+                        ++n;
+                    }
+                if (n == 0) continue;
+                // token rows embedded: every position (refresh) or the block's
+                for (int k = 0; k < n; ++k) {
+                    const int i = up[k], s = up[b + k];
+                    if (kind == 0)
+                        for (int j = 0; j < r.L; ++j) up.push_back(i * r.L + j);
+                    else
+                        for (int j = 0; j < B; ++j) up.push_back(i * r.L + s + j);
+                }
+                if (kind == 0) {   // the new blocks' rows among the forward's rows
+                    up.resize((size_t)2 * b + (size_t)b * r.L, 0);
+                    for (int k = 0; k < n; ++k)
+                        for (int j = 0; j < B; ++j) up.push_back(k * r.L + up[b + k] + j);
+                }
+                int rc = r.ps_upload(up, n, st);
+                if (!rc) rc = kind == 0 ? r.ps_refresh(n, st) : r.ps_cached(n, st);
+                if (rc) return rc;
+                stepped += n;
+            }
+            if (stepped == 0) break;
+            ++steps;
+            e = cudaMemcpyAsync(host_rem.data(), r.remaining(), (size_t)b * 4,
+                                cudaMemcpyDeviceToHost, st);
+            if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) return cuda_fail(e, "generate: counters");
+            for (int i = 0; i < b; ++i) {
+                if (state[i] == 2 || host_rem[i] > 0) {
+                    if (state[i] == 0) state[i] = 1;
+                    continue;
+                }
+                state[i] = ++blk[i] < nblk_gen ? 0 : 2;
+            }
+        }
     } else {
         std::vector<int32_t> host_rem(b);
         for (int blk = 0; blk < gen / B; ++blk) {

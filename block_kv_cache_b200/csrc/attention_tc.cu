@@ -60,6 +60,7 @@ struct AttnPlan {
     int tiles;     // 64-key tiles per (sequence, kv head)
     int tps;       // tiles per split
     int n_splits;  // cluster size
+    int units;     // (query block, kv head, chunk) units the split count is planned for
 };
 
 // At most `splits` splits of the key tiles (at least one tile each).
@@ -81,7 +82,12 @@ AttnPlan attn_tc_plan(const AttnShape& s, int sm_count) {
     p.rows = p.hc * s.block_len;
     p.mt = p.rows > 128 ? 2 : 1;
     p.tiles = (s.seq_len + ATT_KT - 1) / ATT_KT;
-    const int units = s.batch * s.n_kv_heads * p.n_chunks;
+    // A compacted batch (seq_map) is planned as the whole batch of kv_batch
+    // sequences, so that a sequence's splits, and with them the order of its
+    // sums, do not depend on which other sequences are in the launch.
+    const int blocks = s.kv_batch > 0 ? s.kv_batch * s.q_per_kv : s.batch;
+    const int units = blocks * s.n_kv_heads * p.n_chunks;
+    p.units = units;
     attn_set_splits(p, sm_count / units);
     return p;
 }
@@ -170,7 +176,8 @@ struct AttnArgs {
     int push;           // splits push their partial rows to the owner's buffer
     float scale_log2;
     int* err;
-    const int32_t* seq_map;   // compacted batch: caches of sequence seq_map[bb], else bb
+    const int32_t* seq_map;   // compacted batch: caches of sequence seq_map[bb / q_per_kv]
+    const int32_t* blk0_map;  // sequences at their own blocks: slot of bb at blk0_map[bb]
 };
 
 // ---- prologues: work every CTA does after the preceding kernel -----------------
@@ -206,6 +213,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
     const EpiQKV& p = pro.p;
     const int N = (p.n_q_heads + 2 * p.n_kv_heads) * 128;
     const int kv_seq = p.cache_seq(bb);         // whose cache rows the block slot is
+    const int blk0 = p.pos0_of(bb);             // where its block slot starts
     for (int e0 = tid; e0 < n; e0 += U * nthreads) {
         float4 v[U][4], bs[U][4], cs[U][4];
 #pragma unroll
@@ -222,7 +230,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
             } else {                             // k or v of a block-slot row
                 const int f = e - nq, kind = (f >> 3) & 1;
                 pc = f & 7;
-                i = kv0 + (f >> 4) - a.blk0;
+                i = kv0 + (f >> 4) - blk0;
                 col = (p.n_q_heads + kind * p.n_kv_heads + g) * 128;
                 rot = kind == 0;
             }
@@ -243,7 +251,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
             }
             if (rot) {
                 const float4* c4 = reinterpret_cast<const float4*>(
-                    p.rope + (size_t)(p.pos0 + i) * 64 + pc * 8);
+                    p.rope + (size_t)(blk0 + i) * 64 + pc * 8);
 #pragma unroll
                 for (int x = 0; x < 4; ++x) cs[u][x] = __ldg(c4 + x);
             } else {
@@ -295,7 +303,7 @@ __device__ __forceinline__ void qkv_items(const ProQKV& pro, const AttnArgs& a, 
                 *reinterpret_cast<uint4*>(dst) = w0;
                 *reinterpret_cast<uint4*>(dst + 64) = w1;
                 // only this thread reads these sums: zero them for the next call
-                float* src = pro.acc + (size_t)(bb * a.B + row - a.blk0) * N +
+                float* src = pro.acc + (size_t)(bb * a.B + row - blk0) * N +
                              (p.n_q_heads + kind * p.n_kv_heads + g) * 128 + pc * 8;
                 const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
                 __stcg(reinterpret_cast<float4*>(src), z);
@@ -371,15 +379,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int kv_w0 = live_warps < 4 * MT ? live_warps : 0;
     // Tile order: with the fused prologue the tiles holding block-slot rows of
     // this split come last (a rotation; the online softmax is order-free).
+    // this sequence's block slot [blk0, blk1)
+    const int blk0 = a.blk0_map ? __ldg(a.blk0_map + bb) : a.blk0, blk1 = blk0 + (a.blk1 - a.blk0);
     int rot = 0;
     if constexpr (Pro::kActive) {
-        if (a.blk0 < k_end && a.blk1 > k_begin)
-            rot = ((min(a.blk1, k_end) - 1 - k_begin) / KT + 1) % nt;
+        if (blk0 < k_end && blk1 > k_begin)
+            rot = ((min(blk1, k_end) - 1 - k_begin) / KT + 1) % nt;
     }
     auto tile_of = [&](int t) { const int u = t + rot; return u >= nt ? u - nt : u; };
     auto in_block = [&](int tile) {
         const int k0 = k_begin + tile * KT;
-        return k0 < a.blk1 && k0 + KT > a.blk0;
+        return k0 < blk1 && k0 + KT > blk0;
     };
     // split merge: split c owns packed rows [c * rpc, c * rpc + own)
     const int rpc = (a.rows + a.n_splits - 1) / a.n_splits;
@@ -417,7 +427,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (push) cluster_arrive();
     bool rcv_ready = !push;
     const uint32_t tmem = *tmem_slot;
-    const int kv_seq = a.seq_map ? __ldg(a.seq_map + bb) : bb / a.q_per_kv;
+    const int kv_seq = a.seq_map ? __ldg(a.seq_map + bb / a.q_per_kv) : bb / a.q_per_kv;
     const int krow0 = (kv_seq * a.Hkv + g) * a.L + k_begin;
     const uint64_t kv_policy = l2_evict_first();
     // one copy per tile and operand: all D columns as DC sub-tiles
@@ -629,7 +639,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         if constexpr (Pro::kActive) {
             if (warp >= kv_w0) {
                 // the block-slot K/V rows of this split's key range
-                const int kv0 = max(a.blk0, k_begin), kv1 = min(a.blk1, k_end);
+                const int kv0 = max(blk0, k_begin), kv1 = min(blk1, k_end);
                 qkv_items<S::Q_CHUNK>(pro, a, smem + S::OFF_Q, g, bb, kv0, 0,
                                       kv1 > kv0 ? (kv1 - kv0) * 16 : 0,
                                       threadIdx.x - kv_w0 * 32, (4 * MT - kv_w0) * 32, false);
@@ -973,10 +983,9 @@ cudaError_t run_tc(AttnPlan p, const CUtensorMap& tq, const CUtensorMap& tk,
                                          (int)S::TOTAL);
     if (e != cudaSuccess) return e;
     // fewer splits while the grid's clusters would not all be resident at once
-    const int units = batch * hkv * p.n_chunks;
     while (p.n_splits > 1) {
         const int cap = cluster_capacity<D, MT, Pro>(p.n_splits, st);
-        if (cap <= 0 || units <= cap) break;
+        if (cap <= 0 || p.units <= cap) break;
         attn_set_splits(p, p.n_splits - 1);
     }
     a.tps = p.tps;
@@ -1046,6 +1055,7 @@ cudaError_t launch_attn(const AttnShape& s, const void* q, const void* k, const 
     a.scale_log2 = s.scale * 1.4426950408889634f;
     a.err = err;
     a.seq_map = s.seq_map;
+    a.blk0_map = s.blk0_map;
     const int hb = s.batch, hk = s.n_kv_heads;
     if (D == 128)
         return p.mt == 2 ? run_tc<128, 2>(p, tq, tk, tv, a, hb, hk, st, pro)
@@ -1080,7 +1090,8 @@ cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQ
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
                                        int seq_len, int n_q, float scale, const void* q,
                                        const void* k, const void* v, void* out, int sm_count,
-                                       int* dev_err, cudaStream_t st) {
+                                       int* dev_err, cudaStream_t st, const int32_t* seq_map,
+                                       int kv_batch) {
     // The n_q query rows of a sequence (the last n_q positions; all of them at
     // a refresh) in query blocks of Bq rows: as many whole heads of a GQA group
     // per 256 rows. Each query block is one "sequence" of the attention kernel
@@ -1091,6 +1102,8 @@ cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads,
     if (n_q < 1 || n_q > seq_len || n_q % bq) return cudaErrorInvalidValue;
     AttnShape s{batch * (n_q / bq), n_q_heads, n_kv_heads, head_dim, seq_len, 0, bq, scale,
                 1, n_q / bq};
+    s.seq_map = seq_map;
+    s.kv_batch = seq_map ? kv_batch : 0;
     return launch_attention_bf16(s, q, k, v, out, nullptr, nullptr, sm_count, dev_err, st);
 }
 

@@ -32,8 +32,14 @@ struct EpiQKV {              // N = (n_q_heads + 2 n_kv_heads) * 128
     // Compacted batch: the rows of sequence i write the cache rows of sequence
     // seq_map[i] (null: of sequence i).
     const int32_t* seq_map = nullptr;
+    // Sequences at their own positions: sequence i's rows start at position
+    // pos0_map[i] (null: at pos0).
+    const int32_t* pos0_map = nullptr;
     __device__ __forceinline__ int cache_seq(int i) const {
         return seq_map ? __ldg(seq_map + i) : i;
+    }
+    __device__ __forceinline__ int pos0_of(int i) const {
+        return pos0_map ? __ldg(pos0_map + i) : pos0;
     }
 };
 

@@ -102,7 +102,7 @@ struct EpiQKVOp {
         constexpr int D = 128;
         const int nq = p.n_q_heads * D, nk = p.n_kv_heads * D;
         const int seq = row < M ? p.cache_seq(row / p.rows_per_seq) : 0;
-        const int pos = p.pos0 + row % p.rows_per_seq;
+        const int pos = (row < M ? p.pos0_of(row / p.rows_per_seq) : p.pos0) + row % p.rows_per_seq;
 #pragma unroll 1
         for (int hc = 0; hc < BN; hc += D) {
             const int col = n0 + hc;

@@ -137,14 +137,16 @@ struct SkQKV {
         for (int j = 0; j < 32; ++j) {
             const int t = j0 + j;
             cs[j] = rot && t < M
-                        ? __ldg(p.rope + (size_t)(p.pos0 + t % p.rows_per_seq) * (D / 2) + (r & 63))
+                        ? __ldg(p.rope + (size_t)(p.pos0_of(t / p.rows_per_seq) + t % p.rows_per_seq) *
+                                             (D / 2) + (r & 63))
                         : make_float2(1.f, 0.f);
         }
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             const int t = j0 + j;
             if (t >= M) break;
-            const int seq = p.cache_seq(t / p.rows_per_seq), pos = p.pos0 + t % p.rows_per_seq;
+            const int seq = p.cache_seq(t / p.rows_per_seq);
+            const int pos = p.pos0_of(t / p.rows_per_seq) + t % p.rows_per_seq;
             float y = v[j] + bias;
             if (rot) {
                 const float other = xs[(r ^ 64) * 33 + j] + pb;
@@ -581,7 +583,8 @@ __global__ void finish_qkv_kernel(float* __restrict__ acc, int M, EpiQKV p) {
     const int N = heads * D;
     float* row = acc + (size_t)t * N + h * D;
     float y = row[r] + (p.bias ? p.bias[h * D + r] : 0.f);
-    const int seq = p.cache_seq(t / p.rows_per_seq), pos = p.pos0 + t % p.rows_per_seq;
+    const int seq = p.cache_seq(t / p.rows_per_seq);
+            const int pos = p.pos0_of(t / p.rows_per_seq) + t % p.rows_per_seq;
     if (h < p.n_q_heads + p.n_kv_heads) {
         const float other = row[r ^ 64] + (p.bias ? p.bias[h * D + (r ^ 64)] : 0.f);
         const float2 cs = p.rope[(size_t)pos * (D / 2) + (r & 63)];

@@ -19,6 +19,9 @@ struct AttnShape {
     // the identity and batch).
     const int32_t* seq_map = nullptr;
     int kv_batch = 0;
+    // Sequences at their own blocks: query block i's block slot starts at
+    // blk0_map[i] (null: at block_start for all).
+    const int32_t* blk0_map = nullptr;
 };
 
 // Query the cluster capacities the attention launches use to size their split
@@ -50,10 +53,13 @@ cudaError_t launch_qkv_attention_bf16(const AttnShape& s, float* acc, const EpiQ
 // Full bidirectional attention of the last n_q positions of every sequence
 // over all seq_len positions (n_q = seq_len: the refresh forward; n_q = L - s:
 // a PrefixCache step): q, out [b, n_q, Hq, d] bf16; caches [b, Hkv, L, d].
+// With seq_map, sequence i of q/out is sequence seq_map[i] of caches that hold
+// kv_batch sequences.
 cudaError_t launch_full_attention_bf16(int batch, int n_q_heads, int n_kv_heads, int head_dim,
                                        int seq_len, int n_q, float scale, const void* q,
                                        const void* k, const void* v, void* out, int sm_count,
-                                       int* dev_err, cudaStream_t st);
+                                       int* dev_err, cudaStream_t st,
+                                       const int32_t* seq_map = nullptr, int kv_batch = 0);
 
 cudaError_t launch_kv_store(int batch, int n_kv_heads, int head_dim, int seq_len,
                             int elem_bytes, const void* k_new, const void* v_new,
@@ -75,6 +81,7 @@ cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
                                     const int32_t* tok, int32_t* x, uint8_t* masked,
                                     int32_t* remaining, int32_t* n_decoded,
                                     int* dev_err, cudaStream_t st,
-                                    const int32_t* seq_map = nullptr);
+                                    const int32_t* seq_map = nullptr,
+                                    const int32_t* s_map = nullptr);
 
 }  // namespace fdl

@@ -8,7 +8,8 @@
 //
 // One CTA per sequence, one thread per block position. With a compacted batch
 // (only the sequences that still have masked positions in the block), CTA i
-// reads row i of conf/tok and updates sequence seq_map[i]. The work is a few
+// reads row i of conf/tok and updates sequence seq_map[i]; with s_map, that
+// sequence's block starts at s_map[i] instead of block_start. The work is a few
 // compares per position, so the kernel is latency-bound; it reads B floats,
 // B ints and B bytes per sequence and writes at most B ints and B bytes.
 #include "common.cuh"
@@ -22,7 +23,7 @@ threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restric
                         int32_t* __restrict__ x, uint8_t* __restrict__ masked,
                         int32_t* __restrict__ remaining, int32_t* __restrict__ n_decoded,
                         int L, int s, int B, float tau, const int32_t* __restrict__ seq_map,
-                        int* err) {
+                        const int32_t* __restrict__ s_map, int* err) {
     pdl_wait();
     pdl_trigger();
     __shared__ float s_val[32];
@@ -30,6 +31,7 @@ threshold_unmask_kernel(const float* __restrict__ conf, const int32_t* __restric
     __shared__ int s_win;
     const int ci = blockIdx.x;                      // row of conf / tok
     const int b = seq_map ? seq_map[ci] : ci;       // sequence updated
+    if (s_map) s = s_map[ci];                       // its own block
     const int j = threadIdx.x;
     const int lane = j & 31, warp = j >> 5, nwarps = blockDim.x >> 5;
 
@@ -83,11 +85,12 @@ cudaError_t launch_threshold_unmask(int batch, int seq_len, int block_start,
                                     int block_len, float tau, const float* conf,
                                     const int32_t* tok, int32_t* x, uint8_t* masked,
                                     int32_t* remaining, int32_t* n_decoded,
-                                    int* dev_err, cudaStream_t st, const int32_t* seq_map) {
+                                    int* dev_err, cudaStream_t st, const int32_t* seq_map,
+                                    const int32_t* s_map) {
     int threads = ((block_len + 31) / 32) * 32;
     return launch_pdl(threshold_unmask_kernel, dim3(batch), dim3(threads), 0, st, 0, conf, tok, x,
                       masked, remaining, n_decoded, seq_len, block_start, block_len, tau,
-                      seq_map, dev_err);
+                      seq_map, s_map, dev_err);
 }
 
 }  // namespace fdl

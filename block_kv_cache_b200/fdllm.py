@@ -44,7 +44,7 @@ class AttnDesc(ctypes.Structure):
                 ("scale", ctypes.c_float)]
 
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 
 
 class LMHeadDesc(ctypes.Structure):
@@ -92,7 +92,10 @@ CACHE_MODES = {"dual": FDL_CACHE_DUAL, "prefix": FDL_CACHE_PREFIX, "none": FDL_C
 class GenerateOpts(ctypes.Structure):
     _fields_ = [("cache", ctypes.c_int), ("device_loop", ctypes.c_int),
                 ("bias_tok", ctypes.c_void_p), ("bias_val", ctypes.c_void_p),
-                ("compact", ctypes.c_int)]
+                ("batching", ctypes.c_int)]
+
+
+BATCHING = {"lockstep": 0, "compact": 1, "per_sequence": 2}
 
 
 class FdlError(RuntimeError):
@@ -435,7 +438,8 @@ class Context:
         return out
 
     def generate(self, model: Model, prompt, gen_len, *, block=32, tau=0.9, cache="dual",
-                 bias_tok=None, bias_val=None, device_loop=False, compact=False, stream=None):
+                 bias_tok=None, bias_val=None, device_loop=False, batching="lockstep",
+                 stream=None):
         """The whole decode in the library (fdl_generate). prompt [b, P] int32,
         a CUDA tensor or a host tensor (then copied to the device first, and
         the result copied back to a host tensor: the public call with host
@@ -444,9 +448,10 @@ class Context:
         generated positions. device_loop: the decode as one CUDA graph with the
         steps sequenced on the device (kept in the context for the next call
         with the same arguments; the workspace is kept by this Context so that
-        it does). compact (DualCache, host loop): cached steps run only on the
-        sequences with masked positions left in the block. Returns (x [b, P +
-        gen_len] int32, steps)."""
+        it does). batching (DualCache, host loop for the last two): "lockstep",
+        "compact" (cached steps only on the sequences with masked positions
+        left in the block) or "per_sequence" (each sequence moves to its next
+        block on its own). Returns (x [b, P + gen_len] int32, steps)."""
         on_host = not prompt.is_cuda
         dev = torch.device("cuda", self.device)
         if on_host:
@@ -469,7 +474,7 @@ class Context:
         opts = GenerateOpts(CACHE_MODES[cache], int(bool(device_loop)),
                             None if bias_tok is None else bias_tok.data_ptr(),
                             None if bias_val is None else bias_val.data_ptr(),
-                            int(bool(compact)))
+                            BATCHING[batching])
         _check(L.fdl_generate(self._h, model._h, _ptr(prompt), b, P, int(gen_len), int(block),
                               float(tau), ctypes.byref(opts), _ptr(x), ctypes.byref(steps),
                               _ptr(ws), ws.numel(), _stream(stream)))

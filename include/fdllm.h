@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define FDL_ABI_VERSION 5
+#define FDL_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define FDL_API __attribute__((visibility("default")))
@@ -458,6 +458,23 @@ typedef enum {
     FDL_CACHE_NONE = 2     /* no cache: every step is a full forward over all positions */
 } fdl_cache_mode;
 
+/* How the sequences of a batch move through their blocks. Every sequence
+ * decodes the same tokens in all three; they differ in what a step computes. */
+typedef enum {
+    FDL_BATCH_LOCKSTEP = 0,   /* every step runs on the whole batch; the batch moves to
+                                 the next block (one refresh for all) when every
+                                 sequence's block is decoded */
+    FDL_BATCH_COMPACT = 1,    /* as lockstep, but a cached step runs only on the sequences
+                                 that still have masked positions in the block, compacted
+                                 into a smaller batch */
+    FDL_BATCH_PER_SEQUENCE = 2 /* every sequence moves to its next block as soon as its own
+                                 block is decoded: a step refreshes the sequences that have
+                                 just moved on and takes a DualCache step of the others,
+                                 each at its own block; steps_out counts these steps */
+} fdl_batching;
+/* FDL_BATCH_COMPACT and FDL_BATCH_PER_SEQUENCE need FDL_CACHE_DUAL and the host
+ * loop (device_loop = 0); otherwise fdl_generate returns FDL_EINVAL. */
+
 typedef struct {
     int cache;                /* fdl_cache_mode */
     /* 0: the host runs the loop, reading the block's masked counts back after
@@ -477,14 +494,7 @@ typedef struct {
      * of sequence i gets + bias_val[i, p - prompt_len]. */
     const int32_t* bias_tok;  /* [batch, gen_len] int32 device, entries in [0, V), or NULL */
     const float* bias_val;    /* [batch, gen_len] f32 device; required iff bias_tok */
-    /* 1 (FDL_CACHE_DUAL with the host loop only; else FDL_EINVAL): a cached
-     * step runs on the sequences that still have masked positions in the
-     * block, compacted into a smaller batch, instead of on all of them (the
-     * ones done with the block would decode nothing). Every sequence decodes
-     * the same tokens in the same steps as without compaction; the block's
-     * refresh still runs on the whole batch. 0: every step runs on the whole
-     * batch (lockstep). */
-    int compact;
+    int batching;             /* fdl_batching */
 } fdl_generate_opts;
 
 /* Decode gen_len positions after the prompts of `batch` sequences.
@@ -495,8 +505,8 @@ typedef struct {
  *           (FDL_CACHE_PREFIX: prompt_len + gen_len and every block start also
  *           multiples of 32)
  *   tau     threshold in [0, 1] (tau = 1 decodes exactly one position per step)
- *   opts    cache mode, loop, optional planted bias, compaction; NULL =
- *           FDL_CACHE_DUAL, host loop, no bias, lockstep
+ *   opts    cache mode, loop, optional planted bias, batching; NULL =
+ *           FDL_CACHE_DUAL, host loop, no bias, FDL_BATCH_LOCKSTEP
  *   *steps_out (host) the decode steps taken (refresh steps included)
  *   ws      device workspace of fdl_generate_workspace_bytes bytes, 256-byte
  *           aligned

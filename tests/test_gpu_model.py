@@ -493,7 +493,7 @@ def test_native_generate_compact_equals_lockstep(ctx, tau):
     prompt = torch.from_numpy(synth.prompt_ids(12, b, Lp, P.mask_id)).cuda()
     kw = dict(block=B, tau=tau, bias_tok=bias_tok, bias_val=bias_val)
     x_l, s_l = ctx.generate(m, prompt, gen, **kw)
-    x_c, s_c = ctx.generate(m, prompt, gen, compact=True, **kw)
+    x_c, s_c = ctx.generate(m, prompt, gen, batching="compact", **kw)
     ctx.device_status()
     assert s_c == s_l
     assert np.array_equal(x_c.cpu().numpy(), x_l.cpu().numpy())
@@ -508,10 +508,46 @@ def test_native_generate_compact_equals_lockstep(ctx, tau):
     assert np.array_equal(x_1.cpu().numpy()[0], x_c.cpu().numpy()[0])
 
 
+@pytest.mark.parametrize("tau", [0.9, 0.5])
+def test_native_generate_per_sequence_blocks(ctx, tau):
+    """fdl_generate with every sequence moving to its next block as soon as
+    its own block is decoded (a step refreshes the sequences that have just
+    moved on, each at its own positions, and takes a DualCache step of the
+    others at their own blocks): bit for bit the tokens of the lockstep decode
+    (the attention plans its splits for the whole batch, so a sequence's sums
+    do not depend on which others share a launch), in no more steps; one
+    sequence alone decodes exactly as the lockstep decode of it alone."""
+    from block_kv_cache_b200.model import DeviceWeights
+    P = _small_params(11, hq=4, hkv=2, bias=True)
+    w = DeviceWeights.from_params(P)
+    m = w.native()
+    b, Lp, gen, B = 5, 64, 96, 32
+    bias_tok, bias_val = _spread_bias(P.mask_id, b, gen, 71)
+    prompt = torch.from_numpy(synth.prompt_ids(12, b, Lp, P.mask_id)).cuda()
+    kw = dict(block=B, tau=tau, bias_tok=bias_tok, bias_val=bias_val)
+    x_l, s_l = ctx.generate(m, prompt, gen, **kw)
+    x_p, s_p = ctx.generate(m, prompt, gen, batching="per_sequence", **kw)
+    ctx.device_status()
+    assert np.array_equal(x_p.cpu().numpy(), x_l.cpu().numpy())
+    assert s_p <= s_l
+    one = dict(block=B, tau=tau, bias_tok=bias_tok[:1].contiguous(),
+               bias_val=bias_val[:1].contiguous())
+    x_a, s_a = ctx.generate(m, prompt[:1].contiguous(), gen, **one)
+    x_1, s_1 = ctx.generate(m, prompt[:1].contiguous(), gen, batching="per_sequence", **one)
+    assert s_1 == s_a
+    assert np.array_equal(x_1.cpu().numpy(), x_a.cpu().numpy())
+    # no bias: every sequence decodes one position per step, in lockstep anyway
+    x_n, s_n = ctx.generate(m, prompt, gen, block=B, tau=1.0, batching="per_sequence")
+    assert s_n == gen
+    assert np.array_equal(x_n.cpu().numpy(), ctx.generate(m, prompt, gen, block=B, tau=1.0)[0]
+                          .cpu().numpy())
+
+
 def test_native_generate_compact_fused_shapes(ctx):
-    """Compaction on shapes that take the fused split-K calls (hidden 1024,
-    GQA 8/2 with bias; the compacted batch's sequence map reaches the split-K
-    q/k/v sums, the attention's block-slot writes and its cache reads): the
+    """Compaction and per-sequence blocks on shapes that take the fused
+    split-K calls (hidden 1024, GQA 8/2 with bias; the sequence map and the
+    per-sequence block starts reach the split-K q/k/v sums, the attention's
+    block-slot writes and its cache reads, and the refresh of a subset): the
     prompts are kept, every position is decoded, and the tokens agree with the
     lockstep decode (exactly, unless the order of split-K atomic additions
     tips a decision; at least 90 % of positions). Compaction is refused with
@@ -527,14 +563,17 @@ def test_native_generate_compact_fused_shapes(ctx):
     m = w.native()
     kw = dict(block=B, tau=0.9, bias_tok=bias_tok, bias_val=bias_val)
     x_l, s_l = ctx.generate(m, prompt, gen, **kw)
-    x_c, s_c = ctx.generate(m, prompt, gen, compact=True, **kw)
-    ctx.device_status()
-    xc, xl = x_c.cpu().numpy(), x_l.cpu().numpy()
-    assert np.array_equal(xc[:, :Lp], prompt.cpu().numpy())
-    assert (xc[:, Lp:] != sh.mask_id).all() and xc.min() >= 0 and xc.max() < sh.vocab
-    assert (xc[:, Lp:] == xl[:, Lp:]).mean() >= 0.9
-    assert s_c <= gen and s_l <= gen
-    for bad in (dict(compact=True, device_loop=True), dict(compact=True, cache="prefix")):
+    for batching in ("compact", "per_sequence"):
+        x_c, s_c = ctx.generate(m, prompt, gen, batching=batching, **kw)
+        ctx.device_status()
+        xc, xl = x_c.cpu().numpy(), x_l.cpu().numpy()
+        assert np.array_equal(xc[:, :Lp], prompt.cpu().numpy())
+        assert (xc[:, Lp:] != sh.mask_id).all() and xc.min() >= 0 and xc.max() < sh.vocab
+        assert (xc[:, Lp:] == xl[:, Lp:]).mean() >= 0.9
+        assert s_c <= gen and s_l <= gen
+    for bad in (dict(batching="compact", device_loop=True), dict(batching="compact", cache="prefix"),
+                dict(batching="per_sequence", device_loop=True),
+                dict(batching="per_sequence", cache="none")):
         with pytest.raises(fdllm.FdlError):
             ctx.generate(m, prompt, gen, **kw, **bad)
 
