@@ -71,3 +71,56 @@ def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(fdllm, "LIB_PATH", str(tmp_path / "libfdllm.so"))
     with pytest.raises(RuntimeError, match="not built"):
         fdllm.load()
+
+
+def _header():
+    return open(os.path.join(ROOT, "include", "fdllm.h")).read()
+
+
+def _typedef_body(src, kind, name):
+    end = re.search(r"\}\s*" + name + r"\s*;", src).start()
+    start = src.rindex("typedef " + kind + " {", 0, end)
+    return re.sub(r"/\*.*?\*/", "", src[start:end].split("{", 1)[1], flags=re.S)
+
+
+def _struct_fields(src, name):
+    body = _typedef_body(src, "struct", name)
+    return re.findall(r"([\w\s\*]+?)\s*\b(\w+);", body)
+
+
+def _enum(src, name):
+    body = _typedef_body(src, "enum", name)
+    return {k: int(v) for k, v in re.findall(r"(\w+)\s*=\s*(\d+)", body)}
+
+
+def test_binding_structs_match_the_header():
+    """The ctypes mirrors of the descriptor structs have the header's fields in
+    the header's order, with C types of the same size."""
+    src = _header()
+    sizes = {"int": 4, "float": 4, "int32_t": 4, "uint64_t": 8, "size_t": 8}
+    for cname, py in (("fdl_generate_opts", fdllm.GenerateOpts),
+                      ("fdl_attn_desc", fdllm.AttnDesc),
+                      ("fdl_lmhead_desc", fdllm.LMHeadDesc),
+                      ("fdl_unmask_desc", fdllm.UnmaskDesc),
+                      ("fdl_qkv_desc", fdllm.QKVDesc),
+                      ("fdl_model_desc", fdllm.ModelDesc),
+                      ("fdl_layer_weights", fdllm.LayerWeights),
+                      ("fdl_model_weights", fdllm.ModelWeights)):
+        fields = _struct_fields(src, cname)
+        assert [f for _, f in fields] == [f for f, _ in py._fields_], cname
+        for (ctype, fname), (_, pytype) in zip(fields, py._fields_):
+            ctype = ctype.replace("const", "").strip()
+            want = 8 if "*" in ctype else sizes[ctype]
+            assert ctypes.sizeof(pytype) == want, (cname, fname)
+
+
+def test_binding_enums_match_the_header():
+    src = _header()
+    batching = _enum(src, "fdl_batching")
+    assert batching == {"FDL_BATCH_LOCKSTEP": fdllm.BATCHING["lockstep"],
+                        "FDL_BATCH_COMPACT": fdllm.BATCHING["compact"],
+                        "FDL_BATCH_PER_SEQUENCE": fdllm.BATCHING["per_sequence"]}
+    cache = _enum(src, "fdl_cache_mode")
+    assert cache == {"FDL_CACHE_DUAL": fdllm.CACHE_MODES["dual"],
+                     "FDL_CACHE_PREFIX": fdllm.CACHE_MODES["prefix"],
+                     "FDL_CACHE_NONE": fdllm.CACHE_MODES["none"]}
