@@ -1260,9 +1260,11 @@ int fdl_generate(fdl_ctx* ctx, const fdl_model* m, const int32_t* prompt, int b,
                     "DualCache mode and the host loop");
     const fdl_model_desc& d = m->d;
     r.L = P + gen;
-    if (r.mode == FDL_CACHE_PREFIX && r.L % 32)
-        return fail(FDL_EINVAL, "generate: the PrefixCache mode needs prompt_len + gen_len and "
-                    "the block starts at multiples of 32");
+    if (r.L % 32)   // the refresh's full attention takes query blocks of 32 rows
+        return fail(FDL_EINVAL, "generate: prompt_len + gen_len must be a multiple of 32");
+    if (r.mode == FDL_CACHE_PREFIX && (P % 32 || B % 32))
+        return fail(FDL_EINVAL, "generate: the PrefixCache mode needs the block starts at "
+                    "multiples of 32 (prompt_len and block)");
     const int rf = b * r.L, rb = b * B;
     r.g = gen_layout(d, b, r.L, B, lm_ws_bytes(ctx, d, rb));
     if (!ws || ws_bytes < r.g.total)

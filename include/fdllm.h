@@ -501,9 +501,9 @@ typedef struct {
  *   prompt  [batch, prompt_len] int32 device (token ids)
  *   out_x   [batch, prompt_len + gen_len] int32 device (written: the prompts,
  *           then the decoded tokens)
- *   block   positions per block, 1..128; prompt_len and gen_len multiples of it
- *           (FDL_CACHE_PREFIX: prompt_len + gen_len and every block start also
- *           multiples of 32)
+ *   block   positions per block, 1..128; prompt_len and gen_len multiples of it,
+ *           prompt_len + gen_len a multiple of 32 (FDL_CACHE_PREFIX: prompt_len
+ *           and block too, so that every block starts at a multiple of 32)
  *   tau     threshold in [0, 1] (tau = 1 decodes exactly one position per step)
  *   opts    cache mode, loop, optional planted bias, batching; NULL =
  *           FDL_CACHE_DUAL, host loop, no bias, FDL_BATCH_LOCKSTEP

@@ -543,6 +543,35 @@ def test_native_generate_per_sequence_blocks(ctx, tau):
                           .cpu().numpy())
 
 
+@pytest.mark.parametrize("B,Lp,gen,tau", [(16, 48, 112, 0.9), (64, 64, 128, 0.7), (32, 32, 96, 0.0)])
+def test_native_generate_batchings_other_blocks(ctx, B, Lp, gen, tau):
+    """The three batchings on other block sizes and lengths (blocks of 16 and
+    64, whose attention takes the unfused calls; L = 160 ends in a partial key
+    tile; tau = 0 decodes a whole block per step): the same tokens bit for bit,
+    and with tau = 0 one step per block. A total length that is not a
+    multiple of 32 is refused before any work."""
+    from block_kv_cache_b200.model import DeviceWeights
+    P = _small_params(17, hq=2, hkv=2, bias=False)
+    w = DeviceWeights.from_params(P)
+    m = w.native()
+    b = 4
+    bias_tok, bias_val = _spread_bias(P.mask_id, b, gen, 73)
+    prompt = torch.from_numpy(synth.prompt_ids(18, b, Lp, P.mask_id)).cuda()
+    kw = dict(block=B, tau=tau, bias_tok=bias_tok, bias_val=bias_val)
+    x_l, s_l = ctx.generate(m, prompt, gen, **kw)
+    for batching in ("compact", "per_sequence"):
+        x_b, s_b = ctx.generate(m, prompt, gen, batching=batching, **kw)
+        ctx.device_status()
+        assert np.array_equal(x_b.cpu().numpy(), x_l.cpu().numpy()), batching
+        assert s_b <= s_l
+        if tau == 0.0:
+            assert s_b == s_l == gen // B
+    if B == 16:   # 48 + 112 - 16 = 144: not a multiple of 32
+        from block_kv_cache_b200 import fdllm
+        with pytest.raises(fdllm.FdlError):
+            ctx.generate(m, prompt, gen - B, block=B, tau=tau)
+
+
 def test_native_generate_compact_fused_shapes(ctx):
     """Compaction and per-sequence blocks on shapes that take the fused
     split-K calls (hidden 1024, GQA 8/2 with bias; the sequence map and the
