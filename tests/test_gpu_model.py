@@ -74,7 +74,10 @@ def test_embed_gather_exact(ctx):
 @pytest.mark.parametrize("M,N,K", [(32, 4096, 4096), (300, 512, 256), (1, 64, 64), (129, 320, 192),
                                    (32, 4096, 12288), (200, 1024, 512), (1, 128, 64),
                                    (64, 12288, 4096),
-                                   (300, 3584, 256), (1000, 3584, 512)])   # Dream widths
+                                   (300, 3584, 256), (1000, 3584, 512),    # Dream widths
+                                   # the 128-row GEMM at the refresh's and the Dream-shape
+                                   # cached step's sizes, and ragged rows
+                                   (1024, 3584, 3584), (2048, 4096, 4096), (1000, 1024, 1280)])
 def test_linear_residual(ctx, M, N, K):
     g = synth.rng(M + N)
     x = bf_vals(g.standard_normal((M, K)))
